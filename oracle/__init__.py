@@ -1,0 +1,7 @@
+"""fp64 CPU oracle for tile-sparse video attention. TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The product path (the CUDA library and
+its Python binding) never calls it and shares no code with it.
+"""
+from .vsa_oracle import *  # noqa: F401,F403

@@ -1,0 +1,369 @@
+"""Plain fp64 CPU oracle of one tile-sparse attention layer. TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import or call this module. It is slow on purpose: tiles are
+lists of token indices, every score and every softmax is evaluated in fp64 with
+numpy, and nothing is blocked, fused or reordered beyond what the method
+states. It shares no code with the CUDA library.
+
+What it computes, in the order the pages give it:
+
+1. Tiling.  Video tokens on the (T, H, W) latent grid are grouped into 3D
+   tiles of 64 tokens -- 4x4x4 for VSA (Ref2VA VSA README, "two-tier attention
+   layout"; "From 650 s to 72 s", "The method"), or one (pt, ph, pw) per head
+   with pt*ph*pw = 64 for head-aware tiling (BSAI VedaSparse README, "Core
+   Technology: Head-Aware Tiling"; "Implementation": ``_tile_3d`` returns the
+   tile and its key mask). The conditioning prefix (text, reference image,
+   reference audio) is split into segment-pure tiles that never mix two
+   segments (Ref2VA VSA news page, "Патч внимания с двумя уровнями", item 1).
+2. Scoring of every (video query tile, video key tile) pair, either by the
+   VSA gate on mean-pooled tiles (Ref2VA VSA README, gating projection
+   ``to_gate_compress``), or by TripPool: the Avg+Max+Min descriptor of each
+   tile with per-head Q/K projections (BSAI VedaSparse README, "Core
+   Technology: TripPool"; "Scorer Modes"; Veda news page, "Что делает Veda").
+3. Per head, each video query tile keeps its top-k video key tiles; prefix key
+   tiles are never pruned and prefix query rows stay dense (BSAI VedaSparse
+   README, "v3.4 Highlights": ``sink = exact_kv_and_rows``; Ref2VA README
+   items 1-2).
+4. Exact softmax attention over the kept tiles only (BSAI VedaSparse README,
+   "Core Technology: Tile-Skipping"; "Implementation": ``_veda_sparse``).
+
+Readings where the pages are silent (each also listed in the design doc):
+* VSA score: S[i, j] = (qbar_i G) . (kbar_j G) / sqrt(d), one d x d gate G per
+  layer shared by all heads; qbar/kbar are means over the tile's tokens.
+* TripPool score: S = (desc_q W_q[h]) . (desc_k W_k[h]) / sqrt(p), desc = [avg;
+  max; min] over the tile's tokens (3d wide), p the projection width.
+* The query side pools Q tiles, the key side pools K tiles.
+* k from a sparsity s over n tiles: n - floor(s*n + 0.5), clamped to [1, n].
+* Ties in top-k: equal scores keep the lower key-tile index; the kept list is
+  returned sorted ascending.
+* Prefix query rows attend to every token; no mask other than tile pruning.
+* A segment whose length is not a multiple of 64 ends in a partial tile; a
+  video tile cut by the grid edge is partial too. Partial tiles hold only their
+  valid tokens, in (t, h, w) raster order within the tile.
+* Softmax scale 1/sqrt(head_dim).
+"""
+from __future__ import annotations
+
+import dataclasses
+import itertools
+import math
+
+import numpy as np
+
+TILE = 64
+
+# ---------------------------------------------------------------------------
+# 1. tiling
+# ---------------------------------------------------------------------------
+
+
+def prefix_tiles(segments) -> list[np.ndarray]:
+    """Segment-pure prefix tiles: 64 consecutive tokens of one segment each.
+
+    Ref2VA VSA news page, "Патч внимания с двумя уровнями" item 1 (the geometry
+    mapper keeps text / reference-image / reference-audio tokens in tiles that
+    hold one segment only). The last tile of a segment may be partial.
+    """
+    tiles, base = [], 0
+    for length in segments:
+        for s0 in range(0, length, TILE):
+            tiles.append(np.arange(base + s0, base + min(length, s0 + TILE), dtype=np.int64))
+        base += length
+    return tiles
+
+
+def video_tiles(T: int, H: int, W: int, shape, n_prefix: int) -> list[np.ndarray]:
+    """3D video tiles of shape (pt, ph, pw) over the latent grid, in (ti, hi, wi) raster order.
+
+    Ref2VA VSA README, "two-tier attention layout" (4x4x4 spatial-temporal
+    tiles); BSAI VedaSparse README, "Core Technology: Head-Aware Tiling"
+    (per-head (pt, ph, pw), product 64). Tokens inside a tile are listed in
+    (t, h, w) raster order; tiles at the grid's far edge keep only the tokens
+    that exist.
+    """
+    pt, ph, pw = shape
+    tiles = []
+    for ti in range(-(-T // pt)):
+        t = np.arange(ti * pt, min(T, (ti + 1) * pt))
+        for hi in range(-(-H // ph)):
+            y = np.arange(hi * ph, min(H, (hi + 1) * ph))
+            for wi in range(-(-W // pw)):
+                x = np.arange(wi * pw, min(W, (wi + 1) * pw))
+                tok = (t[:, None, None] * H + y[None, :, None]) * W + x[None, None, :]
+                tiles.append(n_prefix + tok.ravel().astype(np.int64))
+    return tiles
+
+
+@dataclasses.dataclass
+class HeadTiling:
+    prefix: list          # list of token-index arrays
+    video: list           # list of token-index arrays
+
+    @property
+    def n_prefix(self) -> int:
+        return len(self.prefix)
+
+    @property
+    def n_video(self) -> int:
+        return len(self.video)
+
+    @property
+    def all(self) -> list:
+        return self.prefix + self.video
+
+
+def head_tiling(cfg, h: int) -> HeadTiling:
+    if np.prod(cfg.tile_shapes[h]) != TILE:
+        raise ValueError("tile shape must hold 64 tokens")
+    return HeadTiling(prefix_tiles(cfg.segments),
+                      video_tiles(cfg.T, cfg.H, cfg.W, cfg.tile_shapes[h], cfg.n_prefix_tokens))
+
+
+def pack(x: np.ndarray, cfg) -> tuple[np.ndarray, np.ndarray]:
+    """Token-major ``[B, N, heads, d]`` -> tile-major ``[B, heads, NT, 64, d]`` plus valid counts.
+
+    A pure permutation of rows: slot s of tile n holds token ``tiles[n][s]``;
+    slots past the tile's token count are zero. NT is the largest per-head tile
+    count; a head with fewer tiles leaves its trailing tiles empty (count 0).
+    """
+    B, N, Hh, d = x.shape
+    tilings = [head_tiling(cfg, h) for h in range(Hh)]
+    nt = max(len(t.all) for t in tilings)
+    out = np.zeros((B, Hh, nt, TILE, d), dtype=x.dtype)
+    counts = np.zeros((Hh, nt), dtype=np.int32)
+    for h, til in enumerate(tilings):
+        for n, tok in enumerate(til.all):
+            out[:, h, n, :len(tok)] = x[:, tok, h]
+            counts[h, n] = len(tok)
+    return out, counts
+
+
+def unpack(xp: np.ndarray, cfg) -> np.ndarray:
+    """Inverse of :func:`pack`: tile-major rows back to ``[B, N, heads, d]``."""
+    B, Hh = xp.shape[:2]
+    out = np.zeros((B, cfg.n_tokens, Hh, xp.shape[-1]), dtype=xp.dtype)
+    for h in range(Hh):
+        for n, tok in enumerate(head_tiling(cfg, h).all):
+            out[:, tok, h] = xp[:, h, n, :len(tok)]
+    return out
+
+
+# ---------------------------------------------------------------------------
+# 2. scoring
+# ---------------------------------------------------------------------------
+
+
+def k_from_sparsity(sparsity: float, n_tiles: int) -> int:
+    """Kept video key tiles per query tile at a given sparsity.
+
+    Sparsity is the pruned share of video key tiles (Ref2VA VSA README: "75%
+    video sparsity top-k"; BSAI README node table: keep_percent 5 = 95%
+    sparsity). k = n - round-half-up(s * n), clamped to [1, n].
+    """
+    k = n_tiles - math.floor(sparsity * n_tiles + 0.5)
+    return max(1, min(n_tiles, k))
+
+
+def mean_pool(x: np.ndarray) -> np.ndarray:
+    """Mean over a tile's tokens (rows)."""
+    return x.sum(axis=0) / x.shape[0]
+
+
+def tripool(x: np.ndarray) -> np.ndarray:
+    """TripPool descriptor of a tile: avg, max and min over its tokens, concatenated (3d).
+
+    BSAI VedaSparse README, "Core Technology" (Avg+Max+Min), "Implementation"
+    (``_tripool``, the paper's eq. 5).
+    """
+    return np.concatenate([mean_pool(x), x.max(axis=0), x.min(axis=0)])
+
+
+def tile_scores(q_h: np.ndarray, k_h: np.ndarray, til: HeadTiling, cfg, h: int,
+                gate=None, w_q=None, w_k=None) -> np.ndarray:
+    """Scores S[i, j] for video query tile i and video key tile j of head h (fp64).
+
+    ``q_h``/``k_h`` are the head's token rows ``[N, d]``. Prefix tiles are not
+    scored: they are never pruned.
+    """
+    if cfg.score_mode == "meanpool_gate":
+        g = np.asarray(gate, dtype=np.float64)
+        qd = np.stack([mean_pool(q_h[t]) for t in til.video]) @ g
+        kd = np.stack([mean_pool(k_h[t]) for t in til.video]) @ g
+        width = g.shape[1]
+    elif cfg.score_mode == "tripool":
+        wq = np.asarray(w_q[h], dtype=np.float64)
+        wk = np.asarray(w_k[h], dtype=np.float64)
+        qd = np.stack([tripool(q_h[t]) for t in til.video]) @ wq
+        kd = np.stack([tripool(k_h[t]) for t in til.video]) @ wk
+        width = wq.shape[1]
+    else:
+        raise ValueError(cfg.score_mode)
+    return (qd @ kd.T) / math.sqrt(width)
+
+
+# ---------------------------------------------------------------------------
+# 3. top-k selection
+# ---------------------------------------------------------------------------
+
+
+def topk_row(scores_row: np.ndarray, k: int) -> np.ndarray:
+    """The k best key tiles of one query tile: by score descending, lower index first on ties.
+
+    Veda news page, "Что делает Veda" (head-aware top-k forms the tile mask);
+    Ref2VA VSA README item 2 (top-k only over generated-video key tiles).
+    Returned sorted ascending.
+    """
+    j = np.arange(scores_row.shape[0])
+    order = np.lexsort((j, -scores_row))
+    return np.sort(order[:k])
+
+
+# ---------------------------------------------------------------------------
+# 4. attention
+# ---------------------------------------------------------------------------
+
+
+def softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    """Exact softmax attention of query rows over key rows, fp64.
+
+    Returns (out, lse, row_sum): lse is the natural-log sum of exp of the
+    scaled logits; row_sum is the sum of the normalised weights (1 up to
+    rounding).
+    """
+    x = scale * (q @ k.T)
+    m = x.max(axis=1, keepdims=True)
+    e = np.exp(x - m)
+    s = e.sum(axis=1, keepdims=True)
+    p = e / s
+    return p @ v, (m + np.log(s))[:, 0], p.sum(axis=1)
+
+
+def query_key_tokens(til: HeadTiling, tile_id: int, kept_video) -> np.ndarray:
+    """Key tokens that query tile ``tile_id`` (index into ``til.all``) attends to.
+
+    Prefix query tiles see every token (BSAI README "cond rows always dense";
+    Ref2VA README item 1). Video query tiles see every prefix tile plus their
+    kept video tiles (Ref2VA README items 1-2).
+    """
+    if tile_id < til.n_prefix:
+        return np.concatenate(til.all)
+    return np.concatenate(til.prefix + [til.video[j] for j in kept_video])
+
+
+@dataclasses.dataclass
+class LayerResult:
+    scores: list                 # per head [NTv_h, NTv_h] fp64
+    kept: list                   # per head [NTv_h, k_h] int64 (ascending)
+    out: np.ndarray              # [B, N, heads, d] fp64 (rows not computed are NaN)
+    lse: np.ndarray              # [B, N, heads] fp64
+    row_sum: np.ndarray          # [B, N, heads] fp64
+    computed_pairs: int          # sum over computed query rows of their key count
+
+
+def run_layer(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, k_per_head,
+              gate=None, w_q=None, w_k=None, query_tiles=None,
+              heads=None) -> LayerResult:
+    """The whole layer, in fp64: tile, score, select, attend.
+
+    ``q``, ``k``, ``v``: ``[B, N, heads, d]`` (any float dtype; widened to fp64).
+    ``query_tiles``: optional {head: iterable of tile ids into the head's tile
+    list (prefix first, then video)} restricting which query tiles get
+    attention rows; the others stay NaN. ``heads`` restricts the heads computed.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, N, Hh, d = q.shape
+    scale = 1.0 / math.sqrt(d)
+    heads = range(Hh) if heads is None else heads
+    out = np.full((B, N, Hh, d), np.nan)
+    lse = np.full((B, N, Hh), np.nan)
+    row_sum = np.full((B, N, Hh), np.nan)
+    all_scores, all_kept = [None] * Hh, [None] * Hh
+    pairs = 0
+    for h in heads:
+        til = head_tiling(cfg, h)
+        kh = int(k_per_head[h])
+        tiles_h = range(len(til.all)) if query_tiles is None else query_tiles.get(h, ())
+        for b in range(B):
+            s = tile_scores(q[b, :, h], k[b, :, h], til, cfg, h, gate, w_q, w_k)
+            kept = np.stack([topk_row(s[i], kh) for i in range(til.n_video)])
+            if b == 0:
+                all_scores[h], all_kept[h] = s, kept
+            for t in tiles_h:
+                qt = til.all[t]
+                kv = query_key_tokens(til, t, None if t < til.n_prefix else kept[t - til.n_prefix])
+                o, l, rs = softmax_attention(q[b, qt, h], k[b, kv, h], v[b, kv, h], scale)
+                out[b, qt, h], lse[b, qt, h], row_sum[b, qt, h] = o, l, rs
+                pairs += len(qt) * len(kv)
+    return LayerResult(all_scores, all_kept, out, lse, row_sum, pairs)
+
+
+# ---------------------------------------------------------------------------
+# independent checks used to pin the oracle
+# ---------------------------------------------------------------------------
+
+
+def dense_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
+    """Brute-force N x N softmax attention per (batch, head), no tiles at all."""
+    q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    B, N, Hh, d = q.shape
+    out = np.empty_like(q)
+    for b in range(B):
+        for h in range(Hh):
+            x = scale * (q[b, :, h] @ k[b, :, h].T)
+            x -= x.max(axis=1, keepdims=True)
+            p = np.exp(x)
+            p /= p.sum(axis=1, keepdims=True)
+            out[b, :, h] = p @ v[b, :, h]
+    return out
+
+
+def masked_dense_attention(q_h: np.ndarray, k_h: np.ndarray, v_h: np.ndarray,
+                           allowed: np.ndarray, scale: float) -> np.ndarray:
+    """N x N attention of one head with an explicit 0/-inf mask (``allowed`` is boolean N x N)."""
+    x = scale * (q_h @ k_h.T)
+    x = np.where(allowed, x, -np.inf)
+    x -= x.max(axis=1, keepdims=True)
+    p = np.exp(x)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ v_h
+
+
+def exhaustive_topk(scores_row: np.ndarray, k: int) -> np.ndarray:
+    """The k-subset with the largest score sum, ties broken toward lower indices.
+
+    Enumerates every subset, so only for tiny rows. Among subsets with equal
+    sums the lexicographically smallest sorted index tuple wins, which is the
+    lower-index tie rule.
+    """
+    best, best_sum = None, -np.inf
+    for sub in itertools.combinations(range(scores_row.shape[0]), k):
+        s = float(np.sum(scores_row[list(sub)]))
+        if s > best_sum:
+            best, best_sum = sub, s
+    return np.array(best, dtype=np.int64)
+
+
+def attention_flops(cfg, k_per_head) -> int:
+    """Algorithmic attention FLOPs: 4 * d * sum over valid query rows of their key count.
+
+    Counts QK^T and PV only; softmax and any work on padding are excluded.
+    Mirrors the "Attention computed: X% of full attention" accounting of the
+    Veda node (Veda news page, "Узел ComfyUI").
+    """
+    total_pairs = 0
+    for h in range(cfg.heads):
+        til = head_tiling(cfg, h)
+        n_pre_tok = sum(len(t) for t in til.prefix)
+        n_all = cfg.n_tokens
+        total_pairs += n_pre_tok * n_all
+        # every video tile keeps k tiles; their sizes depend on which tiles are
+        # kept only when tiles are partial, so this closed form needs full tiles
+        sizes = [len(t) for t in til.video]
+        if min(sizes) != TILE:
+            raise ValueError("closed-form count needs full video tiles")
+        kh = int(k_per_head[h])
+        total_pairs += sum(sizes) * (n_pre_tok + kh * TILE)
+    return 4 * cfg.head_dim * total_pairs * cfg.batch

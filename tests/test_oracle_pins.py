@@ -1,0 +1,348 @@
+"""Pins for the fp64 oracle: checks against things other than the oracle itself.
+
+* k = all tiles must reproduce brute-force dense attention (the BSAI VedaSparse
+  README, "Correctness", reports keep=100% sparse equal to dense within 2.4e-7;
+  the fp64 oracle must reach 1e-12).
+* On tiny grids the selected tiles equal exhaustive enumeration of all
+  k-subsets, and the tile loop equals one N x N softmax with an explicit mask.
+* Closed forms: Q = 0 gives uniform weights; V = c gives c; a zero gate makes
+  all scores tie so the k lowest tiles win; constant tiles pool to their
+  constant; one-hot tiles fix which key tile wins and so the orientation of the
+  score matrix.
+* The tile permutation matches a closed-form (tile, slot) formula.
+* Mutation tests plant plausible mistakes in the oracle and check that a pin
+  catches each of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle.vsa_oracle as O
+from vsa_synth import get_config, make_layer_inputs, LayerConfig
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def ragged_config(batch=2):
+    """Small grid with partial prefix tiles and partial, head-specific video tiles."""
+    return LayerConfig(
+        name="ragged", batch=batch, heads=4, head_dim=16, T=6, H=8, W=8,
+        segments=(100, 30), tile_shapes=((4, 4, 4), (16, 2, 2), (2, 4, 8), (8, 4, 2)),
+        score_mode="meanpool_gate", proj_dim=16, sparsity=(0.5,), seed=11)
+
+
+def ragged_tripool_config():
+    return ragged_config(batch=1).with_(name="ragged_tp", score_mode="tripool", proj_dim=8, seed=12)
+
+
+def inputs_f64(cfg):
+    inp = make_layer_inputs(cfg)
+    return inp, inp.as_f64("q"), inp.as_f64("k"), inp.as_f64("v")
+
+
+def n_video_tiles(cfg, h):
+    pt, ph, pw = cfg.tile_shapes[h]
+    return -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw)
+
+
+def closed_form_tile_slot(cfg, h, r):
+    """(tile index in the head's tile list, slot) of token r, from the tiling rules alone."""
+    n_pre = cfg.n_prefix_tokens
+    if r < n_pre:
+        base_tok, base_tile = 0, 0
+        for length in cfg.segments:
+            if r < base_tok + length:
+                j = r - base_tok
+                return base_tile + j // 64, j % 64
+            base_tok += length
+            base_tile += -(-length // 64)
+    n_pre_tiles = sum(-(-length // 64) for length in cfg.segments)
+    pt, ph, pw = cfg.tile_shapes[h]
+    v = r - n_pre
+    t, y, x = v // (cfg.H * cfg.W), (v // cfg.W) % cfg.H, v % cfg.W
+    nY, nX = -(-cfg.H // ph), -(-cfg.W // pw)
+    ti, yi, xi = t // pt, y // ph, x // pw
+    t0, y0, x0 = ti * pt, yi * ph, xi * pw
+    eh, ew = min(ph, cfg.H - y0), min(pw, cfg.W - x0)
+    return n_pre_tiles + (ti * nY + yi) * nX + xi, ((t - t0) * eh + (y - y0)) * ew + (x - x0)
+
+
+def video_tile_of_token(cfg, h, v):
+    """Video tile index of video token v (0-based within the grid), closed form."""
+    pt, ph, pw = cfg.tile_shapes[h]
+    t, y, x = v // (cfg.H * cfg.W), (v // cfg.W) % cfg.H, v % cfg.W
+    nY, nX = -(-cfg.H // ph), -(-cfg.W // pw)
+    return ((t // pt) * nY + y // ph) * nX + x // pw
+
+
+def k_list(cfg, s):
+    return [O.k_from_sparsity(s, n_video_tiles(cfg, h)) for h in range(cfg.heads)]
+
+
+# ---------------------------------------------------------------- pins ------
+
+def pin_dense_when_k_is_all(cfg):
+    inp, q, k, v = inputs_f64(cfg)
+    kk = [n_video_tiles(cfg, h) for h in range(cfg.heads)]
+    res = O.run_layer(cfg, q, k, v, kk, gate=inp.gate, w_q=inp.w_q, w_k=inp.w_k)
+    ref = O.dense_attention(q, k, v, 1.0 / math.sqrt(cfg.head_dim))
+    err = np.max(np.abs(res.out - ref))
+    assert err <= 1e-12, err
+    assert np.max(np.abs(res.row_sum - 1.0)) <= 1e-12
+
+
+def pin_gate_zero_keeps_lowest(cfg):
+    inp, q, k, v = inputs_f64(cfg)
+    kk = k_list(cfg, 0.5)
+    res = O.run_layer(cfg, q, k, v, kk, gate=np.zeros_like(inp.gate), query_tiles={})
+    for h in range(cfg.heads):
+        assert np.all(res.scores[h] == 0.0)
+        want = np.arange(kk[h])
+        assert all(np.array_equal(row, want) for row in res.kept[h]), h
+
+
+def pin_one_hot_orientation():
+    """Query tile i pools to e_i, key tile j to e_{(j+3) mod 8}: row i must keep tile (i-3) mod 8."""
+    cfg = LayerConfig(name="onehot", batch=1, heads=1, head_dim=16, T=4, H=8, W=16,
+                      segments=(64,), tile_shapes=((4, 4, 4),), score_mode="meanpool_gate",
+                      proj_dim=16, sparsity=(0.875,), seed=0)
+    n_pre = 64
+    N = cfg.n_tokens
+    q = np.zeros((1, N, 1, 16))
+    k = np.zeros((1, N, 1, 16))
+    for v_tok in range(cfg.n_video_tokens):
+        j = video_tile_of_token(cfg, 0, v_tok)
+        q[0, n_pre + v_tok, 0, j] = 1.0
+        k[0, n_pre + v_tok, 0, (j + 3) % 8] = 1.0
+    kk = [O.k_from_sparsity(0.875, 8)]
+    assert kk == [1]
+    res = O.run_layer(cfg, q, k, q.copy(), kk, gate=np.eye(16), query_tiles={})
+    got = res.kept[0][:, 0]
+    assert np.array_equal(got, (np.arange(8) - 3) % 8), got
+
+
+def pin_constant_tiles_pool(cfg):
+    """Token value = 1 + its slot: a tile of n tokens pools to avg (n+1)/2, max n, min 1."""
+    for h in range(cfg.heads):
+        til = O.head_tiling(cfg, h)
+        x = np.zeros((cfg.n_tokens, 3))
+        for r in range(cfg.n_tokens):
+            x[r] = 1 + closed_form_tile_slot(cfg, h, r)[1]
+        for tok in til.video:
+            n = len(tok)
+            assert np.allclose(O.mean_pool(x[tok]), (n + 1) / 2, rtol=0, atol=1e-14)
+            tp = O.tripool(x[tok])
+            assert np.allclose(tp, np.r_[[(n + 1) / 2] * 3, [n] * 3, [1] * 3], rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------- tests -----
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "ragged_tp"])
+def test_dense_when_k_is_all(name):
+    cfg = {"tiny": get_config("tiny"), "ragged": ragged_config(),
+           "ragged_tp": ragged_tripool_config()}[name]
+    pin_dense_when_k_is_all(cfg)
+
+
+def test_exhaustive_selection_tiny():
+    cfg = get_config("tiny")
+    inp, q, k, v = inputs_f64(cfg)
+    kk = k_list(cfg, 0.5)
+    res = O.run_layer(cfg, q, k, v, kk, gate=inp.gate, query_tiles={})
+    for h in range(cfg.heads):
+        for i in range(4):
+            assert np.array_equal(res.kept[h][i], O.exhaustive_topk(res.scores[h][i], kk[h]))
+
+
+def test_exhaustive_with_ties():
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        row = rng.integers(0, 3, size=7).astype(np.float64)
+        kk = int(rng.integers(1, 7))
+        assert np.array_equal(O.topk_row(row, kk), O.exhaustive_topk(row, kk))
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "ragged_tp"])
+def test_tile_loop_equals_explicit_mask(name):
+    cfg = {"tiny": get_config("tiny"), "ragged": ragged_config(batch=1),
+           "ragged_tp": ragged_tripool_config()}[name]
+    inp, q, k, v = inputs_f64(cfg)
+    kk = k_list(cfg, 0.5)
+    res = O.run_layer(cfg, q, k, v, kk, gate=inp.gate, w_q=inp.w_q, w_k=inp.w_k)
+    N, n_pre = cfg.n_tokens, cfg.n_prefix_tokens
+    for h in range(cfg.heads):
+        vt = np.array([video_tile_of_token(cfg, h, x) for x in range(cfg.n_video_tokens)])
+        allowed = np.zeros((N, N), dtype=bool)
+        allowed[:n_pre, :] = True                 # prefix rows: every key
+        allowed[:, :n_pre] = True                 # every row: every prefix key
+        for r in range(n_pre, N):
+            kept = res.kept[h][vt[r - n_pre]]
+            allowed[r, n_pre:] = np.isin(vt, kept)
+        ref = O.masked_dense_attention(q[0, :, h], k[0, :, h], v[0, :, h], allowed,
+                                       1.0 / math.sqrt(cfg.head_dim))
+        assert np.max(np.abs(ref - res.out[0, :, h])) <= 1e-12
+
+
+def test_invariants_ragged():
+    cfg = ragged_config()
+    inp, q, k, v = inputs_f64(cfg)
+    kk = k_list(cfg, 0.5)
+    res = O.run_layer(cfg, q, k, v, kk, gate=inp.gate)
+    for h in range(cfg.heads):
+        nv = n_video_tiles(cfg, h)
+        assert res.kept[h].shape == (nv, kk[h])
+        for row in res.kept[h]:
+            assert len(set(row.tolist())) == kk[h]
+            assert np.all(np.diff(row) > 0) and row.min() >= 0 and row.max() < nv
+    assert np.max(np.abs(res.row_sum - 1.0)) <= 1e-12
+    assert np.all(np.isfinite(res.out))
+
+
+def test_q_zero_gives_uniform_mean():
+    cfg = ragged_config(batch=1)
+    inp, q, k, v = inputs_f64(cfg)
+    q[:] = 0.0
+    kk = k_list(cfg, 0.5)
+    res = O.run_layer(cfg, q, k, v, kk, gate=inp.gate)
+    n_pre = cfg.n_prefix_tokens
+    for h in range(cfg.heads):
+        vt = np.array([video_tile_of_token(cfg, h, x) for x in range(cfg.n_video_tokens)])
+        keys = np.r_[np.arange(n_pre), n_pre + np.nonzero(vt < kk[h])[0]]   # ties: lowest k tiles
+        want_video = v[0, keys, h].mean(axis=0)
+        want_prefix = v[0, :, h].mean(axis=0)
+        assert np.max(np.abs(res.out[0, n_pre:, h] - want_video)) <= 1e-12
+        assert np.max(np.abs(res.out[0, :n_pre, h] - want_prefix)) <= 1e-12
+
+
+def test_v_constant_gives_constant():
+    cfg = ragged_tripool_config()
+    inp, q, k, v = inputs_f64(cfg)
+    v[:] = 0.375
+    res = O.run_layer(cfg, q, k, v, k_list(cfg, 0.5), w_q=inp.w_q, w_k=inp.w_k)
+    assert np.max(np.abs(res.out - 0.375)) <= 1e-13
+
+
+def test_gate_zero_keeps_lowest():
+    pin_gate_zero_keeps_lowest(ragged_config(batch=1))
+
+
+def test_one_hot_orientation():
+    pin_one_hot_orientation()
+
+
+def test_constant_tiles_pool():
+    pin_constant_tiles_pool(ragged_config(batch=1))
+
+
+def test_permutation_closed_form():
+    cfg = ragged_config()
+    inp, q, k, v = inputs_f64(cfg)
+    packed, counts = O.pack(q, cfg)
+    seen = np.zeros(packed.shape[1:4], dtype=bool)
+    for h in range(cfg.heads):
+        for r in range(cfg.n_tokens):
+            n, s = closed_form_tile_slot(cfg, h, r)
+            assert np.array_equal(packed[:, h, n, s], q[:, r, h])
+            assert s < counts[h, n]
+            seen[h, n, s] = True
+    assert np.all(packed[:, ~seen] == 0.0)          # padding slots are zero
+    assert seen.sum() == cfg.heads * cfg.n_tokens
+    assert np.array_equal(O.unpack(packed, cfg), q)
+
+
+def test_custom_tiling_golden_partitions_grid():
+    with open(os.path.join(GOLDEN, "custom_tiling.txt")) as f:
+        line = [x for x in f.read().splitlines() if x and not x.startswith("#")][0]
+    shapes = [tuple(int(a) for a in part.split(",")) for part in line.split(";")]
+    assert shapes == [(4, 4, 4), (8, 4, 2), (2, 4, 8), (4, 8, 2)]
+    T, H, W = 28, 48, 80
+    for shp in shapes:
+        assert shp[0] * shp[1] * shp[2] == 64
+        tiles = O.video_tiles(T, H, W, shp, 0)
+        assert len(tiles) == -(-T // shp[0]) * -(-H // shp[1]) * -(-W // shp[2])
+        allt = np.concatenate(tiles)
+        assert np.array_equal(np.sort(allt), np.arange(T * H * W))
+
+
+def test_head_aware_tile_counts():
+    # (16,2,2) on 28 frames: 2 x 24 x 40 tiles, the second temporal row holds 12 frames
+    tiles = O.video_tiles(28, 48, 80, (16, 2, 2), 0)
+    sizes = np.array([len(t) for t in tiles])
+    assert len(tiles) == 1920 and np.sum(sizes == 48) == 960 and np.sum(sizes == 64) == 960
+    assert len(O.prefix_tiles((512, 3840, 640))) == 78
+    assert [len(t) for t in O.prefix_tiles((100, 30))] == [64, 36, 30]
+
+
+def test_k_from_sparsity():
+    with open(os.path.join(GOLDEN, "sparsity_levels.txt")) as f:
+        levels = [float(x.split()[0]) for x in f.read().splitlines() if x and not x.startswith("#")]
+    for s in levels:
+        for n in (4, 120, 1680, 1920, 3600):
+            k = O.k_from_sparsity(s, n)
+            if abs(s * n - round(s * n)) < 1e-9:        # s*n integral: exactly (1-s)*n kept
+                assert k == n - round(s * n), (s, n, k)
+            assert 1 <= k <= n
+    assert O.k_from_sparsity(0.95, 1680) == 84          # not 85: (1-s)*n is 84.00000000000007
+    assert O.k_from_sparsity(0.0, 1680) == 1680
+    assert O.k_from_sparsity(1.0, 1680) == 1
+    assert [O.k_from_sparsity(s, 3600) for s in (0, .5, .75, .9, .95)] == [3600, 1800, 900, 360, 180]
+
+
+def test_flop_count_matches_run():
+    cfg = get_config("tiny")
+    inp, q, k, v = inputs_f64(cfg)
+    kk = k_list(cfg, 0.5)
+    res = O.run_layer(cfg, q, k, v, kk, gate=inp.gate)
+    assert O.attention_flops(cfg, kk) == 4 * cfg.head_dim * res.computed_pairs
+    full = get_config("full")
+    f = O.attention_flops(full, [420] * 24)
+    dense = 4 * 128 * 24 * full.n_tokens ** 2
+    assert abs(f / dense - 0.3151) < 5e-4
+
+
+# ------------------------------------------------------- planted mistakes ---
+
+def _expect_pin_failure(pin, *args):
+    with pytest.raises(AssertionError):
+        pin(*args)
+
+
+def test_mutation_tie_rule(monkeypatch):
+    def bad(row, k):                       # ties resolved toward the higher index
+        j = np.arange(row.shape[0])
+        return np.sort(np.lexsort((-j, -row))[:k])
+    monkeypatch.setattr(O, "topk_row", bad)
+    _expect_pin_failure(pin_gate_zero_keeps_lowest, ragged_config(batch=1))
+
+
+def test_mutation_smallest_instead_of_largest(monkeypatch):
+    monkeypatch.setattr(O, "topk_row", lambda row, k: np.sort(np.lexsort((np.arange(row.size), row))[:k]))
+    _expect_pin_failure(pin_one_hot_orientation)
+
+
+def test_mutation_transposed_scores(monkeypatch):
+    good = O.tile_scores
+    monkeypatch.setattr(O, "tile_scores", lambda *a, **kw: good(*a, **kw).T)
+    _expect_pin_failure(pin_one_hot_orientation)
+
+
+def test_mutation_wrong_scale(monkeypatch):
+    good = O.softmax_attention
+    monkeypatch.setattr(O, "softmax_attention", lambda q, k, v, s: good(q, k, v, 2 * s))
+    _expect_pin_failure(pin_dense_when_k_is_all, get_config("tiny"))
+
+
+def test_mutation_video_rows_lose_prefix(monkeypatch):
+    def bad(til, tile_id, kept):
+        if tile_id < til.n_prefix:
+            return np.concatenate(til.all)
+        return np.concatenate([til.video[j] for j in kept])
+    monkeypatch.setattr(O, "query_key_tokens", bad)
+    _expect_pin_failure(pin_dense_when_k_is_all, get_config("tiny"))
+
+
+def test_mutation_pool_over_64(monkeypatch):
+    monkeypatch.setattr(O, "mean_pool", lambda x: x.sum(axis=0) / 64.0)
+    _expect_pin_failure(pin_constant_tiles_pool, ragged_config(batch=1))

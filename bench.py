@@ -1,0 +1,423 @@
+"""Benchmark: one tile-sparse attention layer of a 1344x768-like clip on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one whole layer -- tile pack, tile score, top-k select, block-sparse
+attention, tile unpack -- through the C ABI of libvsa, on inputs already in
+HBM. Workload: B=1, 24 heads, head_dim 128, video grid 28x48x80 (107,520
+tokens, 1,680 tiles of 4x4x4) after a 4,992-token prefix (512 text, 3,840
+reference-image, 640 reference-audio tokens), mean-pool gate scoring, 75% video
+sparsity (420 kept tiles); the 90% line is measured in the same run. Inputs are
+seeded synthetic tensors (3 x 691 MB, larger than L2).
+
+Multi-GPU (torchrun): every rank runs its own layer (independent problems, no
+collective on the data path); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference there is) on a
+bounded sample of the same workload and extrapolates to one layer.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+CONFIG = "full"
+SPARSITY = 0.75
+SECONDARY_SPARSITY = 0.9
+KERNELS_PER_STEP = 8  # pack 1, score 4 (pool, 2 projections, scores), select 1, attention 1, unpack 1
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=CONFIG)
+    ap.add_argument("--sparsity", type=float, default=SPARSITY)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------- work counts --
+
+def k_list(cfg, s):
+    import oracle.vsa_oracle as O  # the k rule only; no attention work
+    return [O.k_from_sparsity(s, -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw))
+            for (pt, ph, pw) in cfg.tile_shapes]
+
+
+def attention_flops(cfg, ks):
+    """4 * d * sum over query rows of their key count (full tiles: closed form)."""
+    n = cfg.n_tokens
+    npre = cfg.n_prefix_tokens
+    nv = cfg.n_video_tokens
+    pairs = 0
+    for kh in ks:
+        pairs += npre * n + nv * (npre + kh * 64)
+    return 4 * cfg.head_dim * pairs * cfg.batch
+
+
+def layer_bytes(cfg, ks):
+    """Algorithmic HBM bytes of the element-wise stages (pack, pool, select, unpack)."""
+    tok = cfg.batch * cfg.n_tokens * cfg.heads * cfg.head_dim * 2
+    return {"pack": 2 * 3 * tok, "unpack": 2 * tok}
+
+
+# ------------------------------------------------------------------ clocks ----
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r[2] > 300.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i in range(4) if r[3][i + 1].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(load), "power_w_max": max(r[2] for r in rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------- CPU oracle ----
+
+class OracleSample:
+    """The fp64 oracle, as it stands, timed on a bounded sample of one layer (head 0).
+
+    Scores and top-k of the head are timed in full; attention is timed on
+    randomly drawn query tiles (three video tiles per prefix tile) until a time
+    budget is spent; the per-tile means are extrapolated to every query tile of
+    every head of the layer.
+    """
+
+    def __init__(self, cfg, sparsity):
+        import numpy as np
+        import oracle.vsa_oracle as O
+        from vsa_synth import bf16_bits_to_f32, make_layer_inputs
+        self.np, self.O = np, O
+        self.cfg = cfg
+        self.sub = cfg.with_(heads=1, tile_shapes=cfg.tile_shapes[:1])
+        self.inp = make_layer_inputs(self.sub)
+        f = lambda b: bf16_bits_to_f32(b).astype(np.float64)
+        self.q, self.k, self.v = f(self.inp.q), f(self.inp.k), f(self.inp.v)
+        self.ks = k_list(self.sub, sparsity)
+        self.til = O.head_tiling(self.sub, 0)
+        self.rng = np.random.default_rng(0)
+
+    def run(self, budget_s):
+        np, O, sub, til, inp = self.np, self.O, self.sub, self.til, self.inp
+        t0 = time.perf_counter()
+        s = O.tile_scores(self.q[0, :, 0], self.k[0, :, 0], til, sub, 0, inp.gate, inp.w_q, inp.w_k)
+        kept = np.stack([O.topk_row(s[i], self.ks[0]) for i in range(til.n_video)])
+        t_select = time.perf_counter() - t0
+        t_pre = t_vid = 0.0
+        n_pre = n_vid = 0
+        t_start = time.perf_counter()
+        while time.perf_counter() - t_start < budget_s or n_vid == 0:
+            for kind in ("video", "video", "video", "prefix"):
+                if kind == "prefix" and til.n_prefix == 0:
+                    continue
+                t = (int(self.rng.integers(0, til.n_prefix)) if kind == "prefix"
+                     else til.n_prefix + int(self.rng.integers(0, til.n_video)))
+                t1 = time.perf_counter()
+                O.run_layer(sub, self.q, self.k, self.v, self.ks, gate=inp.gate, w_q=inp.w_q, w_k=inp.w_k,
+                            query_tiles={0: [t]}, kept={0: kept})
+                dt = time.perf_counter() - t1
+                if kind == "prefix":
+                    t_pre, n_pre = t_pre + dt, n_pre + 1
+                else:
+                    t_vid, n_vid = t_vid + dt, n_vid + 1
+        # run_layer also recomputes the head's scores on every call: remove that share
+        t_vid_row = max(t_vid / n_vid - t_select, 0.0)
+        t_pre_row = max(t_pre / n_pre - t_select, 0.0) if n_pre else 0.0
+        per_head = t_select + t_vid_row * til.n_video + t_pre_row * til.n_prefix
+        ms = per_head * self.cfg.heads * self.cfg.batch * 1e3
+        try:
+            cores = len(os.sched_getaffinity(0))
+        except AttributeError:
+            cores = os.cpu_count()
+        sample = (f"head 0 of {self.cfg.heads}: scores + top-k of all {til.n_video} video query tiles, attention "
+                  f"of {n_vid} video and {n_pre} prefix query tiles drawn at random (fp64 numpy; BLAS on all "
+                  f"cores); extrapolated to {self.cfg.heads} heads x ({til.n_video} video + {til.n_prefix} "
+                  f"prefix) query tiles")
+        return {"value": round(ms, 1), "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample,
+                "extrapolated": True, "cpu_seconds": round(time.perf_counter() - t0, 1)}
+
+
+def cpu_baseline(cfg, sparsity, budget_s=20.0):
+    return OracleSample(cfg, sparsity).run(budget_s)
+
+
+# ---------------------------------------------------------------- GPU arm ----
+
+def e2e_measure(args, layer, q, k, v, out, stream, world, barrier, max_over_ranks):
+    """The same layer through the public API from pinned host buffers, copies inside the timing."""
+    import torch
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    steps = max(3, min(args.steps, 10))
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        layer.forward(dq, dk, dv, out)
+        ho.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps) / world
+    return {"value": round(ms, 3), "unit": "ms", "h2d_bytes_per_step": 3 * q.numel() * q.element_size() * world,
+            "d2h_bytes_per_step": out.numel() * out.element_size() * world, "steps": steps}
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import tile_sparse_video_pack_b200 as T
+    from tile_sparse_video_pack_b200.build import build
+    from vsa_synth import get_config, make_layer_inputs
+
+    build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = get_config(args.config)
+    if args.heads:
+        cfg = cfg.with_(heads=args.heads, tile_shapes=cfg.tile_shapes[:args.heads])
+    inp = make_layer_inputs(cfg)
+    to_dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    if cfg.score_mode == "meanpool_gate":
+        pq = pk = torch.from_numpy(inp.gate).to(dev)
+    else:
+        pq, pk = torch.from_numpy(inp.w_q).to(dev), torch.from_numpy(inp.w_k).to(dev)
+    peaks = measured_peaks()
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed_layer(sparsity, steps, warmup, sample_clocks):
+        layer = T.TileSparseAttention.from_config(cfg, sparsity, pq, pk)
+        out = torch.empty_like(q)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        for _ in range(warmup):
+            layer.stages(q, k, v, out)
+        layer.plan.check()
+        barrier()
+        torch.cuda.synchronize()
+        clk = ClockSampler(local_rank) if sample_clocks else None
+        if clk:
+            clk.start()
+        barrier()
+        torch.cuda.synchronize()
+        b, p = layer.bufs, layer.plan
+        for i in range(steps):
+            e = ev[i]
+            e[0].record(stream)
+            p.tile_pack(q, k, v, b["qp"], b["kp"], b["vp"])
+            e[1].record(stream)
+            p.tile_score(b["qp"], b["kp"], pq, pk, b["scores"], b["workspace"])
+            e[2].record(stream)
+            p.topk_select(b["scores"], b["idx"])
+            e[3].record(stream)
+            p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], None)
+            e[4].record(stream)
+            p.tile_unpack(b["op"], out)
+            e[5].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        clocks = clk.stop() if clk else None
+        layer.plan.check()
+        total = sum(ev[i][0].elapsed_time(ev[i][5]) for i in range(steps))
+        stages = {name: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps)) / steps
+                  for j, name in enumerate(("pack", "score", "select", "attn", "unpack"))}
+        ms_step = max_over_ranks(total / steps)
+        stats = layer.plan.stats()
+        return layer, out, ms_step, stages, clocks, stats
+
+    ks = k_list(cfg, args.sparsity)
+    layer, out, ms_step, stages, clocks, stats = timed_layer(args.sparsity, args.steps, args.warmup, True)
+    flops = attention_flops(cfg, ks)
+    attn_ms = max_over_ranks(stages["attn"])
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "kernel": "attn_kernel (vsa_sparse_attn)",
+                "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
+                "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),
+                "algorithmic_flops_per_launch": flops}
+
+    # end to end through host buffers: pinned H2D of q, k, v, the layer, D2H of o
+    e2e = None if args.no_e2e else e2e_measure(args, layer, q, k, v, out, stream, world, barrier, max_over_ranks)
+
+    secondary = None
+    if not args.no_secondary:
+        ks2 = k_list(cfg, SECONDARY_SPARSITY)
+        _, _, ms2, st2, _, _ = timed_layer(SECONDARY_SPARSITY, max(3, args.steps // 2), 2, False)
+        f2 = attention_flops(cfg, ks2)
+        secondary = {"sparsity": SECONDARY_SPARSITY, "k": ks2[0], "ms_per_layer": round(ms2 / world, 3),
+                     "stages_ms": {a: round(b, 3) for a, b in st2.items()},
+                     "attn_tflops": round(f2 / (st2["attn"] * 1e-3) / 1e12, 1),
+                     "layer_tflops": round(f2 / (ms2 * 1e-3) / 1e12, 1)}
+
+    value = ms_step / world
+    line = {
+        "metric": "ms per attention layer at 107k video tokens, 75% video sparsity (90% in secondary); effective TFLOP/s",
+        "value": round(value, 3), "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: one layer, B={cfg.batch}, {cfg.heads} heads, d={cfg.head_dim}, "
+                               f"grid {cfg.T}x{cfg.H}x{cfg.W} + prefix {list(cfg.segments)}, "
+                               f"{cfg.score_mode}, sparsity {args.sparsity} (k={ks[0]})",
+                   "tokens": cfg.n_tokens, "heads": cfg.heads, "head_dim": cfg.head_dim, "k": ks[0],
+                   "layers_per_step": world, "parallelism": f"independent layers x{world}",
+                   "l2": "inputs larger than L2 (Q, K, V 691 MB each)"},
+        "stages_ms": {a: round(b, 3) for a, b in stages.items()},
+        "effective_tflops": {"attn_kernel": round(achieved, 1),
+                             "layer": round(flops / (ms_step * 1e-3) / 1e12, 1)},
+        "score_select_share": round((stages["score"] + stages["select"]) / sum(stages.values()), 4),
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clocks,
+        "attention_computed_pct": round(100.0 * stats["computed_pairs"] / stats["dense_pairs"], 2),
+        "secondary": secondary,
+    }
+    return line
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        from vsa_synth import get_config
+        cfg = get_config(args.config)
+        sampler = OracleSample(cfg, args.sparsity)
+        per_step = max(2.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+        vals = []
+        for _ in range(args.warmup):
+            sampler.run(per_step / 2)
+        t0 = time.time()
+        last = None
+        for _ in range(args.steps):
+            last = sampler.run(per_step)
+            vals.append(last["value"])
+        v = statistics.median(vals)
+        line = {"impl": "reference", "metric": "ms per attention layer at 107k video tokens, 75% video sparsity",
+                "value": v, "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": v, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic",
+                "config": {"workload": f"{cfg.name}: one layer, sparsity {args.sparsity}", "tokens": cfg.n_tokens},
+                "cpu_baseline": {**last, "value": v},
+                "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                "wall_s": round(time.time() - t0, 1)}
+        print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        import torch
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            from vsa_synth import get_config
+            line["cpu_baseline"] = cpu_baseline(get_config(args.config), args.sparsity)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

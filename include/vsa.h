@@ -1,0 +1,208 @@
+/*
+ * vsa.h -- C ABI of libvsa: tile-sparse video attention with a dense-exempt
+ * conditioning prefix, for NVIDIA B200 (sm_100a).
+ *
+ * One attention layer of a video-diffusion transformer runs as five calls on
+ * one CUDA stream:
+ *
+ *   vsa_tile_pack   -> vsa_tile_score -> vsa_topk_select -> vsa_sparse_attn
+ *                                                       -> vsa_tile_unpack
+ *
+ * The method (tiles of 64 tokens; a prefix of text / reference-image /
+ * reference-audio tokens in segment-pure tiles that are never pruned; per-head
+ * top-k selection of video key tiles; exact softmax over the kept tiles) is
+ * described on the Ref2VA VSA pages ("Патч внимания с двумя уровнями"; README
+ * "two-tier attention layout") and the Veda / BSAI VedaSparse pages ("Что
+ * делает Veda"; README "Core Technology", "Implementation").
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *    16-byte aligned, and stay valid until the stream reaches the call.
+ *  - Q/K/V/O are bf16 (raw 16-bit patterns, passed as void*). There is no
+ *    other dtype and no implicit conversion: anything else is rejected, as the
+ *    Ref2VA VSA node rejects non-bf16 inputs instead of falling back
+ *    ("From 650 s to 72 s", "The method" / "What transfers": fail loudly).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t, passed as void*; NULL
+ *    is the legacy default stream). Argument errors are returned before
+ *    anything is launched. Errors raised on the device are latched in the plan
+ *    and returned by vsa_plan_check().
+ *  - The library allocates only the plan's small tables and its error word.
+ *    There is no CPU path and no fallback kernel.
+ *  - A plan may be used by one stream at a time; calls on the same plan that
+ *    overlap on the GPU share the attention kernel's work counter and race.
+ */
+#ifndef VSA_H_
+#define VSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define VSA_API __attribute__((visibility("default")))
+#else
+#define VSA_API
+#endif
+
+#define VSA_TILE 64          /* tokens per tile */
+#define VSA_MAX_HEADS 64
+#define VSA_MAX_SEGMENTS 8
+
+typedef enum {
+  VSA_OK = 0,
+  VSA_ERR_INVALID_ARG = 1,     /* bad pointer, size, shape or alignment */
+  VSA_ERR_UNSUPPORTED = 2,     /* valid request this build does not run */
+  VSA_ERR_CUDA = 3,            /* a CUDA runtime or driver call failed */
+  VSA_ERR_DEVICE_TIMEOUT = 4,  /* a device-side wait ran past its limit */
+  VSA_ERR_BAD_INDEX = 5,       /* a kept-tile list holds an out-of-range or repeated tile */
+  VSA_ERR_NO_MEMORY = 6        /* host or device allocation failed */
+} vsa_status;
+
+typedef enum {
+  VSA_SCORE_MEANPOOL_GATE = 0, /* VSA: (mean(Q tile) G) . (mean(K tile) G) / sqrt(d) */
+  VSA_SCORE_TRIPPOOL = 1       /* Veda: ([avg;max;min](Q) Wq[h]) . ([avg;max;min](K) Wk[h]) / sqrt(p) */
+} vsa_score_mode;
+
+/* Layer description. Sequence = prefix segments in order, then the video grid
+ * T x H x W in (t, h, w) raster order (w fastest). Token-major tensors are
+ * [batch, n_tokens, heads, head_dim]. */
+typedef struct {
+  int32_t batch;
+  int32_t heads;                        /* 1 .. VSA_MAX_HEADS */
+  int32_t head_dim;                     /* 64 or 128 */
+  int32_t T, H, W;                      /* video latent grid, each >= 1 */
+  int32_t n_segments;                   /* 0 .. VSA_MAX_SEGMENTS */
+  int32_t seg_len[VSA_MAX_SEGMENTS];    /* prefix segment lengths (>= 1); any length: a
+                                           segment's last tile may be partial */
+  int32_t tile_shape[VSA_MAX_HEADS][3]; /* (pt, ph, pw) per head, pt*ph*pw == 64 */
+  int32_t k_per_head[VSA_MAX_HEADS];    /* kept video key tiles per video query tile,
+                                           1 .. number of video tiles of that head */
+  int32_t score_mode;                   /* vsa_score_mode */
+  int32_t proj_dim;                     /* mean-pool gate: == head_dim; TripPool: 16..128, %16 == 0 */
+  float softmax_scale;                  /* 0 -> 1/sqrt(head_dim) */
+} vsa_desc;
+
+/* Sizes a caller needs to allocate buffers for a plan. */
+typedef struct {
+  int64_t n_tokens;                     /* prefix + video tokens */
+  int32_t n_prefix_tiles;               /* segment-pure prefix tiles (shared by all heads) */
+  int32_t nt_max;                       /* tiles per head in the packed layout (max over heads) */
+  int32_t ntv_max;                      /* video tiles, max over heads */
+  int32_t ntv[VSA_MAX_HEADS];           /* video tiles of each head */
+  int32_t k_max;                        /* max over heads of k_per_head */
+  int64_t packed_elems;                 /* batch*heads*nt_max*64*head_dim (bf16 elements) */
+  int64_t score_elems;                  /* batch*heads*ntv_max*ntv_max (fp32) */
+  int64_t index_elems;                  /* batch*heads*ntv_max*k_max (int32) */
+  int64_t workspace_bytes;              /* scratch for vsa_tile_score */
+  int64_t lse_elems;                    /* batch*heads*nt_max*64 (fp32) */
+  int64_t attn_work_items;              /* 128-row blocks the attention kernel schedules */
+} vsa_plan_info;
+
+typedef struct vsa_plan vsa_plan;
+
+/* Per-plan counters (host-side, updated by the calls). */
+typedef struct {
+  int64_t calls_pack, calls_score, calls_select, calls_attn, calls_unpack;
+  int64_t errors;                       /* non-OK statuses returned by any call */
+  int64_t computed_pairs;               /* (query row, key row) pairs the last attention call
+                                           computed, counting valid rows only: the
+                                           "attention computed X% of full attention" figure
+                                           of the Veda node (Veda page, "Узел ComfyUI") */
+  int64_t dense_pairs;                  /* valid query rows x valid key rows, all heads */
+} vsa_plan_stats;
+
+/* Validates `desc`, builds the tiling tables and the attention work list on
+ * the host, and uploads them to the current CUDA device (the plan is bound to
+ * that device). Blocks until the upload finishes. On any error *out is NULL.
+ * Returns VSA_ERR_INVALID_ARG for a malformed descriptor (checked before any
+ * CUDA call), VSA_ERR_UNSUPPORTED for shapes the kernels do not handle,
+ * VSA_ERR_CUDA / VSA_ERR_NO_MEMORY for device failures. */
+VSA_API vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out);
+
+/* Frees the plan's device tables. Synchronises the device first. NULL is OK. */
+VSA_API vsa_status vsa_plan_destroy(vsa_plan* plan);
+
+VSA_API vsa_status vsa_plan_query(const vsa_plan* plan, vsa_plan_info* out);
+VSA_API vsa_status vsa_plan_get_stats(const vsa_plan* plan, vsa_plan_stats* out);
+
+/* Kept tiles for a sparsity s in [0, 1] over n video tiles:
+ * n - floor(s*n + 0.5) clamped to [1, n] (the pruned share of video key tiles;
+ * Ref2VA VSA README: "75% video sparsity top-k"). Returns 0 for bad input. */
+VSA_API int32_t vsa_k_from_sparsity(double sparsity, int32_t n_tiles);
+
+/* a1. Pack token-major Q, K, V ([B, N, heads, d] bf16) into tile-major
+ * [B, heads, nt_max, 64, d] bf16. Slot s of tile n of head h holds that tile's
+ * s-th token; prefix tiles come first (segment order, 64 consecutive tokens
+ * of one segment each), then video tiles in (ti, hi, wi) raster order with
+ * tokens in (t, h, w) raster order inside the tile; a partial tile's tokens
+ * fill its first slots. Unused slots and unused trailing tiles are zero.
+ * Tiling: Ref2VA VSA README (4x4x4 tiles, segment-pure prefix tiles); BSAI
+ * VedaSparse README "Core Technology: Head-Aware Tiling" and "Implementation"
+ * (_tile_3d returns tiles and their key mask). Any of q/k/v may be NULL to
+ * skip it (its packed pointer is then ignored). */
+VSA_API vsa_status vsa_tile_pack(vsa_plan* plan, const void* q, const void* k, const void* v,
+                         void* qp, void* kp, void* vp, void* stream);
+
+/* a2-a4. Pool every video tile of packed Q and K (mean, or avg/max/min for
+ * TripPool) in fp32, project, and write the tile scores
+ * scores[b][h][i][j] (fp32, [B, heads, ntv_max, ntv_max]; rows/cols past a
+ * head's own ntv are left untouched) for video query tile i and video key tile
+ * j. proj_q/proj_k are fp32 device arrays: mean-pool gate -> both point to G
+ * [d][d] (row-major; q_hat = mean(Q) G); TripPool -> Wq, Wk [heads][3d][p].
+ * workspace: >= workspace_bytes of device scratch, 256-byte aligned.
+ * Ref2VA VSA README (gating projection to_gate_compress decides which tiles
+ * each query attends to); BSAI VedaSparse README "Core Technology: TripPool",
+ * "Scorer Modes" (eq. 5 descriptor, eq. 6 per-head projection score). */
+VSA_API vsa_status vsa_tile_score(vsa_plan* plan, const void* qp, const void* kp,
+                          const float* proj_q, const float* proj_k, float* scores,
+                          void* workspace, void* stream);
+
+/* a5. For every (b, h, video query tile i) keep the k_per_head[h] video key
+ * tiles with the largest scores; equal scores keep the lower tile index. The
+ * kept tile indices (0-based video tile ids) are written sorted ascending to
+ * idx[b][h][i][0 .. k-1] (int32, [B, heads, ntv_max, k_max]). -0.0 and +0.0
+ * compare equal; NaN scores are rejected on the device (VSA_ERR_BAD_INDEX via
+ * vsa_plan_check). Veda page "Что делает Veda" (head-aware top-k forms the
+ * tile mask); Ref2VA VSA README item 2 (top-k only over video key tiles). */
+VSA_API vsa_status vsa_topk_select(vsa_plan* plan, const float* scores, int32_t* idx, void* stream);
+
+/* a6. Block-sparse exact attention on packed tiles. A prefix query tile
+ * attends to every valid key of its head; a video query tile attends to every
+ * prefix tile plus the video tiles listed in idx[b][h][i][0 .. k-1] (ascending,
+ * distinct, in range -- otherwise the rows are skipped and VSA_ERR_BAD_INDEX is
+ * latched). o = softmax(scale * q k^T over the valid keys) v, fp32 accumulation,
+ * written as bf16 to op ([B, heads, nt_max, 64, d]); rows of unused slots of
+ * a head's tiles are zero, and tiles past a head's own tile count (heads with
+ * fewer video tiles than ntv_max) are not written. lse (nullable, fp32
+ * [B, heads, nt_max, 64]) gets the natural-log sum-exp of the scaled logits per
+ * row (0 for unused slots, not written past a head's tiles).
+ * BSAI VedaSparse README "Core Technology: Tile-Skipping", "v3.4 Highlights"
+ * (sink = exact_kv_and_rows: conditioning rows and keys stay exact). */
+VSA_API vsa_status vsa_sparse_attn(vsa_plan* plan, const void* qp, const void* kp, const void* vp,
+                           const int32_t* idx, void* op, float* lse, void* stream);
+
+/* a7. Inverse of the pack permutation: [B, heads, nt_max, 64, d] -> [B, N, heads, d]. */
+VSA_API vsa_status vsa_tile_unpack(vsa_plan* plan, const void* op, void* o, void* stream);
+
+/* All five calls in order on one stream, on caller-provided buffers (sizes
+ * from vsa_plan_query). Returns the first failing call's status. */
+VSA_API vsa_status vsa_layer_forward(vsa_plan* plan, const void* q, const void* k, const void* v,
+                             const float* proj_q, const float* proj_k,
+                             void* qp, void* kp, void* vp, float* scores, int32_t* idx,
+                             void* op, float* lse, void* workspace, void* o, void* stream);
+
+/* Waits for the plan's device (cudaDeviceSynchronize), then returns and clears
+ * the latched device error (VSA_OK if none), or VSA_ERR_CUDA if the device
+ * reports a CUDA error. */
+VSA_API vsa_status vsa_plan_check(vsa_plan* plan);
+
+VSA_API const char* vsa_status_string(vsa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H_ */

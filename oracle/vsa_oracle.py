@@ -263,13 +263,16 @@ class LayerResult:
 
 def run_layer(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, k_per_head,
               gate=None, w_q=None, w_k=None, query_tiles=None,
-              heads=None) -> LayerResult:
+              heads=None, kept=None) -> LayerResult:
     """The whole layer, in fp64: tile, score, select, attend.
 
     ``q``, ``k``, ``v``: ``[B, N, heads, d]`` (any float dtype; widened to fp64).
     ``query_tiles``: optional {head: iterable of tile ids into the head's tile
     list (prefix first, then video)} restricting which query tiles get
     attention rows; the others stay NaN. ``heads`` restricts the heads computed.
+    ``kept``: optional {head: [NTv_h, k_h] array} (or {(b, head): ...}) of kept
+    video tiles to attend with instead of the oracle's own top-k (the scores
+    are still computed and returned).
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -288,12 +291,15 @@ def run_layer(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, k_per_head,
         tiles_h = range(len(til.all)) if query_tiles is None else query_tiles.get(h, ())
         for b in range(B):
             s = tile_scores(q[b, :, h], k[b, :, h], til, cfg, h, gate, w_q, w_k)
-            kept = np.stack([topk_row(s[i], kh) for i in range(til.n_video)])
+            if kept is not None:
+                kept_bh = np.asarray(kept[(b, h)] if (b, h) in kept else kept[h])
+            else:
+                kept_bh = np.stack([topk_row(s[i], kh) for i in range(til.n_video)])
             if b == 0:
-                all_scores[h], all_kept[h] = s, kept
+                all_scores[h], all_kept[h] = s, kept_bh
             for t in tiles_h:
                 qt = til.all[t]
-                kv = query_key_tokens(til, t, None if t < til.n_prefix else kept[t - til.n_prefix])
+                kv = query_key_tokens(til, t, None if t < til.n_prefix else kept_bh[t - til.n_prefix])
                 o, l, rs = softmax_attention(q[b, qt, h], k[b, kv, h], v[b, kv, h], scale)
                 out[b, qt, h], lse[b, qt, h], row_sum[b, qt, h] = o, l, rs
                 pairs += len(qt) * len(kv)

@@ -1,0 +1,747 @@
+// a6: block-sparse exact attention over kept tiles, TMA + tcgen05 (TMEM) on sm_100a.
+//
+// What it computes (BSAI VedaSparse README, "Core Technology: Tile-Skipping"
+// and "v3.4 Highlights": conditioning rows and keys stay exact; Ref2VA VSA
+// README, "two-tier attention layout"): for every query tile, exact softmax
+// attention over the valid keys of the tiles it keeps -- all tiles for a prefix
+// query tile, the prefix tiles plus its top-k video tiles for a video query
+// tile. Scores and accumulation are fp32, P is rounded to bf16 for the PV
+// product, O is rounded to bf16 once.
+//
+// How: one persistent CTA per SM walks a work list of 128-row blocks. A block
+// is two query tiles of one (batch, head) -- neighbours along h on the video
+// grid, or two prefix tiles -- so the tensor core runs M = 128 MMAs. They
+// share one key list: the union of their kept tiles, each entry tagged with
+// which of the two rows-halves keeps it; a row-half masks the other's tiles to
+// -inf. Key tiles go through smem two at a time (128 keys per step).
+//
+// Warp roles (256 threads):
+//   warp 0  TMA producer: Q pair once per block, then K / V tile pairs (2 stages)
+//   warp 1  MMA issuer: S = Q K^T into TMEM (double buffered), O += P V
+//   warp 2  scheduler: fetches the next block from a global counter and builds
+//           its merged key list in smem (double buffered)
+//   warps 4-7  softmax: thread r owns row r (TMEM lane r): online softmax in
+//           fp32, O rescale in TMEM, P to smem (bf16, 128B-swizzled), epilogue
+//
+// Shared-memory operand layouts are the canonical 128-byte-swizzled UMMA
+// layouts that TMA SWIZZLE_128B writes: Q, K and P K-major, V MN-major.
+// Every wait is bounded (about two seconds); on expiry the CTA latches a
+// timeout in the plan's error word, drains its copies and MMAs, frees TMEM and
+// returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "vsa_internal.h"
+
+namespace vsa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr uint32_t kTileBytes = 64 * 64 * 2;  // one 64 x 64 bf16 TMA box
+
+// ------------------------------------------------------------------ PTX ----
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+#define VSA_R32(X)                                                                                            \
+  "+r"(X[0]), "+r"(X[1]), "+r"(X[2]), "+r"(X[3]), "+r"(X[4]), "+r"(X[5]), "+r"(X[6]), "+r"(X[7]), "+r"(X[8]),     \
+      "+r"(X[9]), "+r"(X[10]), "+r"(X[11]), "+r"(X[12]), "+r"(X[13]), "+r"(X[14]), "+r"(X[15]), "+r"(X[16]),    \
+      "+r"(X[17]), "+r"(X[18]), "+r"(X[19]), "+r"(X[20]), "+r"(X[21]), "+r"(X[22]), "+r"(X[23]), "+r"(X[24]),   \
+      "+r"(X[25]), "+r"(X[26]), "+r"(X[27]), "+r"(X[28]), "+r"(X[29]), "+r"(X[30]), "+r"(X[31])
+
+// 32 consecutive TMEM columns of this thread's lane. The registers hold
+// nothing until tmem_wait_ld(): the wait (and reg_fence) name them as in-out
+// operands so that no use of them can be scheduled above the wait.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : VSA_R32(r)::"memory");
+}
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) { asm volatile("" : VSA_R32(r)::"memory"); }
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {  // v: 32 fp32 values
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// UMMA shared-memory descriptor, 128-byte swizzle (layout type 2), version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
+         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) |
+         (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// ------------------------------------------------------- shared layout ----
+
+struct ItemInfo {
+  int32_t bh, qa, qb, n_entries;
+  int32_t rows_a, rows_b, end, bad;
+};
+
+template <int D>
+struct Smem {
+  static constexpr uint32_t kHalfBytes = 128 * 128;               // 128 rows x 128 B
+  static constexpr uint32_t kQBytes = (D / 64) * kHalfBytes;       // Q pair (K-major)
+  static constexpr uint32_t kKBytes = kQBytes;                     // K tile pair
+  static constexpr uint32_t kVBytes = kQBytes;                     // V tile pair (MN-major)
+  static constexpr uint32_t kPBytes = 2 * kHalfBytes;              // P: 128 rows x 128 keys
+  static constexpr uint32_t oQ = 0;
+  static constexpr uint32_t oK = oQ + kQBytes;
+  static constexpr uint32_t oV = oK + 2 * kKBytes;
+  static constexpr uint32_t oP = oV + 2 * kVBytes;
+  static constexpr uint32_t oBar = oP + kPBytes;
+  static constexpr uint32_t kNumBars = 24;
+  static constexpr uint32_t oInfo = oBar + kNumBars * 8;
+  static constexpr uint32_t oMisc = oInfo + 2 * sizeof(ItemInfo);  // tmem base, abort flag
+  static constexpr uint32_t oList = oMisc + 16;
+};
+
+// barrier indices
+enum {
+  B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1, B_VFULL0, B_VFULL1, B_VEMPTY0, B_VEMPTY1,
+  B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1, B_PFULL, B_PEMPTY, B_LFULL0, B_LFULL1, B_LEMPTY0, B_LEMPTY1,
+  B_DRAIN
+};
+
+struct AttnParams {
+  const int32_t* idx;      // [B, heads, ntv_max, k_max]
+  const int32_t* counts;   // [heads, nt_max]
+  const WorkItem* items;
+  int64_t n_items;
+  __nv_bfloat16* out;      // packed O
+  float* lse;
+  uint32_t* state;         // [0] error word, [1] work counter, [2..3] computed pairs
+  int32_t heads, nt_max, ntv_max, k_max, n_pre;
+  int32_t list_cap, bitmap_words;
+  float scale_log2;
+  int32_t ntv[VSA_MAX_HEADS];
+  int32_t k[VSA_MAX_HEADS];
+};
+
+// Bounded wait on an mbarrier phase. Returns false on timeout or when another
+// role has aborted; a timeout latches the error and raises the abort flag.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                         uint32_t* gerr) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      *abort_flag = 1u;
+      atomicOr(gerr, kErrTimeout);
+      return false;
+    }
+  }
+}
+
+// Short bounded wait used only while draining after an abort.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < kTimeoutNs) {
+  }
+}
+
+__device__ __forceinline__ int warp_excl_scan(int v, int lane, int* total) {
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  *total = __shfl_sync(0xffffffffu, x, 31);
+  return x - v;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                const __grid_constant__ CUtensorMap tv, const __grid_constant__ AttnParams prm) {
+  using L = Smem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzle atoms
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) { return sbase + L::oBar + 8u * uint32_t(i); };
+  ItemInfo* info = reinterpret_cast<ItemInfo*>(smem + L::oInfo);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::oMisc);
+  volatile uint32_t* abort_flag = misc + 1;
+  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + L::oList);
+  uint32_t* bitmaps = lists + 2 * prm.list_cap;
+  uint32_t* gerr = prm.state;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QFULL), 1);
+    mbar_init(bar(B_QEMPTY), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_KFULL0 + i), 1);
+      mbar_init(bar(B_KEMPTY0 + i), 1);
+      mbar_init(bar(B_VFULL0 + i), 1);
+      mbar_init(bar(B_VEMPTY0 + i), 1);
+      mbar_init(bar(B_SFULL0 + i), 1);
+      mbar_init(bar(B_SFREE0 + i), 128);
+      mbar_init(bar(B_LFULL0 + i), 32);
+      mbar_init(bar(B_LEMPTY0 + i), 128);
+    }
+    mbar_init(bar(B_PFULL), 128);
+    mbar_init(bar(B_PEMPTY), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    misc[1] = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sbase + L::oMisc),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const uint32_t tS = tmem;          // two S buffers: columns [0,128) and [128,256)
+  const uint32_t tO = tmem + 256;    // O: columns [256, 256 + D)
+
+  if (warp == 2) {
+    // ------------------------------------------------ scheduler / lists ---
+    for (uint32_t it = 0;; ++it) {
+      const int slot = it & 1;
+      bool ok = true;
+      if (lane == 0) ok = wait_bar(bar(B_LEMPTY0 + slot), ((it >> 1) & 1) ^ 1, abort_flag, gerr);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      long long item = 0;
+      if (lane == 0) item = (long long)atomicAdd(prm.state + 1, 1u);
+      item = __shfl_sync(0xffffffffu, item, 0);
+      ItemInfo& inf = info[slot];
+      if (item >= prm.n_items) {
+        if (lane == 0) inf.end = 1;
+        __syncwarp();
+        mbar_arrive(bar(B_LFULL0 + slot));
+        break;
+      }
+      const WorkItem wi = prm.items[item];
+      const int h = wi.bh % prm.heads;
+      const int b = wi.bh / prm.heads;
+      const int ntv = prm.ntv[h];
+      const int nt = prm.n_pre + ntv;
+      const int32_t* cnt = prm.counts + size_t(h) * prm.nt_max;
+      uint32_t* list = lists + slot * prm.list_cap;
+      const uint32_t maskab = wi.qb >= 0 ? 3u : 1u;
+      int n_entries = 0;
+      bool bad = false;
+      if (wi.kind == 0) {
+        // prefix query tiles: every tile of the head, kept by both rows-halves
+        for (int t = lane; t < nt; t += 32) list[t] = uint32_t(t) | (maskab << 16) | (uint32_t(cnt[t]) << 24);
+        n_entries = nt;
+      } else {
+        for (int t = lane; t < prm.n_pre; t += 32)
+          list[t] = uint32_t(t) | (maskab << 16) | (uint32_t(cnt[t]) << 24);
+        uint32_t* bmA = bitmaps;
+        uint32_t* bmB = bitmaps + prm.bitmap_words;
+        const int words = (ntv + 31) >> 5;
+        for (int w = lane; w < words; w += 32) {
+          bmA[w] = 0u;
+          bmB[w] = 0u;
+        }
+        __syncwarp();
+        const int kh = prm.k[h];
+        for (int side = 0; side < 2; ++side) {
+          const int qt = side == 0 ? wi.qa : wi.qb;
+          if (qt < 0) continue;
+          const int32_t* row = prm.idx + ((size_t(b) * prm.heads + h) * prm.ntv_max + (qt - prm.n_pre)) * prm.k_max;
+          uint32_t* bm = side == 0 ? bmA : bmB;
+          for (int e = lane; e < kh; e += 32) {
+            const int j = row[e];
+            const int jp = e > 0 ? row[e - 1] : -1;
+            if (j < 0 || j >= ntv || j <= jp) {
+              bad = true;
+            } else {
+              atomicOr(bm + (j >> 5), 1u << (j & 31));
+            }
+          }
+        }
+        bad = __any_sync(0xffffffffu, bad);
+        __syncwarp();
+        int base = prm.n_pre;
+        if (!bad) {
+          for (int w0 = 0; w0 < words; w0 += 32) {
+            const int w = w0 + lane;
+            const uint32_t a = w < words ? bmA[w] : 0u;
+            const uint32_t bb = w < words ? bmB[w] : 0u;
+            uint32_t u = a | bb;
+            int total;
+            int pos = base + warp_excl_scan(__popc(u), lane, &total);
+            while (u) {
+              const int bit = __ffs(u) - 1;
+              u &= u - 1;
+              const int j = (w << 5) + bit;
+              const uint32_t m = ((a >> bit) & 1u) | (((bb >> bit) & 1u) << 1);
+              const int t = prm.n_pre + j;
+              list[pos++] = uint32_t(t) | (m << 16) | (uint32_t(cnt[t]) << 24);
+            }
+            base += total;
+          }
+        } else if (lane == 0) {
+          atomicOr(gerr, kErrBadIndex);
+        }
+        n_entries = base;
+      }
+      __syncwarp();
+      // valid-pair count for the stats: rows x keys each row-half keeps
+      unsigned long long ka = 0, kb = 0;
+      for (int e = lane; e < n_entries; e += 32) {
+        const uint32_t v = list[e];
+        const uint32_t c = v >> 24;
+        if (v & (1u << 16)) ka += c;
+        if (v & (2u << 16)) kb += c;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ka += __shfl_xor_sync(0xffffffffu, ka, o);
+        kb += __shfl_xor_sync(0xffffffffu, kb, o);
+      }
+      const int rows_a = cnt[wi.qa];
+      const int rows_b = wi.qb >= 0 ? cnt[wi.qb] : 0;
+      if (lane == 0) {
+        inf.bh = wi.bh;
+        inf.qa = wi.qa;
+        inf.qb = wi.qb;
+        inf.n_entries = n_entries;
+        inf.rows_a = rows_a;
+        inf.rows_b = rows_b;
+        inf.end = 0;
+        inf.bad = bad ? 1 : 0;
+        if (!bad)
+          atomicAdd(reinterpret_cast<unsigned long long*>(prm.state + 2),
+                    (unsigned long long)rows_a * ka + (unsigned long long)rows_b * kb);
+      }
+      __syncwarp();
+      mbar_arrive(bar(B_LFULL0 + slot));
+    }
+  } else if (warp == 0) {
+    // ---------------------------------------------------------- producer ---
+    if (lane == 0) {
+      uint32_t g = 0;         // running key-block counter
+      uint32_t issuedQ = 0;   // Q loads issued
+      for (uint32_t it = 0;; ++it) {
+        const int slot = it & 1;
+        if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr)) break;
+        const ItemInfo inf = info[slot];
+        if (inf.end) break;
+        const uint32_t* list = lists + slot * prm.list_cap;
+        const int row_base = inf.bh * prm.nt_max;
+        if (!wait_bar(bar(B_QEMPTY), (it & 1) ^ 1, abort_flag, gerr)) break;
+        mbar_expect_tx(bar(B_QFULL), 2 * (D / 64) * kTileBytes);
+        const int qb = inf.qb >= 0 ? inf.qb : inf.qa;
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_2d(sbase + L::oQ + c * L::kHalfBytes, &tq, 64 * c, (row_base + inf.qa) * 64, bar(B_QFULL));
+          tma_load_2d(sbase + L::oQ + c * L::kHalfBytes + 8192, &tq, 64 * c, (row_base + qb) * 64, bar(B_QFULL));
+        }
+        ++issuedQ;
+        const int nblk = (inf.n_entries + 1) >> 1;
+        bool ok = true;
+        for (int j = 0; j < nblk && ok; ++j, ++g) {
+          const int st = g & 1;
+          const uint32_t ph = (g >> 1) & 1;
+          const int ta = int(list[2 * j] & 0xFFFFu);
+          const int tb = 2 * j + 1 < inf.n_entries ? int(list[2 * j + 1] & 0xFFFFu) : ta;
+          ok = wait_bar(bar(B_KEMPTY0 + st), ph ^ 1, abort_flag, gerr);
+          if (!ok) break;
+          mbar_expect_tx(bar(B_KFULL0 + st), 2 * (D / 64) * kTileBytes);
+          const uint32_t sk = sbase + L::oK + st * L::kKBytes;
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(sk + c * L::kHalfBytes, &tk, 64 * c, (row_base + ta) * 64, bar(B_KFULL0 + st));
+            tma_load_2d(sk + c * L::kHalfBytes + 8192, &tk, 64 * c, (row_base + tb) * 64, bar(B_KFULL0 + st));
+          }
+          ok = wait_bar(bar(B_VEMPTY0 + st), ph ^ 1, abort_flag, gerr);
+          if (!ok) {
+            drain_wait(bar(B_KFULL0 + st), ph);
+            break;
+          }
+          mbar_expect_tx(bar(B_VFULL0 + st), 2 * (D / 64) * kTileBytes);
+          const uint32_t sv = sbase + L::oV + st * L::kVBytes;
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(sv + c * 8192, &tv, 64 * c, (row_base + ta) * 64, bar(B_VFULL0 + st));
+            tma_load_2d(sv + (D / 64) * 8192 + c * 8192, &tv, 64 * c, (row_base + tb) * 64, bar(B_VFULL0 + st));
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        // let every copy this CTA issued land before shared memory is released
+        drain_wait(bar(B_QFULL), (issuedQ - 1) & 1);
+        for (uint32_t gg = (g >= 2 ? g - 2 : 0); gg < g; ++gg) {
+          drain_wait(bar(B_KFULL0 + (gg & 1)), (gg >> 1) & 1);
+          drain_wait(bar(B_VFULL0 + (gg & 1)), (gg >> 1) & 1);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- MMA ---
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idPV = idesc_bf16(128, D, 0, 1);
+      uint32_t g = 0;
+      bool ok = true;
+      auto issue_pv = [&](uint32_t gg, bool first) -> bool {
+        const int st = gg & 1;
+        if (!wait_bar(bar(B_PFULL), gg & 1, abort_flag, gerr)) return false;
+        if (!wait_bar(bar(B_VFULL0 + st), (gg >> 1) & 1, abort_flag, gerr)) return false;
+        tc_fence_after();
+        const uint32_t sv = sbase + L::oV + st * L::kVBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = sw128_desc(sbase + L::oP + (kk >> 2) * L::kHalfBytes + (kk & 3) * 32, 16, 1024);
+          const uint64_t bdesc = sw128_desc(sv + (kk >> 2) * (D / 64) * 8192 + (kk & 3) * 2048, 8192, 1024);
+          tc_mma(tO, a, bdesc, idPV, (first && kk == 0) ? 0u : 1u);
+        }
+        tc_commit(bar(B_VEMPTY0 + st));
+        tc_commit(bar(B_PEMPTY));
+        return true;
+      };
+      for (uint32_t it = 0; ok; ++it) {
+        const int slot = it & 1;
+        if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr)) break;
+        const ItemInfo inf = info[slot];
+        if (inf.end) break;
+        if (!wait_bar(bar(B_QFULL), it & 1, abort_flag, gerr)) break;
+        const int nblk = (inf.n_entries + 1) >> 1;
+        const uint32_t g0 = g;
+        for (int j = 0; j < nblk; ++j, ++g) {
+          const int st = g & 1;
+          if (!(ok = wait_bar(bar(B_KFULL0 + st), (g >> 1) & 1, abort_flag, gerr))) break;
+          if (!(ok = wait_bar(bar(B_SFREE0 + st), ((g >> 1) & 1) ^ 1, abort_flag, gerr))) break;
+          tc_fence_after();
+          const uint32_t sk = sbase + L::oK + st * L::kKBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
+            tc_mma(tS + st * 128, sw128_desc(sbase + L::oQ + off, 16, 1024), sw128_desc(sk + off, 16, 1024), idS,
+                   kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(B_SFULL0 + st));
+          tc_commit(bar(B_KEMPTY0 + st));
+          if (j == nblk - 1) tc_commit(bar(B_QEMPTY));
+          if (j > 0 && !(ok = issue_pv(g - 1, g - 1 == g0))) break;
+        }
+        if (!ok) break;
+        if (!(ok = issue_pv(g - 1, g - 1 == g0))) break;
+      }
+      // nothing of ours may still run on the tensor core when TMEM is freed
+      tc_commit(bar(B_DRAIN));
+      drain_wait(bar(B_DRAIN), 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ----------------------------------------------------------- softmax ---
+    const int r = threadIdx.x - 128;             // row = TMEM lane
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t my_bit = r < 64 ? 1u : 2u;
+    uint32_t g = 0;
+    uint32_t pv_waited = 0;                       // PV completions consumed
+    bool ok = true;
+    for (uint32_t it = 0; ok; ++it) {
+      const int slot = it & 1;
+      ok = wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const ItemInfo inf = info[slot];
+      if (inf.end) break;
+      const uint32_t* list = lists + slot * prm.list_cap;
+      const int nblk = (inf.n_entries + 1) >> 1;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nblk; ++j, ++g) {
+        const int sb = g & 1;
+        ok = wait_bar(bar(B_SFULL0 + sb), (g >> 1) & 1, abort_flag, gerr);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + sb * 128 + lane_off + 32 * c, sr[c]);
+        tmem_wait_ld(sr[0]);
+        reg_fence(sr[1]);
+        reg_fence(sr[2]);
+        reg_fence(sr[3]);
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+        tc_fence_before();
+        mbar_arrive(bar(B_SFREE0 + sb));
+        const uint32_t ea = list[2 * j];
+        const uint32_t eb = 2 * j + 1 < inf.n_entries ? list[2 * j + 1] : 0u;
+        const int ca = ((ea >> 16) & my_bit) ? int(ea >> 24) : 0;   // valid keys of tile a for this row
+        const int cb = ((eb >> 16) & my_bit) ? int(eb >> 24) : 0;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          if (c < ca) mx = fmaxf(mx, s[c]);
+          if (c < cb) mx = fmaxf(mx, s[64 + c]);
+        }
+        const float m_new = fmaxf(m, mx * prm.scale_log2);
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        // a row that has seen no valid key yet holds O = 0 and l = 0: nothing to rescale
+        const float alpha = m == -INFINITY ? 1.f : ex2(m - m_use);
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float pa = c < ca ? ex2(fmaf(s[c], prm.scale_log2, -m_use)) : 0.f;
+          const float pb = c < cb ? ex2(fmaf(s[64 + c], prm.scale_log2, -m_use)) : 0.f;
+          s[c] = pa;
+          s[64 + c] = pb;
+          rs += pa + pb;
+        }
+        l = l * alpha + rs;
+        m = m_new;
+        // the previous PV must be done: it reads the P buffer and writes O
+        if (g > 0 && pv_waited < g) {
+          ok = wait_bar(bar(B_PEMPTY), (g - 1) & 1, abort_flag, gerr);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          pv_waited = g;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
+          const float a = j > 0 ? alpha : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(tO + lane_off + 32 * c, orr);
+            tmem_wait_ld(orr);
+            float o[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]) * a;
+            tmem_st32(tO + lane_off + 32 * c, o);
+          }
+          tmem_wait_st();
+        }
+        // P row -> smem, bf16, K-major 128B swizzle (16-byte chunk c of row r at c ^ (r & 7))
+        uint8_t* prow = smem + L::oP + r * 128;
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch) {
+          const int half = ch >> 3, cc = ch & 7;
+          uint4 pk;
+          __nv_bfloat162 t0 = __floats2bfloat162_rn(s[8 * ch + 0], s[8 * ch + 1]);
+          __nv_bfloat162 t1 = __floats2bfloat162_rn(s[8 * ch + 2], s[8 * ch + 3]);
+          __nv_bfloat162 t2 = __floats2bfloat162_rn(s[8 * ch + 4], s[8 * ch + 5]);
+          __nv_bfloat162 t3 = __floats2bfloat162_rn(s[8 * ch + 6], s[8 * ch + 7]);
+          pk.x = *reinterpret_cast<uint32_t*>(&t0);
+          pk.y = *reinterpret_cast<uint32_t*>(&t1);
+          pk.z = *reinterpret_cast<uint32_t*>(&t2);
+          pk.w = *reinterpret_cast<uint32_t*>(&t3);
+          *reinterpret_cast<uint4*>(prow + half * L::kHalfBytes + ((cc ^ (r & 7)) << 4)) = pk;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL));
+      }
+      if (!ok) break;
+      // epilogue: final O after the last PV
+      ok = wait_bar(bar(B_PEMPTY), (g - 1) & 1, abort_flag, gerr);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      pv_waited = g;
+      tc_fence_after();
+      const int tile = r < 64 ? inf.qa : inf.qb;
+      const int slot_r = r & 63;
+      const int rows = r < 64 ? inf.rows_a : inf.rows_b;
+      const bool write = tile >= 0 && !inf.bad;
+      const bool valid = write && slot_r < rows;
+      const float inv = (valid && l > 0.f) ? 1.f / l : 0.f;
+      const size_t orow = (size_t(inf.bh) * prm.nt_max + (tile >= 0 ? tile : 0)) * 64 + slot_r;
+      uint4* dst = reinterpret_cast<uint4*>(prm.out + orow * D);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t orr[32];
+        tmem_ld32(tO + lane_off + 32 * c, orr);
+        tmem_wait_ld(orr);
+        float o[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]);
+        if (write) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 pk;
+            __nv_bfloat162 t0 = __floats2bfloat162_rn(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+            __nv_bfloat162 t1 = __floats2bfloat162_rn(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+            __nv_bfloat162 t2 = __floats2bfloat162_rn(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+            __nv_bfloat162 t3 = __floats2bfloat162_rn(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+            pk.x = *reinterpret_cast<uint32_t*>(&t0);
+            pk.y = *reinterpret_cast<uint32_t*>(&t1);
+            pk.z = *reinterpret_cast<uint32_t*>(&t2);
+            pk.w = *reinterpret_cast<uint32_t*>(&t3);
+            dst[c * 4 + q] = pk;
+          }
+        }
+      }
+      if (write && prm.lse) prm.lse[orow] = valid && l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : 0.f;
+      tc_fence_before();
+      mbar_arrive(bar(B_LEMPTY0 + slot));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
+
+// --------------------------------------------------------------- host ----
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Packed [rows, d] bf16 viewed as a 2D tensor; 64 x 64 boxes, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int d) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int attn_smem_bytes(int list_cap) {
+  using L = Smem<128>;
+  const int bitmap_words = (list_cap / 32) + 2;
+  return 1024 + int(L::oList) + 2 * list_cap * 4 + 2 * bitmap_words * 4;
+}
+
+cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp, const int32_t* idx, void* op,
+                        float* lse, cudaStream_t s) {
+  const Geometry& g = p->geo;
+  const int64_t rows = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, qp, rows, g.d) || !make_map(&tk, kp, rows, g.d) || !make_map(&tv, vp, rows, g.d))
+    return cudaErrorInvalidValue;
+  AttnParams prm;
+  prm.idx = idx;
+  prm.counts = p->d_tile_count;
+  prm.items = p->d_items;
+  prm.n_items = p->n_items;
+  prm.out = static_cast<__nv_bfloat16*>(op);
+  prm.lse = lse;
+  prm.state = p->d_state;
+  prm.heads = g.Hh;
+  prm.nt_max = g.nt_max;
+  prm.ntv_max = g.ntv_max;
+  prm.k_max = g.k_max;
+  prm.n_pre = g.n_pre_tiles;
+  prm.list_cap = p->list_cap;
+  prm.bitmap_words = (p->list_cap / 32) + 2;
+  prm.scale_log2 = p->desc.softmax_scale * 1.4426950408889634f;
+  for (int h = 0; h < VSA_MAX_HEADS; ++h) {
+    prm.ntv[h] = h < g.Hh ? g.ntv[h] : 0;
+    prm.k[h] = h < g.Hh ? g.k[h] : 0;
+  }
+  // reset the work counter and the pair count
+  cudaError_t e = cudaMemsetAsync(p->d_state + 1, 0, 12, s);
+  if (e != cudaSuccess) return e;
+  const int smem = p->attn_smem_bytes;
+  const int grid = int(p->n_items < p->num_sms ? p->n_items : p->num_sms);
+  if (g.d == 128) {
+    e = cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attn_kernel<128><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm);
+  } else {
+    e = cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attn_kernel<64><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace vsa

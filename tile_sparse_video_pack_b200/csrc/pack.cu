@@ -1,0 +1,142 @@
+// a1 / a7: tile pack and unpack -- a 16-byte vectorised permutation of bf16 rows.
+//
+// Token-major [B, N, heads, d] <-> tile-major [B, heads, nt_max, 64, d].
+// Tiling: Ref2VA VSA README ("two-tier attention layout": 4x4x4 video tiles,
+// segment-pure prefix tiles) and BSAI VedaSparse README ("Core Technology:
+// Head-Aware Tiling", per-head (pt, ph, pw) with product 64).
+#include <cuda_runtime.h>
+
+#include "vsa_internal.h"
+
+namespace vsa {
+namespace {
+
+// Token held by slot s of packed tile n of head h, or -1 for an unused slot.
+// Prefix tiles: 64 consecutive tokens of one segment. Video tiles: the tile's
+// tokens in (t, h, w) raster order over its actual extent (tiles cut by the
+// grid's far edge hold fewer tokens, packed into the first slots).
+__device__ __forceinline__ int src_token(const Geometry& g, int h, int n, int s) {
+  if (n < g.n_pre_tiles) {
+    int i = 0;
+#pragma unroll 1
+    while (i + 1 < g.n_seg && n >= g.seg_tile0[i + 1]) ++i;
+    const int j = (n - g.seg_tile0[i]) * VSA_TILE + s;
+    return j < g.seg_len[i] ? g.seg_tok0[i] + j : -1;
+  }
+  const int v = n - g.n_pre_tiles;
+  if (v >= g.ntv[h]) return -1;
+  const int nX = g.nX[h], nYX = g.nY[h] * nX;
+  const int ti = v / nYX;
+  const int r = v - ti * nYX;
+  const int yi = r / nX;
+  const int xi = r - yi * nX;
+  const int t0 = ti * g.pt[h], y0 = yi * g.ph[h], x0 = xi * g.pw[h];
+  const int et = min(g.pt[h], g.T - t0), eh = min(g.ph[h], g.H - y0), ew = min(g.pw[h], g.W - x0);
+  if (s >= et * eh * ew) return -1;
+  const int ehw = eh * ew;
+  const int dt = s / ehw;
+  const int r2 = s - dt * ehw;
+  const int dy = r2 / ew;
+  const int dx = r2 - dy * ew;
+  return g.n_pre_tok + ((t0 + dt) * g.H + (y0 + dy)) * g.W + (x0 + dx);
+}
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// One thread moves one 16-byte chunk of one packed row of each of up to three
+// tensors (Q, K, V share the permutation).
+template <int CPR>  // 16-byte chunks per row: d / 8
+__global__ void __launch_bounds__(256) pack_kernel(Geometry g, const uint4* __restrict__ q,
+                                                   const uint4* __restrict__ k,
+                                                   const uint4* __restrict__ v, uint4* __restrict__ qp,
+                                                   uint4* __restrict__ kp, uint4* __restrict__ vp) {
+  const int64_t total = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE * CPR;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t row = i / CPR;
+    const int c = int(i - row * CPR);
+    const int s = int(row % VSA_TILE);
+    const int64_t tile = row / VSA_TILE;
+    const int n = int(tile % g.nt_max);
+    const int bh = int(tile / g.nt_max);
+    const int h = bh % g.Hh, b = bh / g.Hh;
+    const int tok = src_token(g, h, n, s);
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    const int64_t src = tok >= 0 ? ((int64_t(b) * g.n_tokens + tok) * g.Hh + h) * CPR + c : 0;
+    uint4 a = zero, bb = zero, cc = zero;
+    if (tok >= 0) {
+      if (q) a = ld_stream(q + src);
+      if (k) bb = ld_stream(k + src);
+      if (v) cc = ld_stream(v + src);
+    }
+    if (q) qp[i] = a;
+    if (k) kp[i] = bb;
+    if (v) vp[i] = cc;
+  }
+}
+
+template <int CPR>
+__global__ void __launch_bounds__(256) unpack_kernel(Geometry g, const uint4* __restrict__ op,
+                                                     uint4* __restrict__ o) {
+  const int64_t total = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE * CPR;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t row = i / CPR;
+    const int c = int(i - row * CPR);
+    const int s = int(row % VSA_TILE);
+    const int64_t tile = row / VSA_TILE;
+    const int n = int(tile % g.nt_max);
+    const int bh = int(tile / g.nt_max);
+    const int h = bh % g.Hh, b = bh / g.Hh;
+    const int tok = src_token(g, h, n, s);
+    if (tok < 0) continue;
+    o[((int64_t(b) * g.n_tokens + tok) * g.Hh + h) * CPR + c] = ld_stream(op + i);
+  }
+}
+
+int grid_for(const vsa_plan* p, int64_t total) {
+  const int64_t want = (total + 255) / 256;
+  const int64_t cap = int64_t(p->num_sms) * 8;  // 8 blocks of 256 threads per SM
+  return int(want < cap ? want : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const vsa_plan* p, const void* q, const void* k, const void* v, void* qp,
+                        void* kp, void* vp, cudaStream_t s) {
+  const Geometry& g = p->geo;
+  const int cpr = g.d / 8;
+  const int64_t total = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE * cpr;
+  const int grid = grid_for(p, total);
+  auto* q4 = static_cast<const uint4*>(q);
+  auto* k4 = static_cast<const uint4*>(k);
+  auto* v4 = static_cast<const uint4*>(v);
+  auto* qp4 = q ? static_cast<uint4*>(qp) : nullptr;
+  auto* kp4 = k ? static_cast<uint4*>(kp) : nullptr;
+  auto* vp4 = v ? static_cast<uint4*>(vp) : nullptr;
+  if (cpr == 16)
+    pack_kernel<16><<<grid, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4);
+  else
+    pack_kernel<8><<<grid, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack(const vsa_plan* p, const void* op, void* o, cudaStream_t s) {
+  const Geometry& g = p->geo;
+  const int cpr = g.d / 8;
+  const int64_t total = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE * cpr;
+  const int grid = grid_for(p, total);
+  if (cpr == 16)
+    unpack_kernel<16><<<grid, 256, 0, s>>>(g, static_cast<const uint4*>(op), static_cast<uint4*>(o));
+  else
+    unpack_kernel<8><<<grid, 256, 0, s>>>(g, static_cast<const uint4*>(op), static_cast<uint4*>(o));
+  return cudaGetLastError();
+}
+
+}  // namespace vsa

@@ -1,0 +1,352 @@
+// C ABI of libvsa: plan construction, argument validation and the entry points.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <new>
+#include <vector>
+
+#include "vsa_internal.h"
+
+using vsa::Geometry;
+using vsa::WorkItem;
+
+namespace {
+
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+vsa_status fail(vsa_plan* p, vsa_status s) {
+  if (p && s != VSA_OK) p->stats.errors++;
+  return s;
+}
+
+// Host-side validation of a descriptor; no CUDA call is made here.
+vsa_status validate(const vsa_desc& d) {
+  if (d.batch < 1 || d.heads < 1 || d.heads > VSA_MAX_HEADS) return VSA_ERR_INVALID_ARG;
+  if (d.head_dim != 64 && d.head_dim != 128) return VSA_ERR_INVALID_ARG;
+  if (d.T < 1 || d.H < 1 || d.W < 1) return VSA_ERR_INVALID_ARG;
+  if (d.n_segments < 0 || d.n_segments > VSA_MAX_SEGMENTS) return VSA_ERR_INVALID_ARG;
+  int64_t n_pre = 0;
+  for (int i = 0; i < d.n_segments; ++i) {
+    if (d.seg_len[i] < 1) return VSA_ERR_INVALID_ARG;
+    n_pre += d.seg_len[i];
+  }
+  const int64_t n_video = int64_t(d.T) * d.H * d.W;
+  const int64_t n_tok = n_pre + n_video;
+  if (n_tok >= (int64_t(1) << 31)) return VSA_ERR_INVALID_ARG;
+  for (int h = 0; h < d.heads; ++h) {
+    const int32_t* s = d.tile_shape[h];
+    if (s[0] < 1 || s[1] < 1 || s[2] < 1 || s[0] * s[1] * s[2] != VSA_TILE) return VSA_ERR_INVALID_ARG;
+    const int64_t ntv = int64_t(cdiv(d.T, s[0])) * cdiv(d.H, s[1]) * cdiv(d.W, s[2]);
+    if (d.k_per_head[h] < 1 || d.k_per_head[h] > ntv) return VSA_ERR_INVALID_ARG;
+  }
+  if (d.score_mode == VSA_SCORE_MEANPOOL_GATE) {
+    if (d.proj_dim != d.head_dim) return VSA_ERR_INVALID_ARG;
+  } else if (d.score_mode == VSA_SCORE_TRIPPOOL) {
+    if (d.proj_dim < 8 || d.proj_dim > 256 || d.proj_dim % 8 != 0) return VSA_ERR_INVALID_ARG;
+  } else {
+    return VSA_ERR_INVALID_ARG;
+  }
+  if (!(d.softmax_scale >= 0.0f) || isinf(d.softmax_scale)) return VSA_ERR_INVALID_ARG;
+  return VSA_OK;
+}
+
+// Pairs the video query tiles of one head: tiles (ti, hi, wi) and (ti, hi+1, wi)
+// share one 128-row block; a leftover row (odd tile count along h) pairs along w.
+void video_pairs(int nT, int nY, int nX, std::vector<std::pair<int, int>>& out) {
+  std::vector<char> used(size_t(nT) * nY * nX, 0);
+  std::vector<int> singles;
+  for (int t = 0; t < nT; ++t)
+    for (int y = 0; y < nY; ++y)
+      for (int x = 0; x < nX; ++x) {
+        const int a = (t * nY + y) * nX + x;
+        if (used[a]) continue;
+        if (y % 2 == 0 && y + 1 < nY) {
+          const int b = a + nX;
+          used[a] = used[b] = 1;
+          out.emplace_back(a, b);
+        } else {
+          used[a] = 1;
+          singles.push_back(a);
+        }
+      }
+  for (size_t i = 0; i < singles.size(); i += 2)
+    out.emplace_back(singles[i], i + 1 < singles.size() ? singles[i + 1] : -1);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vsa_status_string(vsa_status s) {
+  switch (s) {
+    case VSA_OK: return "VSA_OK";
+    case VSA_ERR_INVALID_ARG: return "VSA_ERR_INVALID_ARG: invalid argument";
+    case VSA_ERR_UNSUPPORTED: return "VSA_ERR_UNSUPPORTED: shape not supported by these kernels";
+    case VSA_ERR_CUDA: return "VSA_ERR_CUDA: CUDA call failed";
+    case VSA_ERR_DEVICE_TIMEOUT: return "VSA_ERR_DEVICE_TIMEOUT: device-side wait ran out";
+    case VSA_ERR_BAD_INDEX: return "VSA_ERR_BAD_INDEX: invalid kept-tile index list or NaN score";
+    case VSA_ERR_NO_MEMORY: return "VSA_ERR_NO_MEMORY: allocation failed";
+  }
+  return "unknown vsa_status";
+}
+
+int32_t vsa_k_from_sparsity(double s, int32_t n) {
+  if (!(s >= 0.0 && s <= 1.0) || n < 1) return 0;
+  int64_t k = int64_t(n) - int64_t(floor(s * double(n) + 0.5));
+  if (k < 1) k = 1;
+  if (k > n) k = n;
+  return int32_t(k);
+}
+
+vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
+  if (!out) return VSA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!desc) return VSA_ERR_INVALID_ARG;
+  vsa_status st = validate(*desc);
+  if (st != VSA_OK) return st;
+  const vsa_desc& d = *desc;
+
+  vsa_plan* p = new (std::nothrow) vsa_plan();
+  if (!p) return VSA_ERR_NO_MEMORY;
+  p->desc = d;
+  if (p->desc.softmax_scale == 0.0f) p->desc.softmax_scale = 1.0f / sqrtf(float(d.head_dim));
+
+  Geometry& g = p->geo;
+  memset(&g, 0, sizeof(g));
+  g.B = d.batch;
+  g.Hh = d.heads;
+  g.d = d.head_dim;
+  g.T = d.T;
+  g.H = d.H;
+  g.W = d.W;
+  g.n_seg = d.n_segments;
+  int tok = 0, tile = 0;
+  for (int i = 0; i < d.n_segments; ++i) {
+    g.seg_tok0[i] = tok;
+    g.seg_tile0[i] = tile;
+    g.seg_len[i] = d.seg_len[i];
+    tok += d.seg_len[i];
+    tile += cdiv(d.seg_len[i], VSA_TILE);
+  }
+  g.seg_tok0[d.n_segments] = tok;
+  g.seg_tile0[d.n_segments] = tile;
+  g.n_pre_tok = tok;
+  g.n_pre_tiles = tile;
+  g.n_tokens = tok + d.T * d.H * d.W;
+  g.ntv_max = 0;
+  g.k_max = 0;
+  for (int h = 0; h < d.heads; ++h) {
+    g.pt[h] = d.tile_shape[h][0];
+    g.ph[h] = d.tile_shape[h][1];
+    g.pw[h] = d.tile_shape[h][2];
+    g.nY[h] = cdiv(d.H, g.ph[h]);
+    g.nX[h] = cdiv(d.W, g.pw[h]);
+    g.ntv[h] = cdiv(d.T, g.pt[h]) * g.nY[h] * g.nX[h];
+    g.k[h] = d.k_per_head[h];
+    g.ntv_max = std::max(g.ntv_max, g.ntv[h]);
+    g.k_max = std::max(g.k_max, g.k[h]);
+  }
+  g.nt_max = g.n_pre_tiles + g.ntv_max;
+
+  // the attention kernel keeps one item's key list in shared memory
+  p->list_cap = g.nt_max;
+  p->attn_smem_bytes = vsa::attn_smem_bytes(p->list_cap);
+  if (p->attn_smem_bytes > 227 * 1024 || g.nt_max >= 65536) {
+    delete p;
+    return VSA_ERR_UNSUPPORTED;
+  }
+
+  vsa_plan_info& info = p->info;
+  memset(&info, 0, sizeof(info));
+  info.n_tokens = g.n_tokens;
+  info.n_prefix_tiles = g.n_pre_tiles;
+  info.nt_max = g.nt_max;
+  info.ntv_max = g.ntv_max;
+  for (int h = 0; h < d.heads; ++h) info.ntv[h] = g.ntv[h];
+  info.k_max = g.k_max;
+  info.packed_elems = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE * g.d;
+  info.score_elems = int64_t(g.B) * g.Hh * g.ntv_max * g.ntv_max;
+  info.index_elems = int64_t(g.B) * g.Hh * g.ntv_max * g.k_max;
+  info.workspace_bytes = vsa::score_workspace_bytes(g, d.score_mode, d.proj_dim);
+  info.lse_elems = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE;
+
+  // tile valid counts
+  std::vector<int32_t> counts(size_t(g.Hh) * g.nt_max, 0);
+  for (int h = 0; h < g.Hh; ++h) {
+    int32_t* c = &counts[size_t(h) * g.nt_max];
+    for (int s = 0; s < g.n_seg; ++s)
+      for (int t = g.seg_tile0[s]; t < g.seg_tile0[s + 1]; ++t)
+        c[t] = std::min(VSA_TILE, g.seg_len[s] - (t - g.seg_tile0[s]) * VSA_TILE);
+    const int nT = cdiv(g.T, g.pt[h]);
+    for (int ti = 0; ti < nT; ++ti)
+      for (int yi = 0; yi < g.nY[h]; ++yi)
+        for (int xi = 0; xi < g.nX[h]; ++xi) {
+          const int et = std::min(g.pt[h], g.T - ti * g.pt[h]);
+          const int eh = std::min(g.ph[h], g.H - yi * g.ph[h]);
+          const int ew = std::min(g.pw[h], g.W - xi * g.pw[h]);
+          c[g.n_pre_tiles + (ti * g.nY[h] + yi) * g.nX[h] + xi] = et * eh * ew;
+        }
+  }
+
+  // attention work list: head by head, prefix query blocks (heaviest) first
+  std::vector<WorkItem> items;
+  std::vector<std::pair<int, int>> pairs;
+  for (int b = 0; b < g.B; ++b)
+    for (int h = 0; h < g.Hh; ++h) {
+      const int bh = b * g.Hh + h;
+      for (int t = 0; t < g.n_pre_tiles; t += 2)
+        items.push_back({bh, t, t + 1 < g.n_pre_tiles ? t + 1 : -1, 0});
+      pairs.clear();
+      video_pairs(cdiv(g.T, g.pt[h]), g.nY[h], g.nX[h], pairs);
+      for (auto& pr : pairs)
+        items.push_back({bh, g.n_pre_tiles + pr.first,
+                         pr.second >= 0 ? g.n_pre_tiles + pr.second : -1, 1});
+    }
+  p->n_items = int64_t(items.size());
+  info.attn_work_items = p->n_items;
+
+  // dense pair count (valid rows x valid keys) for the stats
+  p->stats.dense_pairs = int64_t(g.B) * g.Hh * int64_t(g.n_tokens) * g.n_tokens;
+
+  // device tables
+  cudaError_t e = cudaGetDevice(&p->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->device);
+  if (e == cudaSuccess) e = cudaMalloc(&p->d_tile_count, counts.size() * sizeof(int32_t));
+  if (e == cudaSuccess) e = cudaMalloc(&p->d_items, items.size() * sizeof(WorkItem));
+  if (e == cudaSuccess) e = cudaMalloc(&p->d_state, 64);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(p->d_tile_count, counts.data(), counts.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(p->d_items, items.data(), items.size() * sizeof(WorkItem), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemset(p->d_state, 0, 64);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    vsa_status r = (e == cudaErrorMemoryAllocation) ? VSA_ERR_NO_MEMORY : VSA_ERR_CUDA;
+    vsa_plan_destroy(p);
+    return r;
+  }
+  *out = p;
+  return VSA_OK;
+}
+
+vsa_status vsa_plan_destroy(vsa_plan* p) {
+  if (!p) return VSA_OK;
+  if (p->d_tile_count || p->d_items || p->d_state) cudaDeviceSynchronize();
+  if (p->d_tile_count) cudaFree(p->d_tile_count);
+  if (p->d_items) cudaFree(p->d_items);
+  if (p->d_state) cudaFree(p->d_state);
+  delete p;
+  return VSA_OK;
+}
+
+vsa_status vsa_plan_query(const vsa_plan* p, vsa_plan_info* out) {
+  if (!p || !out) return VSA_ERR_INVALID_ARG;
+  *out = p->info;
+  return VSA_OK;
+}
+
+vsa_status vsa_plan_get_stats(const vsa_plan* p, vsa_plan_stats* out) {
+  if (!p || !out) return VSA_ERR_INVALID_ARG;
+  *out = p->stats;
+  uint64_t pairs = 0;
+  if (cudaMemcpy(&pairs, reinterpret_cast<const char*>(p->d_state) + 8, 8, cudaMemcpyDeviceToHost) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return VSA_ERR_CUDA;
+  }
+  out->computed_pairs = int64_t(pairs);
+  return VSA_OK;
+}
+
+vsa_status vsa_tile_pack(vsa_plan* p, const void* q, const void* k, const void* v, void* qp, void* kp,
+                         void* vp, void* stream) {
+  if (!p) return VSA_ERR_INVALID_ARG;
+  const void* src[3] = {q, k, v};
+  void* dst[3] = {qp, kp, vp};
+  int n = 0;
+  for (int i = 0; i < 3; ++i) {
+    if (!src[i]) continue;
+    if (!dst[i] || !aligned16(src[i]) || !aligned16(dst[i])) return fail(p, VSA_ERR_INVALID_ARG);
+    ++n;
+  }
+  if (n == 0) return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_pack++;
+  if (vsa::launch_pack(p, q, k, v, qp, kp, vp, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_tile_unpack(vsa_plan* p, const void* op, void* o, void* stream) {
+  if (!p || !op || !o || !aligned16(op) || !aligned16(o)) return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_unpack++;
+  if (vsa::launch_unpack(p, op, o, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_tile_score(vsa_plan* p, const void* qp, const void* kp, const float* proj_q,
+                          const float* proj_k, float* scores, void* ws, void* stream) {
+  if (!p || !qp || !kp || !proj_q || !proj_k || !scores || !ws) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!aligned16(qp) || !aligned16(kp) || !aligned16(proj_q) || !aligned16(proj_k) ||
+      !aligned16(scores) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_score++;
+  if (vsa::launch_score(p, qp, kp, proj_q, proj_k, scores, ws, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_topk_select(vsa_plan* p, const float* scores, int32_t* idx, void* stream) {
+  if (!p || !scores || !idx || !aligned16(scores) || !aligned16(idx)) return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_select++;
+  if (vsa::launch_topk(p, scores, idx, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_sparse_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp,
+                           const int32_t* idx, void* op, float* lse, void* stream) {
+  if (!p || !qp || !kp || !vp || !idx || !op) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(idx) || !aligned16(op) ||
+      (lse && !aligned16(lse)))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_attn++;
+  if (vsa::launch_attn(p, qp, kp, vp, idx, op, lse, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_layer_forward(vsa_plan* p, const void* q, const void* k, const void* v,
+                             const float* proj_q, const float* proj_k, void* qp, void* kp, void* vp,
+                             float* scores, int32_t* idx, void* op, float* lse, void* ws, void* o,
+                             void* stream) {
+  vsa_status s = vsa_tile_pack(p, q, k, v, qp, kp, vp, stream);
+  if (s == VSA_OK) s = vsa_tile_score(p, qp, kp, proj_q, proj_k, scores, ws, stream);
+  if (s == VSA_OK) s = vsa_topk_select(p, scores, idx, stream);
+  if (s == VSA_OK) s = vsa_sparse_attn(p, qp, kp, vp, idx, op, lse, stream);
+  if (s == VSA_OK) s = vsa_tile_unpack(p, op, o, stream);
+  return s;
+}
+
+vsa_status vsa_plan_check(vsa_plan* p) {
+  if (!p) return VSA_ERR_INVALID_ARG;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return fail(p, VSA_ERR_CUDA);
+  uint32_t err = 0;
+  e = cudaMemcpy(&err, p->d_state, 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(p, VSA_ERR_CUDA);
+  if (err) {
+    if (cudaMemset(p->d_state, 0, 4) != cudaSuccess) return fail(p, VSA_ERR_CUDA);
+    if (err & vsa::kErrTimeout) return fail(p, VSA_ERR_DEVICE_TIMEOUT);
+    return fail(p, VSA_ERR_BAD_INDEX);
+  }
+  return VSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,73 @@
+// Internal declarations shared by the libvsa CUDA sources.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/vsa.h"
+
+namespace vsa {
+
+// Bits of the device error word.
+enum : uint32_t {
+  kErrTimeout = 1u << 0,
+  kErrBadIndex = 1u << 1,
+};
+
+// Tiling of one layer, passed by value to the element-wise kernels.
+struct Geometry {
+  int32_t B, Hh, d;
+  int32_t T, H, W;
+  int32_t n_tokens, n_pre_tok, n_pre_tiles, nt_max, ntv_max, k_max;
+  int32_t n_seg;
+  int32_t seg_tok0[VSA_MAX_SEGMENTS + 1];   // first token of each segment (+ end)
+  int32_t seg_tile0[VSA_MAX_SEGMENTS + 1];  // first prefix tile of each segment (+ end)
+  int32_t seg_len[VSA_MAX_SEGMENTS];
+  int32_t pt[VSA_MAX_HEADS], ph[VSA_MAX_HEADS], pw[VSA_MAX_HEADS];
+  int32_t nY[VSA_MAX_HEADS], nX[VSA_MAX_HEADS], ntv[VSA_MAX_HEADS];
+  int32_t k[VSA_MAX_HEADS];
+};
+
+// One 128-row block of attention work: two query tiles of one (batch, head)
+// that share a merged key list (qb < 0: a single query tile).
+struct WorkItem {
+  int32_t bh;      // b * heads + h
+  int32_t qa, qb;  // packed tile ids (prefix tiles first)
+  int32_t kind;    // 0: prefix query tiles (dense rows), 1: video query tiles
+};
+
+}  // namespace vsa
+
+struct vsa_plan {
+  vsa_desc desc;
+  vsa_plan_info info;
+  vsa_plan_stats stats;
+  vsa::Geometry geo;
+  int device;
+  int num_sms;
+  // device tables
+  int32_t* d_tile_count;   // [heads][nt_max] valid tokens per packed tile
+  vsa::WorkItem* d_items;  // attention work list, heaviest first
+  int64_t n_items;
+  uint32_t* d_state;       // [0] error word, [1] work counter
+  int attn_smem_bytes;
+  int list_cap;            // entries of one key-list buffer in the attention kernel
+};
+
+namespace vsa {
+
+// Launchers (return cudaGetLastError()).
+cudaError_t launch_pack(const vsa_plan* p, const void* q, const void* k, const void* v, void* qp,
+                        void* kp, void* vp, cudaStream_t s);
+cudaError_t launch_unpack(const vsa_plan* p, const void* op, void* o, cudaStream_t s);
+cudaError_t launch_score(const vsa_plan* p, const void* qp, const void* kp, const float* proj_q,
+                         const float* proj_k, float* scores, void* workspace, cudaStream_t s);
+int64_t score_workspace_bytes(const Geometry& g, int score_mode, int proj_dim);
+cudaError_t launch_topk(const vsa_plan* p, const float* scores, int32_t* idx, cudaStream_t s);
+cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp,
+                        const int32_t* idx, void* op, float* lse, cudaStream_t s);
+int attn_smem_bytes(int list_cap);
+
+}  // namespace vsa

@@ -1,0 +1,46 @@
+"""One tile-sparse attention layer: a plan, its device buffers and its score weights."""
+from __future__ import annotations
+
+from .vsa import Plan, make_desc, k_from_sparsity
+
+
+class TileSparseAttention:
+    """Runs pack -> score -> select -> sparse attention -> unpack on token-major bf16 Q, K, V.
+
+    ``proj_q`` / ``proj_k``: fp32 CUDA tensors -- the gate G ([d, d], the same
+    tensor for both) for mean-pool scoring, or per-head TripPool projections
+    ([heads, 3d, p]).
+    """
+
+    def __init__(self, plan: Plan, proj_q, proj_k, with_lse: bool = False, device=None):
+        self.plan = plan
+        self.proj_q = proj_q
+        self.proj_k = proj_k
+        self.bufs = plan.allocate(device, with_lse=with_lse)
+
+    @classmethod
+    def from_config(cls, cfg, sparsity, proj_q, proj_k, **kw):
+        return cls(Plan.from_config(cfg, sparsity), proj_q, proj_k, **kw)
+
+    def forward(self, q, k, v, out=None, stream=None):
+        """Token-major ``[B, N, heads, d]`` bf16 CUDA tensors -> output of the same shape."""
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        self.plan.layer_forward(q, k, v, self.proj_q, self.proj_k, self.bufs, out, stream=stream)
+        return out
+
+    __call__ = forward
+
+    def stages(self, q, k, v, out, stream=None):
+        """The five calls one by one (same result as :meth:`forward`)."""
+        b, p = self.bufs, self.plan
+        p.tile_pack(q, k, v, b["qp"], b["kp"], b["vp"], stream)
+        p.tile_score(b["qp"], b["kp"], self.proj_q, self.proj_k, b["scores"], b["workspace"], stream)
+        p.topk_select(b["scores"], b["idx"], stream)
+        p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], b["lse"], stream)
+        p.tile_unpack(b["op"], out, stream)
+        return out
+
+
+__all__ = ["TileSparseAttention", "Plan", "make_desc", "k_from_sparsity"]

@@ -165,11 +165,14 @@ class OracleSample:
         self.rng = np.random.default_rng(0)
 
     def run(self, budget_s):
+        """Times the oracle's own steps: scores + top-k of the head, then its per-tile attention."""
         np, O, sub, til, inp = self.np, self.O, self.sub, self.til, self.inp
         t0 = time.perf_counter()
         s = O.tile_scores(self.q[0, :, 0], self.k[0, :, 0], til, sub, 0, inp.gate, inp.w_q, inp.w_k)
         kept = np.stack([O.topk_row(s[i], self.ks[0]) for i in range(til.n_video)])
         t_select = time.perf_counter() - t0
+        scale = 1.0 / math.sqrt(sub.head_dim)
+        q, k, v = self.q[0, :, 0], self.k[0, :, 0], self.v[0, :, 0]
         t_pre = t_vid = 0.0
         n_pre = n_vid = 0
         t_start = time.perf_counter()
@@ -180,16 +183,17 @@ class OracleSample:
                 t = (int(self.rng.integers(0, til.n_prefix)) if kind == "prefix"
                      else til.n_prefix + int(self.rng.integers(0, til.n_video)))
                 t1 = time.perf_counter()
-                O.run_layer(sub, self.q, self.k, self.v, self.ks, gate=inp.gate, w_q=inp.w_q, w_k=inp.w_k,
-                            query_tiles={0: [t]}, kept={0: kept})
+                # the same two calls run_layer makes for one query tile
+                kv = O.query_key_tokens(til, t, None if t < til.n_prefix else kept[t - til.n_prefix])
+                qt = til.all[t]
+                O.softmax_attention(q[qt], k[kv], v[kv], scale)
                 dt = time.perf_counter() - t1
                 if kind == "prefix":
                     t_pre, n_pre = t_pre + dt, n_pre + 1
                 else:
                     t_vid, n_vid = t_vid + dt, n_vid + 1
-        # run_layer also recomputes the head's scores on every call: remove that share
-        t_vid_row = max(t_vid / n_vid - t_select, 0.0)
-        t_pre_row = max(t_pre / n_pre - t_select, 0.0) if n_pre else 0.0
+        t_vid_row = t_vid / n_vid
+        t_pre_row = t_pre / n_pre if n_pre else 0.0
         per_head = t_select + t_vid_row * til.n_video + t_pre_row * til.n_prefix
         ms = per_head * self.cfg.heads * self.cfg.batch * 1e3
         try:
@@ -206,6 +210,24 @@ class OracleSample:
 
 def cpu_baseline(cfg, sparsity, budget_s=20.0):
     return OracleSample(cfg, sparsity).run(budget_s)
+
+
+# ---------------------------------------------------------------- ranks ------
+
+def max_over_ranks_on(x: float, device, world: int) -> float:
+    """The largest of every rank's x (each rank runs the same number of steps)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_ms_per_layer(ms_step_max: float, layers_per_rank: int, world: int) -> float:
+    """Whole-job time per layer: the slowest rank's step time over all layers processed in a step."""
+    return ms_step_max / (layers_per_rank * world)
 
 
 # ---------------------------------------------------------------- GPU arm ----
@@ -270,11 +292,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_on(x, dev, world)
 
     def timed_layer(sparsity, steps, warmup, sample_clocks):
         layer = T.TileSparseAttention.from_config(cfg, sparsity, pq, pk)
@@ -341,7 +359,7 @@ def run_ours(args, rank, world, local_rank):
                      "attn_tflops": round(f2 / (st2["attn"] * 1e-3) / 1e12, 1),
                      "layer_tflops": round(f2 / (ms2 * 1e-3) / 1e12, 1)}
 
-    value = ms_step / world
+    value = job_ms_per_layer(ms_step, 1, world)
     line = {
         "metric": "ms per attention layer at 107k video tokens, 75% video sparsity (90% in secondary); effective TFLOP/s",
         "value": round(value, 3), "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -82,11 +82,10 @@ def test_long_clip_dense_and_sparse():
     sampled_parity(r, heads=[5], n_video_samples=3)
     # cross-check (not the oracle): torch dense attention on two heads
     for h in (0, 17):
-        qh = r.q[:, :, h].transpose(0, 1).unsqueeze(0).float()
-        kh = r.k_t[:, :, h].transpose(0, 1).unsqueeze(0).float()
-        vh = r.v[:, :, h].transpose(0, 1).unsqueeze(0).float()
-        ref = F.scaled_dot_product_attention(qh.bfloat16(), kh.bfloat16(), vh.bfloat16()).float()
-        got = r.out[:, :, h].transpose(0, 1).unsqueeze(0).float()
+        # [B, N, heads, d] -> [B, 1, N, d] for one head
+        qh, kh, vh = (x[:, :, h].unsqueeze(1) for x in (r.q, r.k_t, r.v))
+        ref = F.scaled_dot_product_attention(qh, kh, vh).float()
+        got = r.out[:, :, h].unsqueeze(1).float()
         err = (got - ref).abs().max().item()
         assert err <= 2e-2, err
     r2 = GpuRun(cfg, 0.9, inputs=r.inp).run()

@@ -20,8 +20,10 @@
 //   warp 1  MMA issuer: S = Q K^T into TMEM (double buffered), O += P V
 //   warp 2  scheduler: fetches the next block from a global counter and builds
 //           its merged key list in smem (double buffered)
-//   warps 4-7  softmax: thread r owns row r (TMEM lane r): online softmax in
-//           fp32, O rescale in TMEM, P to smem (bf16, 128B-swizzled), epilogue
+//   warps 4-11 softmax, two warpgroups: row r (TMEM lane r) is shared by one
+//           thread of each; warpgroup g handles key tile g of every 128-key
+//           block and half of O. Online softmax in fp32 with a lazily raised
+//           running max, O rescale in TMEM, P to smem (bf16, 128B-swizzled)
 //
 // Shared-memory operand layouts are the canonical 128-byte-swizzled UMMA
 // layouts that TMA SWIZZLE_128B writes: Q, K and P K-major, V MN-major.
@@ -38,7 +40,8 @@
 namespace vsa {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
+constexpr float kLazy = 8.0f;  // log2 headroom before the running max is raised
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint32_t kTileBytes = 64 * 64 * 2;  // one 64 x 64 bf16 TMA box
@@ -168,14 +171,15 @@ struct Smem {
   static constexpr uint32_t kNumBars = 24;
   static constexpr uint32_t oInfo = oBar + kNumBars * 8;
   static constexpr uint32_t oMisc = oInfo + 2 * sizeof(ItemInfo);  // tmem base, abort flag
-  static constexpr uint32_t oList = oMisc + 16;
+  static constexpr uint32_t oXchg = oMisc + 16;                     // row max / row sum exchange
+  static constexpr uint32_t oList = oXchg + (2 * 2 * 128 + 2 * 128) * 4;
 };
 
 // barrier indices
 enum {
   B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1, B_VFULL0, B_VFULL1, B_VEMPTY0, B_VEMPTY1,
   B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1, B_PFULL, B_PEMPTY, B_LFULL0, B_LFULL1, B_LEMPTY0, B_LEMPTY1,
-  B_DRAIN
+  B_DRAIN, B_MX0, B_MX1, B_LX
 };
 
 struct AttnParams {
@@ -257,11 +261,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_VFULL0 + i), 1);
       mbar_init(bar(B_VEMPTY0 + i), 1);
       mbar_init(bar(B_SFULL0 + i), 1);
-      mbar_init(bar(B_SFREE0 + i), 128);
+      mbar_init(bar(B_SFREE0 + i), 256);
       mbar_init(bar(B_LFULL0 + i), 32);
-      mbar_init(bar(B_LEMPTY0 + i), 128);
+      mbar_init(bar(B_LEMPTY0 + i), 256);
+      mbar_init(bar(B_MX0 + i), 256);
     }
-    mbar_init(bar(B_PFULL), 128);
+    mbar_init(bar(B_LX), 256);
+    mbar_init(bar(B_PFULL), 256);
     mbar_init(bar(B_PEMPTY), 1);
     mbar_init(bar(B_DRAIN), 1);
     misc[1] = 0u;
@@ -513,9 +519,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ----------------------------------------------------------- softmax ---
-    const int r = threadIdx.x - 128;             // row = TMEM lane
+    // Two warpgroups share every row: warpgroup sg handles key tile sg of each
+    // 128-key S block (columns [64 sg, 64 sg + 64)) and O columns
+    // [sg D/2, (sg+1) D/2). The row max is exchanged through shared memory.
+    const int sg = (warp - 4) >> 2;                // 0 or 1
+    const int r = (warp & 3) * 32 + lane;          // row = TMEM lane
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     const uint32_t my_bit = r < 64 ? 1u : 2u;
+    float* mpart = reinterpret_cast<float*>(smem + L::oXchg);   // [2 buffers][2 groups][128]
+    float* lpart = mpart + 2 * 2 * 128;                          // [2 groups][128]
     uint32_t g = 0;
     uint32_t pv_waited = 0;                       // PV completions consumed
     bool ok = true;
@@ -527,108 +539,132 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (inf.end) break;
       const uint32_t* list = lists + slot * prm.list_cap;
       const int nblk = (inf.n_entries + 1) >> 1;
+      // m: running max (log2 units) used for P; it is raised only when the
+      // block max exceeds it by more than kLazy, so P stays below 2^kLazy.
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < nblk; ++j, ++g) {
         const int sb = g & 1;
         ok = wait_bar(bar(B_SFULL0 + sb), (g >> 1) & 1, abort_flag, gerr);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + sb * 128 + lane_off + 32 * c, sr[c]);
+        uint32_t sr[2][32];
+        tmem_ld32(tS + sb * 128 + lane_off + 64 * sg, sr[0]);
+        tmem_ld32(tS + sb * 128 + lane_off + 64 * sg + 32, sr[1]);
         tmem_wait_ld(sr[0]);
         reg_fence(sr[1]);
-        reg_fence(sr[2]);
-        reg_fence(sr[3]);
-        float s[128];
-#pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
         tc_fence_before();
         mbar_arrive(bar(B_SFREE0 + sb));
-        const uint32_t ea = list[2 * j];
-        const uint32_t eb = 2 * j + 1 < inf.n_entries ? list[2 * j + 1] : 0u;
-        const int ca = ((ea >> 16) & my_bit) ? int(ea >> 24) : 0;   // valid keys of tile a for this row
-        const int cb = ((eb >> 16) & my_bit) ? int(eb >> 24) : 0;
+        const int e_idx = 2 * j + sg;
+        const uint32_t e = e_idx < inf.n_entries ? list[e_idx] : 0u;
+        const int cnt = ((e >> 16) & my_bit) ? int(e >> 24) : 0;   // valid keys of my tile for my row
+        float x[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sr[c >> 5][c & 31]) * prm.scale_log2;
         float mx = -INFINITY;
+        if (cnt == 64) {
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          if (c < ca) mx = fmaxf(mx, s[c]);
-          if (c < cb) mx = fmaxf(mx, s[64 + c]);
-        }
-        const float m_new = fmaxf(m, mx * prm.scale_log2);
-        const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        // a row that has seen no valid key yet holds O = 0 and l = 0: nothing to rescale
-        const float alpha = m == -INFINITY ? 1.f : ex2(m - m_use);
-        float rs = 0.f;
+          for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], x[c]);
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        } else if (cnt > 0) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float pa = c < ca ? ex2(fmaf(s[c], prm.scale_log2, -m_use)) : 0.f;
-          const float pb = c < cb ? ex2(fmaf(s[64 + c], prm.scale_log2, -m_use)) : 0.f;
-          s[c] = pa;
-          s[64 + c] = pb;
-          rs += pa + pb;
+          for (int c = 0; c < 64; ++c)
+            if (c < cnt) mx = fmaxf(mx, x[c]);
         }
-        l = l * alpha + rs;
-        m = m_new;
+        // row max across the two warpgroups
+        mpart[(sb * 2 + sg) * 128 + r] = mx;
+        mbar_arrive(bar(B_MX0 + sb));
+        ok = wait_bar(bar(B_MX0 + sb), (g >> 1) & 1, abort_flag, gerr);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        const float mrow = fmaxf(mpart[(sb * 2 + 0) * 128 + r], mpart[(sb * 2 + 1) * 128 + r]);
+        float alpha = 1.f;
+        if (mrow > m + kLazy) {                    // also taken when m is still -inf
+          alpha = m == -INFINITY ? 1.f : ex2(m - mrow);
+          m = mrow;
+        }
+        const float m_use = m == -INFINITY ? 0.f : m;
+        float rs0 = 0.f, rs1 = 0.f;
+        if (cnt == 64) {
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            x[c] = ex2(x[c] - m_use);
+            x[c + 1] = ex2(x[c + 1] - m_use);
+            rs0 += x[c];
+            rs1 += x[c + 1];
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            x[c] = c < cnt ? ex2(x[c] - m_use) : 0.f;
+            rs0 += x[c];
+          }
+        }
+        l = l * alpha + (rs0 + rs1);
         // the previous PV must be done: it reads the P buffer and writes O
         if (g > 0 && pv_waited < g) {
           ok = wait_bar(bar(B_PEMPTY), (g - 1) & 1, abort_flag, gerr);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           pv_waited = g;
         }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
-          const float a = j > 0 ? alpha : 1.f;
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t orr[32];
-            tmem_ld32(tO + lane_off + 32 * c, orr);
-            tmem_wait_ld(orr);
-            float o[32];
+        // my 64 P values -> smem key half sg, bf16, K-major 128B swizzle
+        // (16-byte chunk c of row r lands at chunk c ^ (r & 7))
+        uint8_t* prow = smem + L::oP + sg * L::kHalfBytes + r * 128;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]) * a;
-            tmem_st32(tO + lane_off + 32 * c, o);
-          }
-          tmem_wait_st();
-        }
-        // P row -> smem, bf16, K-major 128B swizzle (16-byte chunk c of row r at c ^ (r & 7))
-        uint8_t* prow = smem + L::oP + r * 128;
-#pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-          const int half = ch >> 3, cc = ch & 7;
+        for (int ch = 0; ch < 8; ++ch) {
           uint4 pk;
-          __nv_bfloat162 t0 = __floats2bfloat162_rn(s[8 * ch + 0], s[8 * ch + 1]);
-          __nv_bfloat162 t1 = __floats2bfloat162_rn(s[8 * ch + 2], s[8 * ch + 3]);
-          __nv_bfloat162 t2 = __floats2bfloat162_rn(s[8 * ch + 4], s[8 * ch + 5]);
-          __nv_bfloat162 t3 = __floats2bfloat162_rn(s[8 * ch + 6], s[8 * ch + 7]);
+          __nv_bfloat162 t0 = __floats2bfloat162_rn(x[8 * ch + 0], x[8 * ch + 1]);
+          __nv_bfloat162 t1 = __floats2bfloat162_rn(x[8 * ch + 2], x[8 * ch + 3]);
+          __nv_bfloat162 t2 = __floats2bfloat162_rn(x[8 * ch + 4], x[8 * ch + 5]);
+          __nv_bfloat162 t3 = __floats2bfloat162_rn(x[8 * ch + 6], x[8 * ch + 7]);
           pk.x = *reinterpret_cast<uint32_t*>(&t0);
           pk.y = *reinterpret_cast<uint32_t*>(&t1);
           pk.z = *reinterpret_cast<uint32_t*>(&t2);
           pk.w = *reinterpret_cast<uint32_t*>(&t3);
-          *reinterpret_cast<uint4*>(prow + half * L::kHalfBytes + ((cc ^ (r & 7)) << 4)) = pk;
+          *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = pk;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
+          const float a = j > 0 ? alpha : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t orr[32];
+            const uint32_t col = tO + lane_off + sg * (D / 2) + 32 * c;
+            tmem_ld32(col, orr);
+            tmem_wait_ld(orr);
+            float o[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]) * a;
+            tmem_st32(col, o);
+          }
+          tmem_wait_st();
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
         mbar_arrive(bar(B_PFULL));
       }
       if (!ok) break;
-      // epilogue: final O after the last PV
+      // epilogue: final O after the last PV; the row sum is the two groups' sum
       ok = wait_bar(bar(B_PEMPTY), (g - 1) & 1, abort_flag, gerr);
       if (!__all_sync(0xffffffffu, ok)) break;
       pv_waited = g;
       tc_fence_after();
+      lpart[sg * 128 + r] = l;
+      mbar_arrive(bar(B_LX));
+      ok = wait_bar(bar(B_LX), it & 1, abort_flag, gerr);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const float lrow = lpart[r] + lpart[128 + r];
       const int tile = r < 64 ? inf.qa : inf.qb;
       const int slot_r = r & 63;
       const int rows = r < 64 ? inf.rows_a : inf.rows_b;
       const bool write = tile >= 0 && !inf.bad;
       const bool valid = write && slot_r < rows;
-      const float inv = (valid && l > 0.f) ? 1.f / l : 0.f;
+      const float inv = (valid && lrow > 0.f) ? 1.f / lrow : 0.f;
       const size_t orow = (size_t(inf.bh) * prm.nt_max + (tile >= 0 ? tile : 0)) * 64 + slot_r;
-      uint4* dst = reinterpret_cast<uint4*>(prm.out + orow * D);
+      uint4* dst = reinterpret_cast<uint4*>(prm.out + orow * D + sg * (D / 2));
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t orr[32];
-        tmem_ld32(tO + lane_off + 32 * c, orr);
+        tmem_ld32(tO + lane_off + sg * (D / 2) + 32 * c, orr);
         tmem_wait_ld(orr);
         float o[32];
 #pragma unroll
@@ -649,12 +685,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (write && prm.lse) prm.lse[orow] = valid && l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : 0.f;
+      if (write && sg == 0 && prm.lse)
+        prm.lse[orow] = valid && lrow > 0.f ? (m + __log2f(lrow)) * 0.69314718055994531f : 0.f;
       tc_fence_before();
       mbar_arrive(bar(B_LEMPTY0 + slot));
     }
   }
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

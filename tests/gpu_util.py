@@ -63,6 +63,7 @@ class GpuRun:
         self.k = list(k_per_head) if k_per_head is not None else k_list(cfg, sparsity)
         self.plan = T.Plan.from_config(cfg, sparsity, k_per_head=self.k)
         self.bufs = self.plan.allocate(with_lse=True)
+        self.bufs["op"].zero_()          # tiles past a head's own count are never written
         self.q, self.k_t, self.v = (to_device(getattr(self.inp, n)) for n in ("q", "k", "v"))
         if cfg.score_mode == "meanpool_gate":
             g = torch.from_numpy(self.inp.gate).cuda()

@@ -85,6 +85,13 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
+// A from TMEM (K-major, 16-bit elements packed two per 32-bit column), B from smem.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
 __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
       "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
@@ -131,6 +138,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {  // 
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
 }
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {  // v: 32 raw words
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -162,13 +179,11 @@ struct Smem {
   static constexpr uint32_t kQBytes = (D / 64) * kHalfBytes;       // Q pair (K-major)
   static constexpr uint32_t kKBytes = kQBytes;                     // K tile pair
   static constexpr uint32_t kVBytes = kQBytes;                     // V tile pair (MN-major)
-  static constexpr uint32_t kPBytes = 2 * kHalfBytes;              // P: 128 rows x 128 keys
   static constexpr uint32_t oQ = 0;
   static constexpr uint32_t oK = oQ + kQBytes;
   static constexpr uint32_t oV = oK + 2 * kKBytes;
-  static constexpr uint32_t oP = oV + 2 * kVBytes;
-  static constexpr uint32_t oBar = oP + kPBytes;
-  static constexpr uint32_t kNumBars = 24;
+  static constexpr uint32_t oBar = oV + 2 * kVBytes;
+  static constexpr uint32_t kNumBars = 26;
   static constexpr uint32_t oInfo = oBar + kNumBars * 8;
   static constexpr uint32_t oMisc = oInfo + 2 * sizeof(ItemInfo);  // tmem base, abort flag
   static constexpr uint32_t oXchg = oMisc + 16;                     // row max / row sum exchange
@@ -178,8 +193,8 @@ struct Smem {
 // barrier indices
 enum {
   B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1, B_VFULL0, B_VFULL1, B_VEMPTY0, B_VEMPTY1,
-  B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1, B_PFULL, B_PEMPTY, B_LFULL0, B_LFULL1, B_LEMPTY0, B_LEMPTY1,
-  B_DRAIN, B_MX0, B_MX1, B_LX
+  B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1, B_PFULL0, B_PFULL1, B_PEMPTY0, B_PEMPTY1, B_LFULL0, B_LFULL1,
+  B_LEMPTY0, B_LEMPTY1, B_DRAIN, B_MX0, B_MX1, B_LX
 };
 
 struct AttnParams {
@@ -265,10 +280,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_LFULL0 + i), 32);
       mbar_init(bar(B_LEMPTY0 + i), 256);
       mbar_init(bar(B_MX0 + i), 256);
+      mbar_init(bar(B_PFULL0 + i), 256);
+      mbar_init(bar(B_PEMPTY0 + i), 1);
     }
     mbar_init(bar(B_LX), 256);
-    mbar_init(bar(B_PFULL), 256);
-    mbar_init(bar(B_PEMPTY), 1);
     mbar_init(bar(B_DRAIN), 1);
     misc[1] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -282,8 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
-  const uint32_t tS = tmem;          // two S buffers: columns [0,128) and [128,256)
-  const uint32_t tO = tmem + 256;    // O: columns [256, 256 + D)
+  // TMEM columns: S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512).
+  // P holds bf16 pairs (two keys per 32-bit column), the A operand of O += P V.
+  const uint32_t tS = tmem;
+  const uint32_t tO = tmem + 256;
+  const uint32_t tP = tmem + 384;
 
   if (warp == 2) {
     // ------------------------------------------------ scheduler / lists ---
@@ -470,18 +488,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       auto issue_pv = [&](uint32_t gg, bool first) -> bool {
         const int st = gg & 1;
-        if (!wait_bar(bar(B_PFULL), gg & 1, abort_flag, gerr)) return false;
+        if (!wait_bar(bar(B_PFULL0 + st), (gg >> 1) & 1, abort_flag, gerr)) return false;
         if (!wait_bar(bar(B_VFULL0 + st), (gg >> 1) & 1, abort_flag, gerr)) return false;
         tc_fence_after();
         const uint32_t sv = sbase + L::oV + st * L::kVBytes;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sw128_desc(sbase + L::oP + (kk >> 2) * L::kHalfBytes + (kk & 3) * 32, 16, 1024);
+        for (int kk = 0; kk < 8; ++kk) {   // 16 keys per step: 8 TMEM columns of P
           const uint64_t bdesc = sw128_desc(sv + (kk >> 2) * (D / 64) * 8192 + (kk & 3) * 2048, 8192, 1024);
-          tc_mma(tO, a, bdesc, idPV, (first && kk == 0) ? 0u : 1u);
+          tc_mma_ts(tO, tP + st * 64 + kk * 8, bdesc, idPV, (first && kk == 0) ? 0u : 1u);
         }
         tc_commit(bar(B_VEMPTY0 + st));
-        tc_commit(bar(B_PEMPTY));
+        tc_commit(bar(B_PEMPTY0 + st));
         return true;
       };
       for (uint32_t it = 0; ok; ++it) {
@@ -529,7 +546,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* mpart = reinterpret_cast<float*>(smem + L::oXchg);   // [2 buffers][2 groups][128]
     float* lpart = mpart + 2 * 2 * 128;                          // [2 groups][128]
     uint32_t g = 0;
-    uint32_t pv_waited = 0;                       // PV completions consumed
     bool ok = true;
     for (uint32_t it = 0; ok; ++it) {
       const int slot = it & 1;
@@ -592,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             rs0 += x[c];
             rs1 += x[c + 1];
           }
-        } else {
+        } else if (cnt > 0) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
             x[c] = c < cnt ? ex2(x[c] - m_use) : 0.f;
@@ -600,30 +616,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         l = l * alpha + (rs0 + rs1);
-        // the previous PV must be done: it reads the P buffer and writes O
-        if (g > 0 && pv_waited < g) {
-          ok = wait_bar(bar(B_PEMPTY), (g - 1) & 1, abort_flag, gerr);
-          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-          pv_waited = g;
-        }
-        // my 64 P values -> smem key half sg, bf16, K-major 128B swizzle
-        // (16-byte chunk c of row r lands at chunk c ^ (r & 7))
-        uint8_t* prow = smem + L::oP + sg * L::kHalfBytes + r * 128;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint4 pk;
-          __nv_bfloat162 t0 = __floats2bfloat162_rn(x[8 * ch + 0], x[8 * ch + 1]);
-          __nv_bfloat162 t1 = __floats2bfloat162_rn(x[8 * ch + 2], x[8 * ch + 3]);
-          __nv_bfloat162 t2 = __floats2bfloat162_rn(x[8 * ch + 4], x[8 * ch + 5]);
-          __nv_bfloat162 t3 = __floats2bfloat162_rn(x[8 * ch + 6], x[8 * ch + 7]);
-          pk.x = *reinterpret_cast<uint32_t*>(&t0);
-          pk.y = *reinterpret_cast<uint32_t*>(&t1);
-          pk.z = *reinterpret_cast<uint32_t*>(&t2);
-          pk.w = *reinterpret_cast<uint32_t*>(&t3);
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = pk;
-        }
+        // P buffer sb was last read by PV(g-2)
+        ok = wait_bar(bar(B_PEMPTY0 + sb), ((g >> 1) & 1) ^ 1, abort_flag, gerr);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
+        // my 64 P values as bf16 pairs -> TMEM P buffer sb, columns [32 sg, 32 sg + 32)
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            __nv_bfloat162 t = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+            pk[i] = cnt > 0 ? *reinterpret_cast<uint32_t*>(&t) : 0u;   // tiles my row-half skips: P = 0
+          }
+          tmem_st32u(tP + lane_off + sb * 64 + sg * 32, pk);
+        }
+        // O is rescaled only after PV(g-1) has finished accumulating into it
         if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
+          ok = wait_bar(bar(B_PEMPTY0 + (sb ^ 1)), ((g - 1) >> 1) & 1, abort_flag, gerr);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          tc_fence_after();
           const float a = j > 0 ? alpha : 1.f;
 #pragma unroll 1
           for (int c = 0; c < D / 64; ++c) {
@@ -636,17 +647,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]) * a;
             tmem_st32(col, o);
           }
-          tmem_wait_st();
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_PFULL));
+        mbar_arrive(bar(B_PFULL0 + sb));
       }
       if (!ok) break;
       // epilogue: final O after the last PV; the row sum is the two groups' sum
-      ok = wait_bar(bar(B_PEMPTY), (g - 1) & 1, abort_flag, gerr);
+      ok = wait_bar(bar(B_PEMPTY0 + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, gerr);
       if (!__all_sync(0xffffffffu, ok)) break;
-      pv_waited = g;
       tc_fence_after();
       lpart[sg * 128 + r] = l;
       mbar_arrive(bar(B_LX));

@@ -155,6 +155,63 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (sm_100 FFMA2 / FADD2) and the 3-input max.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// 2^x for two values on the FMA pipe instead of the MUFU unit.
+// Cody-Waite style split x = n + f with n = round(x) (adding 1.5 * 2^23 rounds
+// to an integer held in the low mantissa bits), f in [-1/2, 1/2], 2^f from a
+// degree-4 polynomial fitted here by Remez exchange for minimum relative error
+// (max 2.7e-6 in fp32 evaluation; see fit_exp2_poly.py), and 2^n added into
+// the exponent field. x is clamped to -125 so the exponent never underflows;
+// 2^-125 stands in for 0 next to the row's largest term (>= 2^-8).
+#ifndef VSA_EXP_POLY_EVERY
+#define VSA_EXP_POLY_EVERY 8   // one pair in eight goes through the polynomial (0: none)
+#endif
+__device__ __forceinline__ void ex2_fma_pipe(float x0, float x1, float& y0, float& y1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f2pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = fadd2(x, f2pack(kRound, kRound));
+  const uint64_t n = fadd2(t, f2pack(-kRound, -kRound));
+  const uint64_t f = fadd2(x, n ^ 0x8000000080000000ull);   // x - n
+  uint64_t p = ffma2(f2pack(0.009570102207362652f, 0.009570102207362652f), f,
+                     f2pack(0.05591785907745361f, 0.05591785907745361f));
+  p = ffma2(p, f, f2pack(0.240247443318367f, 0.240247443318367f));
+  p = ffma2(p, f, f2pack(0.6931217908859253f, 0.6931217908859253f));
+  p = ffma2(p, f, f2pack(0.9999992847442627f, 0.9999992847442627f));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
 // UMMA shared-memory descriptor, 128-byte swizzle (layout type 2), version 1.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
@@ -573,20 +630,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int e_idx = 2 * j + sg;
         const uint32_t e = e_idx < inf.n_entries ? list[e_idx] : 0u;
         const int cnt = ((e >> 16) & my_bit) ? int(e >> 24) : 0;   // valid keys of my tile for my row
-        float x[64];
+        float sv[64];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sr[c >> 5][c & 31]) * prm.scale_log2;
-        float mx = -INFINITY;
-        if (cnt == 64) {
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
+        if (cnt < 64) {                            // partial or unkept tile: mask the missing keys
 #pragma unroll
-          for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], x[c]);
-          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        } else if (cnt > 0) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < cnt) mx = fmaxf(mx, x[c]);
+          for (int c = 0; c < 64; ++c) sv[c] = c < cnt ? sv[c] : -INFINITY;
         }
+        // raw row max of my 64 scores (the scale is positive, so it commutes with max)
+        float mq[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float t = fmax3(sv[16 * q], sv[16 * q + 1], sv[16 * q + 2]);
+#pragma unroll
+          for (int c = 3; c < 15; c += 2) t = fmax3(t, sv[16 * q + c], sv[16 * q + c + 1]);
+          mq[q] = fmaxf(t, sv[16 * q + 15]);
+        }
+        const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * prm.scale_log2;
         // row max across the two warpgroups
         mpart[(sb * 2 + sg) * 128 + r] = mx;
         mbar_arrive(bar(B_MX0 + sb));
@@ -599,37 +659,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = mrow;
         }
         const float m_use = m == -INFINITY ? 0.f : m;
-        float rs0 = 0.f, rs1 = 0.f;
-        if (cnt == 64) {
+        // p = 2^(s * scale * log2(e) - m), two at a time; row sum in packed pairs
+        const uint64_t c2 = f2pack(prm.scale_log2, prm.scale_log2);
+        const uint64_t nm2 = f2pack(-m_use, -m_use);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t pk[32];
+        if (cnt == 64) {                             // full tile: part of the pairs on the FMA pipe
 #pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            x[c] = ex2(x[c] - m_use);
-            x[c + 1] = ex2(x[c + 1] - m_use);
-            rs0 += x[c];
-            rs1 += x[c + 1];
+          for (int i = 0; i < 32; ++i) {
+            float x0, x1, p0, p1;
+            f2unpack(ffma2(f2pack(sv[2 * i], sv[2 * i + 1]), c2, nm2), x0, x1);
+            constexpr int kPoly = VSA_EXP_POLY_EVERY;
+            bool on_fma = false;
+            if constexpr (kPoly > 0) on_fma = i % kPoly == kPoly - 1;
+            if (on_fma) {
+              ex2_fma_pipe(x0, x1, p0, p1);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            acc[i & 3] = fadd2(acc[i & 3], f2pack(p0, p1));
+            pk[i] = bf16x2(p0, p1);
           }
-        } else if (cnt > 0) {
+        } else if (cnt > 0) {                        // partial tile: masked keys give exactly 0
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            x[c] = c < cnt ? ex2(x[c] - m_use) : 0.f;
-            rs0 += x[c];
+          for (int i = 0; i < 32; ++i) {
+            float x0, x1;
+            f2unpack(ffma2(f2pack(sv[2 * i], sv[2 * i + 1]), c2, nm2), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);   // ex2(-inf) = 0
+            acc[i & 3] = fadd2(acc[i & 3], f2pack(p0, p1));
+            pk[i] = bf16x2(p0, p1);
           }
+        } else {                                     // my row-half does not keep this tile
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pk[i] = 0u;
         }
-        l = l * alpha + (rs0 + rs1);
+        float r0, r1;
+        f2unpack(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), r0, r1);
+        l = l * alpha + (r0 + r1);
         // P buffer sb was last read by PV(g-2)
         ok = wait_bar(bar(B_PEMPTY0 + sb), ((g >> 1) & 1) ^ 1, abort_flag, gerr);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
         // my 64 P values as bf16 pairs -> TMEM P buffer sb, columns [32 sg, 32 sg + 32)
-        {
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            __nv_bfloat162 t = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-            pk[i] = cnt > 0 ? *reinterpret_cast<uint32_t*>(&t) : 0u;   // tiles my row-half skips: P = 0
-          }
-          tmem_st32u(tP + lane_off + sb * 64 + sg * 32, pk);
-        }
+        tmem_st32u(tP + lane_off + sb * 64 + sg * 32, pk);
         // O is rescaled only after PV(g-1) has finished accumulating into it
         if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
           ok = wait_bar(bar(B_PEMPTY0 + (sb ^ 1)), ((g - 1) >> 1) & 1, abort_flag, gerr);

@@ -63,6 +63,39 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# ----------------------------------------------------------- ncu traffic ----
+
+ATTN_SRC = os.path.join(ROOT, "tile_sparse_video_pack_b200", "csrc", "attn.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_kernel_traffic.txt")
+
+
+def attn_source_sha1() -> str:
+    import hashlib
+    with open(ATTN_SRC, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()
+
+
+def measured_traffic(config: str, heads: int):
+    """DRAM bytes per attention launch from the committed ncu capture, if it is of this kernel source.
+
+    The capture runs a smaller case (fewer heads) of the same workload; bytes grow
+    in proportion to the heads, so they are scaled to the benchmarked head count.
+    Returns None when the kernel changed after the capture.
+    """
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    kv = {}
+    with open(TRAFFIC_FILE) as f:
+        for ln in f:
+            if "=" in ln and not ln.startswith("#"):
+                a, b = ln.split("=", 1)
+                kv[a.strip()] = b.strip()
+    if kv.get("attn_source_sha1") != attn_source_sha1() or kv.get("config") != config:
+        return None
+    per_head = (float(kv["dram_bytes_read"]) + float(kv["dram_bytes_write"])) / float(kv["heads"])
+    return int(per_head * heads)
+
+
 # --------------------------------------------------------------- work counts --
 
 def k_list(cfg, s):
@@ -340,7 +373,7 @@ def run_ours(args, rank, world, local_rank):
     achieved = flops / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
+                "frac": round(achieved / peak, 4), "traffic": measured_traffic(args.config, cfg.heads),
                 "kernel": "attn_kernel (vsa_sparse_attn)",
                 "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
                 "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),

@@ -16,14 +16,15 @@
 // -inf. Key tiles go through smem two at a time (128 keys per step).
 //
 // Warp roles (256 threads):
-//   warp 0  TMA producer: Q pair once per block, then K / V tile pairs (2 stages)
+//   warp 0  TMA producer: Q pair once per item, then K tile pairs (2 stages)
+//   warp 3  TMA producer: V tile pairs (2 stages)
 //   warp 1  MMA issuer: S = Q K^T into TMEM (double buffered), O += P V
 //   warp 2  scheduler: fetches the next block from a global counter and builds
 //           its merged key list in smem (double buffered)
-//   warps 4-11 softmax, two warpgroups: row r (TMEM lane r) is shared by one
-//           thread of each; warpgroup g handles key tile g of every 128-key
-//           block and half of O. Online softmax in fp32 with a lazily raised
-//           running max, O rescale in TMEM, P to smem (bf16, 128B-swizzled)
+//   warps 4-11 softmax, two warpgroups: warpgroup p owns the key blocks of
+//           parity p for all 128 rows (TMEM lane = row), with its own running
+//           max, row sum and O accumulator in TMEM; P goes back to TMEM as
+//           bf16 over the consumed S columns; the epilogue merges the two
 //
 // Shared-memory operand layouts are the canonical 128-byte-swizzled UMMA
 // layouts that TMA SWIZZLE_128B writes: Q, K and P K-major, V MN-major.
@@ -244,14 +245,14 @@ struct Smem {
   static constexpr uint32_t oInfo = oBar + kNumBars * 8;
   static constexpr uint32_t oMisc = oInfo + 2 * sizeof(ItemInfo);  // tmem base, abort flag
   static constexpr uint32_t oXchg = oMisc + 16;                     // row max / row sum exchange
-  static constexpr uint32_t oList = oXchg + (2 * 2 * 128 + 2 * 128) * 4;
+  static constexpr uint32_t oList = oXchg + (2 * 128 + 2 * 128) * 4;
 };
 
 // barrier indices
 enum {
   B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1, B_VFULL0, B_VFULL1, B_VEMPTY0, B_VEMPTY1,
-  B_SFULL0, B_SFULL1, B_SFREE0, B_SFREE1, B_PFULL0, B_PFULL1, B_PEMPTY0, B_PEMPTY1, B_LFULL0, B_LFULL1,
-  B_LEMPTY0, B_LEMPTY1, B_DRAIN, B_MX0, B_MX1, B_LX
+  B_SFULL0, B_SFULL1, B_PFULL0, B_PFULL1, B_PEMPTY0, B_PEMPTY1, B_LFULL0, B_LFULL1, B_LEMPTY0, B_LEMPTY1,
+  B_OFULL, B_OFREE, B_LX, B_DRAIN
 };
 
 struct AttnParams {
@@ -333,13 +334,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_VFULL0 + i), 1);
       mbar_init(bar(B_VEMPTY0 + i), 1);
       mbar_init(bar(B_SFULL0 + i), 1);
-      mbar_init(bar(B_SFREE0 + i), 256);
       mbar_init(bar(B_LFULL0 + i), 32);
       mbar_init(bar(B_LEMPTY0 + i), 256);
-      mbar_init(bar(B_MX0 + i), 256);
-      mbar_init(bar(B_PFULL0 + i), 256);
+      mbar_init(bar(B_PFULL0 + i), 128);
       mbar_init(bar(B_PEMPTY0 + i), 1);
     }
+    mbar_init(bar(B_OFULL), 1);
+    mbar_init(bar(B_OFREE), 256);
     mbar_init(bar(B_LX), 256);
     mbar_init(bar(B_DRAIN), 1);
     misc[1] = 0u;
@@ -354,11 +355,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
-  // TMEM columns: S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512).
-  // P holds bf16 pairs (two keys per 32-bit column), the A operand of O += P V.
+  // TMEM columns: S_even [0,128), S_odd [128,256), O_even [256,256+D), O_odd [384,384+D).
+  // Even key blocks go through S_even into O_even, odd ones through S_odd into
+  // O_odd; the two partial results are merged once per work item. P (bf16
+  // pairs, two keys per 32-bit column) is written over the S columns it was
+  // computed from: keys 0-63 at columns [0,32), keys 64-127 at [64,96) of the
+  // buffer. The next S MMA into a buffer is issued after the PV MMA that reads
+  // its P, and one thread's tcgen05.mma operations execute in issue order.
   const uint32_t tS = tmem;
   const uint32_t tO = tmem + 256;
-  const uint32_t tP = tmem + 384;
 
   if (warp == 2) {
     // ------------------------------------------------ scheduler / lists ---
@@ -477,11 +482,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       mbar_arrive(bar(B_LFULL0 + slot));
     }
-  } else if (warp == 0) {
-    // ---------------------------------------------------------- producer ---
+  } else if (warp == 0 || warp == 3) {
+    // --------------------------------------------------------- producers ---
+    // warp 0: the Q pair of every item and the K tile pairs; warp 3: the V tile
+    // pairs. Separate threads, so a K load never queues behind a V load that
+    // is waiting for its stage to be released by a PV MMA.
     if (lane == 0) {
-      uint32_t g = 0;         // running key-block counter
-      uint32_t issuedQ = 0;   // Q loads issued
+      const bool is_k = warp == 0;
+      const CUtensorMap* map = is_k ? &tk : &tv;
+      const int full0 = is_k ? B_KFULL0 : B_VFULL0;
+      const int empty0 = is_k ? B_KEMPTY0 : B_VEMPTY0;
+      uint32_t g = 0;          // key blocks issued
+      uint32_t issuedQ = 0;    // Q loads issued
       for (uint32_t it = 0;; ++it) {
         const int slot = it & 1;
         if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr)) break;
@@ -489,50 +501,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (inf.end) break;
         const uint32_t* list = lists + slot * prm.list_cap;
         const int row_base = inf.bh * prm.nt_max;
-        if (!wait_bar(bar(B_QEMPTY), (it & 1) ^ 1, abort_flag, gerr)) break;
-        mbar_expect_tx(bar(B_QFULL), 2 * (D / 64) * kTileBytes);
-        const int qb = inf.qb >= 0 ? inf.qb : inf.qa;
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_2d(sbase + L::oQ + c * L::kHalfBytes, &tq, 64 * c, (row_base + inf.qa) * 64, bar(B_QFULL));
-          tma_load_2d(sbase + L::oQ + c * L::kHalfBytes + 8192, &tq, 64 * c, (row_base + qb) * 64, bar(B_QFULL));
+        if (is_k) {
+          if (!wait_bar(bar(B_QEMPTY), (it & 1) ^ 1, abort_flag, gerr)) break;
+          mbar_expect_tx(bar(B_QFULL), 2 * (D / 64) * kTileBytes);
+          const int qb = inf.qb >= 0 ? inf.qb : inf.qa;
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(sbase + L::oQ + c * L::kHalfBytes, &tq, 64 * c, (row_base + inf.qa) * 64, bar(B_QFULL));
+            tma_load_2d(sbase + L::oQ + c * L::kHalfBytes + 8192, &tq, 64 * c, (row_base + qb) * 64, bar(B_QFULL));
+          }
+          ++issuedQ;
         }
-        ++issuedQ;
         const int nblk = (inf.n_entries + 1) >> 1;
         bool ok = true;
-        for (int j = 0; j < nblk && ok; ++j, ++g) {
+        for (int j = 0; j < nblk; ++j) {
           const int st = g & 1;
-          const uint32_t ph = (g >> 1) & 1;
           const int ta = int(list[2 * j] & 0xFFFFu);
           const int tb = 2 * j + 1 < inf.n_entries ? int(list[2 * j + 1] & 0xFFFFu) : ta;
-          ok = wait_bar(bar(B_KEMPTY0 + st), ph ^ 1, abort_flag, gerr);
-          if (!ok) break;
-          mbar_expect_tx(bar(B_KFULL0 + st), 2 * (D / 64) * kTileBytes);
-          const uint32_t sk = sbase + L::oK + st * L::kKBytes;
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(sk + c * L::kHalfBytes, &tk, 64 * c, (row_base + ta) * 64, bar(B_KFULL0 + st));
-            tma_load_2d(sk + c * L::kHalfBytes + 8192, &tk, 64 * c, (row_base + tb) * 64, bar(B_KFULL0 + st));
+          if (!(ok = wait_bar(bar(empty0 + st), ((g >> 1) & 1) ^ 1, abort_flag, gerr))) break;
+          mbar_expect_tx(bar(full0 + st), 2 * (D / 64) * kTileBytes);
+          if (is_k) {   // K-major: tile a rows 0-63, tile b rows 64-127 of each 64-column half
+            const uint32_t sk = sbase + L::oK + st * L::kKBytes;
+            for (int c = 0; c < D / 64; ++c) {
+              tma_load_2d(sk + c * L::kHalfBytes, map, 64 * c, (row_base + ta) * 64, bar(full0 + st));
+              tma_load_2d(sk + c * L::kHalfBytes + 8192, map, 64 * c, (row_base + tb) * 64, bar(full0 + st));
+            }
+          } else {      // MN-major: tile a then tile b, each as D/64 boxes of 64 keys x 64 columns
+            const uint32_t sv = sbase + L::oV + st * L::kVBytes;
+            for (int c = 0; c < D / 64; ++c) {
+              tma_load_2d(sv + c * 8192, map, 64 * c, (row_base + ta) * 64, bar(full0 + st));
+              tma_load_2d(sv + (D / 64) * 8192 + c * 8192, map, 64 * c, (row_base + tb) * 64, bar(full0 + st));
+            }
           }
-          ok = wait_bar(bar(B_VEMPTY0 + st), ph ^ 1, abort_flag, gerr);
-          if (!ok) {
-            drain_wait(bar(B_KFULL0 + st), ph);
-            break;
-          }
-          mbar_expect_tx(bar(B_VFULL0 + st), 2 * (D / 64) * kTileBytes);
-          const uint32_t sv = sbase + L::oV + st * L::kVBytes;
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(sv + c * 8192, &tv, 64 * c, (row_base + ta) * 64, bar(B_VFULL0 + st));
-            tma_load_2d(sv + (D / 64) * 8192 + c * 8192, &tv, 64 * c, (row_base + tb) * 64, bar(B_VFULL0 + st));
-          }
+          ++g;
         }
         if (!ok) break;
       }
       if (*abort_flag) {
-        // let every copy this CTA issued land before shared memory is released
-        drain_wait(bar(B_QFULL), (issuedQ - 1) & 1);
-        for (uint32_t gg = (g >= 2 ? g - 2 : 0); gg < g; ++gg) {
-          drain_wait(bar(B_KFULL0 + (gg & 1)), (gg >> 1) & 1);
-          drain_wait(bar(B_VFULL0 + (gg & 1)), (gg >> 1) & 1);
-        }
+        // let every copy this thread issued land before shared memory is released
+        if (is_k && issuedQ) drain_wait(bar(B_QFULL), (issuedQ - 1) & 1);
+        for (uint32_t gg = (g >= 2 ? g - 2 : 0); gg < g; ++gg) drain_wait(bar(full0 + (gg & 1)), (gg >> 1) & 1);
       }
     }
     __syncwarp();
@@ -541,21 +548,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idPV = idesc_bf16(128, D, 0, 1);
-      uint32_t g = 0;
+      // descriptors of the stage bases; a k-step adds (byte offset >> 4) to the start address
+      const uint64_t dq = sw128_desc(sbase + L::oQ, 16, 1024);
+      const uint64_t dk[2] = {sw128_desc(sbase + L::oK, 16, 1024), sw128_desc(sbase + L::oK + L::kKBytes, 16, 1024)};
+      const uint64_t dv[2] = {sw128_desc(sbase + L::oV, 8192, 1024),
+                              sw128_desc(sbase + L::oV + L::kVBytes, 8192, 1024)};
+      uint32_t g = 0;            // key blocks so far (K / V stage ring)
+      uint32_t npv[2] = {0, 0};  // PV MMAs issued per parity (phases of P_FULL)
       bool ok = true;
-      auto issue_pv = [&](uint32_t gg, bool first) -> bool {
+      // O_p += P V for block gg (global) = block jj of the item, parity p = jj & 1
+      auto issue_pv = [&](uint32_t gg, int jj, uint32_t it) -> bool {
         const int st = gg & 1;
-        if (!wait_bar(bar(B_PFULL0 + st), (gg >> 1) & 1, abort_flag, gerr)) return false;
+        const int p = jj & 1;
+        if (jj == 0 && !wait_bar(bar(B_OFREE), (it & 1) ^ 1, abort_flag, gerr)) return false;
+        if (!wait_bar(bar(B_PFULL0 + p), npv[p] & 1, abort_flag, gerr)) return false;
         if (!wait_bar(bar(B_VFULL0 + st), (gg >> 1) & 1, abort_flag, gerr)) return false;
+        ++npv[p];
         tc_fence_after();
-        const uint32_t sv = sbase + L::oV + st * L::kVBytes;
+        const uint32_t o = tO + p * 128;
+        const uint32_t pcol = tS + p * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // 16 keys per step: 8 TMEM columns of P
-          const uint64_t bdesc = sw128_desc(sv + (kk >> 2) * (D / 64) * 8192 + (kk & 3) * 2048, 8192, 1024);
-          tc_mma_ts(tO, tP + st * 64 + kk * 8, bdesc, idPV, (first && kk == 0) ? 0u : 1u);
+          const uint32_t boff = ((kk >> 2) * (D / 64) * 8192 + (kk & 3) * 2048) >> 4;
+          tc_mma_ts(o, pcol + (kk >> 2) * 64 + (kk & 3) * 8, dv[st] + boff, idPV, (jj < 2 && kk == 0) ? 0u : 1u);
         }
         tc_commit(bar(B_VEMPTY0 + st));
-        tc_commit(bar(B_PEMPTY0 + st));
+        tc_commit(bar(B_PEMPTY0 + p));
         return true;
       };
       for (uint32_t it = 0; ok; ++it) {
@@ -565,26 +583,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (inf.end) break;
         if (!wait_bar(bar(B_QFULL), it & 1, abort_flag, gerr)) break;
         const int nblk = (inf.n_entries + 1) >> 1;
-        const uint32_t g0 = g;
         for (int j = 0; j < nblk; ++j, ++g) {
           const int st = g & 1;
           if (!(ok = wait_bar(bar(B_KFULL0 + st), (g >> 1) & 1, abort_flag, gerr))) break;
-          if (!(ok = wait_bar(bar(B_SFREE0 + st), ((g >> 1) & 1) ^ 1, abort_flag, gerr))) break;
           tc_fence_after();
-          const uint32_t sk = sbase + L::oK + st * L::kKBytes;
+          const int p = j & 1;     // S buffer of this block's parity within the item
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
-            tc_mma(tS + st * 128, sw128_desc(sbase + L::oQ + off, 16, 1024), sw128_desc(sk + off, 16, 1024), idS,
-                   kk > 0 ? 1u : 0u);
+            const uint32_t off = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
+            tc_mma(tS + p * 128, dq + off, dk[st] + off, idS, kk > 0 ? 1u : 0u);
           }
-          tc_commit(bar(B_SFULL0 + st));
+          tc_commit(bar(B_SFULL0 + p));
           tc_commit(bar(B_KEMPTY0 + st));
           if (j == nblk - 1) tc_commit(bar(B_QEMPTY));
-          if (j > 0 && !(ok = issue_pv(g - 1, g - 1 == g0))) break;
+          if (j > 0 && !(ok = issue_pv(g - 1, j - 1, it))) break;
         }
         if (!ok) break;
-        if (!(ok = issue_pv(g - 1, g - 1 == g0))) break;
+        if (!(ok = issue_pv(g - 1, nblk - 1, it))) break;
+        tc_commit(bar(B_OFULL));
       }
       // nothing of ours may still run on the tensor core when TMEM is freed
       tc_commit(bar(B_DRAIN));
@@ -593,16 +609,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ----------------------------------------------------------- softmax ---
-    // Two warpgroups share every row: warpgroup sg handles key tile sg of each
-    // 128-key S block (columns [64 sg, 64 sg + 64)) and O columns
-    // [sg D/2, (sg+1) D/2). The row max is exchanged through shared memory.
-    const int sg = (warp - 4) >> 2;                // 0 or 1
-    const int r = (warp & 3) * 32 + lane;          // row = TMEM lane
+    // Warpgroup par (0 or 1) handles the even or odd key blocks of every item
+    // for all 128 rows (row = TMEM lane), with its own running max m, row sum
+    // l and accumulator O_par. The running max is raised only when a block
+    // exceeds it by more than kLazy (log2 units), so P < 2^kLazy and O_par is
+    // rarely rescaled. The epilogue merges (m, l, O) of both warpgroups.
+    const int par = (warp - 4) >> 2;
+    const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     const uint32_t my_bit = r < 64 ? 1u : 2u;
-    float* mpart = reinterpret_cast<float*>(smem + L::oXchg);   // [2 buffers][2 groups][128]
-    float* lpart = mpart + 2 * 2 * 128;                          // [2 groups][128]
-    uint32_t g = 0;
+    const uint32_t tSp = tS + par * 128 + lane_off;
+    const uint32_t tOp = tO + par * 128 + lane_off;
+    float* xm = reinterpret_cast<float*>(smem + L::oXchg);   // [2][128] row max (log2 units)
+    float* xl = xm + 2 * 128;                               // [2][128] row sum
+    const uint64_t c2 = f2pack(prm.scale_log2, prm.scale_log2);
+    uint32_t nb = 0;           // blocks of this parity so far (phases of S_FULL / P_FULL / P_EMPTY)
     bool ok = true;
     for (uint32_t it = 0; ok; ++it) {
       const int slot = it & 1;
@@ -612,167 +633,181 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (inf.end) break;
       const uint32_t* list = lists + slot * prm.list_cap;
       const int nblk = (inf.n_entries + 1) >> 1;
-      // m: running max (log2 units) used for P; it is raised only when the
-      // block max exceeds it by more than kLazy, so P stays below 2^kLazy.
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < nblk; ++j, ++g) {
-        const int sb = g & 1;
-        ok = wait_bar(bar(B_SFULL0 + sb), (g >> 1) & 1, abort_flag, gerr);
+      for (int j = par; j < nblk; j += 2, ++nb) {
+        ok = wait_bar(bar(B_SFULL0 + par), nb & 1, abort_flag, gerr);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sr[2][32];
-        tmem_ld32(tS + sb * 128 + lane_off + 64 * sg, sr[0]);
-        tmem_ld32(tS + sb * 128 + lane_off + 64 * sg + 32, sr[1]);
-        tmem_wait_ld(sr[0]);
-        reg_fence(sr[1]);
-        tc_fence_before();
-        mbar_arrive(bar(B_SFREE0 + sb));
-        const int e_idx = 2 * j + sg;
-        const uint32_t e = e_idx < inf.n_entries ? list[e_idx] : 0u;
-        const int cnt = ((e >> 16) & my_bit) ? int(e >> 24) : 0;   // valid keys of my tile for my row
-        float sv[64];
+        int cnt[2];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
-        if (cnt < 64) {                            // partial or unkept tile: mask the missing keys
-#pragma unroll
-          for (int c = 0; c < 64; ++c) sv[c] = c < cnt ? sv[c] : -INFINITY;
+        for (int h = 0; h < 2; ++h) {
+          const int ei = 2 * j + h;
+          const uint32_t e = ei < inf.n_entries ? list[ei] : 0u;
+          cnt[h] = ((e >> 16) & my_bit) ? int(e >> 24) : 0;   // valid keys of tile h for my row
         }
-        // raw row max of my 64 scores (the scale is positive, so it commutes with max)
-        float mq[4];
+        // 64 scores of tile h (columns [64h, 64h+64)); missing keys of a partial tile -> -inf
+        auto load_tile = [&](int h, float (&sv)[64]) {
+          uint32_t sr[2][32];
+          tmem_ld32(tSp + 64 * h, sr[0]);
+          tmem_ld32(tSp + 64 * h + 32, sr[1]);
+          tmem_wait_ld(sr[0]);
+          reg_fence(sr[1]);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float t = fmax3(sv[16 * q], sv[16 * q + 1], sv[16 * q + 2]);
+          for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
+          if (cnt[h] < 64) {
 #pragma unroll
-          for (int c = 3; c < 15; c += 2) t = fmax3(t, sv[16 * q + c], sv[16 * q + c + 1]);
-          mq[q] = fmaxf(t, sv[16 * q + 15]);
+            for (int c = 0; c < 64; ++c) sv[c] = c < cnt[h] ? sv[c] : -INFINITY;
+          }
+        };
+        // pass 1: raw row max over both tiles
+        float mx = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (cnt[h] == 0) continue;
+          float sv[64];
+          load_tile(h, sv);
+          float mq[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float t = fmax3(sv[16 * q], sv[16 * q + 1], sv[16 * q + 2]);
+#pragma unroll
+            for (int c = 3; c < 15; c += 2) t = fmax3(t, sv[16 * q + c], sv[16 * q + c + 1]);
+            mq[q] = fmaxf(t, sv[16 * q + 15]);
+          }
+          mx = fmax3(mx, fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
         }
-        const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * prm.scale_log2;
-        // row max across the two warpgroups
-        mpart[(sb * 2 + sg) * 128 + r] = mx;
-        mbar_arrive(bar(B_MX0 + sb));
-        ok = wait_bar(bar(B_MX0 + sb), (g >> 1) & 1, abort_flag, gerr);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        const float mrow = fmaxf(mpart[(sb * 2 + 0) * 128 + r], mpart[(sb * 2 + 1) * 128 + r]);
+        mx *= prm.scale_log2;                         // the scale is positive: it commutes with max
         float alpha = 1.f;
-        if (mrow > m + kLazy) {                    // also taken when m is still -inf
-          alpha = m == -INFINITY ? 1.f : ex2(m - mrow);
-          m = mrow;
+        if (mx > m + kLazy) {                         // also taken when m is still -inf
+          alpha = m == -INFINITY ? 1.f : ex2(m - mx);
+          m = mx;
         }
         const float m_use = m == -INFINITY ? 0.f : m;
-        // p = 2^(s * scale * log2(e) - m), two at a time; row sum in packed pairs
-        const uint64_t c2 = f2pack(prm.scale_log2, prm.scale_log2);
         const uint64_t nm2 = f2pack(-m_use, -m_use);
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-        uint32_t pk[32];
-        if (cnt == 64) {                             // full tile: part of the pairs on the FMA pipe
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float x0, x1, p0, p1;
-            f2unpack(ffma2(f2pack(sv[2 * i], sv[2 * i + 1]), c2, nm2), x0, x1);
-            constexpr int kPoly = VSA_EXP_POLY_EVERY;
-            bool on_fma = false;
-            if constexpr (kPoly > 0) on_fma = i % kPoly == kPoly - 1;
-            if (on_fma) {
-              ex2_fma_pipe(x0, x1, p0, p1);
-            } else {
-              p0 = ex2(x0);
-              p1 = ex2(x1);
-            }
-            acc[i & 3] = fadd2(acc[i & 3], f2pack(p0, p1));
-            pk[i] = bf16x2(p0, p1);
-          }
-        } else if (cnt > 0) {                        // partial tile: masked keys give exactly 0
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float x0, x1;
-            f2unpack(ffma2(f2pack(sv[2 * i], sv[2 * i + 1]), c2, nm2), x0, x1);
-            const float p0 = ex2(x0), p1 = ex2(x1);   // ex2(-inf) = 0
-            acc[i & 3] = fadd2(acc[i & 3], f2pack(p0, p1));
-            pk[i] = bf16x2(p0, p1);
-          }
-        } else {                                     // my row-half does not keep this tile
-#pragma unroll
-          for (int i = 0; i < 32; ++i) pk[i] = 0u;
-        }
-        float r0, r1;
-        f2unpack(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), r0, r1);
-        l = l * alpha + (r0 + r1);
-        // P buffer sb was last read by PV(g-2)
-        ok = wait_bar(bar(B_PEMPTY0 + sb), ((g >> 1) & 1) ^ 1, abort_flag, gerr);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after();
-        // my 64 P values as bf16 pairs -> TMEM P buffer sb, columns [32 sg, 32 sg + 32)
-        tmem_st32u(tP + lane_off + sb * 64 + sg * 32, pk);
-        // O is rescaled only after PV(g-1) has finished accumulating into it
-        if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
-          ok = wait_bar(bar(B_PEMPTY0 + (sb ^ 1)), ((g - 1) >> 1) & 1, abort_flag, gerr);
+        // O_par holds earlier blocks of this parity at the old max: rescale it
+        // once the PV of the previous block of this parity has finished
+        if (__any_sync(0xffffffffu, j >= 2 && alpha != 1.f)) {
+          ok = wait_bar(bar(B_PEMPTY0 + par), (nb & 1) ^ 1, abort_flag, gerr);   // PV of block nb-1
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
-          const float a = j > 0 ? alpha : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < D / 64; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t orr[32];
-            const uint32_t col = tO + lane_off + sg * (D / 2) + 32 * c;
-            tmem_ld32(col, orr);
+            tmem_ld32(tOp + 32 * c, orr);
             tmem_wait_ld(orr);
             float o[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]) * a;
-            tmem_st32(col, o);
+            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]) * alpha;
+            tmem_st32(tOp + 32 * c, o);
           }
         }
+        // pass 2: P = 2^(s * scale * log2(e) - m) as bf16 pairs, written over
+        // consumed S columns: tile 0's P to [0,32), tile 1's to [64,96)
+        uint64_t acc[2] = {0ull, 0ull};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+          if (cnt[h] == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pk[i] = 0u;
+          } else {
+            float sv[64];
+            load_tile(h, sv);
+            if (cnt[h] == 64) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                float x0, x1, p0, p1;
+                f2unpack(ffma2(f2pack(sv[2 * i], sv[2 * i + 1]), c2, nm2), x0, x1);
+                constexpr int kPoly = VSA_EXP_POLY_EVERY;
+                bool on_fma = false;
+                if constexpr (kPoly > 0) on_fma = i % kPoly == kPoly - 1;
+                if (on_fma) {
+                  ex2_fma_pipe(x0, x1, p0, p1);
+                } else {
+                  p0 = ex2(x0);
+                  p1 = ex2(x1);
+                }
+                acc[i & 1] = fadd2(acc[i & 1], f2pack(p0, p1));
+                pk[i] = bf16x2(p0, p1);
+              }
+            } else {                                   // partial tile: masked keys give exactly 0
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                float x0, x1;
+                f2unpack(ffma2(f2pack(sv[2 * i], sv[2 * i + 1]), c2, nm2), x0, x1);
+                const float p0 = ex2(x0), p1 = ex2(x1);   // ex2(-inf) = 0
+                acc[i & 1] = fadd2(acc[i & 1], f2pack(p0, p1));
+                pk[i] = bf16x2(p0, p1);
+              }
+            }
+          }
+          tmem_st32u(tSp + 64 * h, pk);
+        }
+        float r0, r1;
+        f2unpack(fadd2(acc[0], acc[1]), r0, r1);
+        l = l * alpha + (r0 + r1);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_PFULL0 + sb));
+        mbar_arrive(bar(B_PFULL0 + par));
       }
       if (!ok) break;
-      // epilogue: final O after the last PV; the row sum is the two groups' sum
-      ok = wait_bar(bar(B_PEMPTY0 + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, gerr);
+      // epilogue: both partial results are final once the item's last PV is done
+      ok = wait_bar(bar(B_OFULL), it & 1, abort_flag, gerr);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      lpart[sg * 128 + r] = l;
+      xm[par * 128 + r] = m;
+      xl[par * 128 + r] = l;
       mbar_arrive(bar(B_LX));
       ok = wait_bar(bar(B_LX), it & 1, abort_flag, gerr);
       if (!__all_sync(0xffffffffu, ok)) break;
-      const float lrow = lpart[r] + lpart[128 + r];
+      const float m0 = xm[r], m1 = xm[128 + r], l0 = xl[r], l1 = xl[128 + r];
+      const float mt = fmaxf(m0, m1);
+      const bool has_odd = nblk >= 2;
+      const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - mt);
+      const float f1 = (!has_odd || m1 == -INFINITY) ? 0.f : ex2(m1 - mt);
+      const float lrow = l0 * f0 + l1 * f1;
       const int tile = r < 64 ? inf.qa : inf.qb;
       const int slot_r = r & 63;
       const int rows = r < 64 ? inf.rows_a : inf.rows_b;
       const bool write = tile >= 0 && !inf.bad;
       const bool valid = write && slot_r < rows;
       const float inv = (valid && lrow > 0.f) ? 1.f / lrow : 0.f;
+      const float w0 = f0 * inv, w1 = f1 * inv;
       const size_t orow = (size_t(inf.bh) * prm.nt_max + (tile >= 0 ? tile : 0)) * 64 + slot_r;
-      uint4* dst = reinterpret_cast<uint4*>(prm.out + orow * D + sg * (D / 2));
+      // this warpgroup writes O columns [par D/2, (par+1) D/2) of its rows
+      uint4* dst = reinterpret_cast<uint4*>(prm.out + orow * D + par * (D / 2));
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
-        uint32_t orr[32];
-        tmem_ld32(tO + lane_off + sg * (D / 2) + 32 * c, orr);
-        tmem_wait_ld(orr);
+        const uint32_t col = lane_off + par * (D / 2) + 32 * c;
+        uint32_t a0[32], a1[32];
+        tmem_ld32(tO + col, a0);
+        if (has_odd) tmem_ld32(tO + 128 + col, a1);
+        tmem_wait_ld(a0);
+        if (has_odd) reg_fence(a1);
         float o[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]);
+        for (int i = 0; i < 32; ++i)
+          o[i] = __uint_as_float(a0[i]) * w0 + (has_odd ? __uint_as_float(a1[i]) * w1 : 0.f);
         if (write) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint4 pk;
-            __nv_bfloat162 t0 = __floats2bfloat162_rn(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
-            __nv_bfloat162 t1 = __floats2bfloat162_rn(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
-            __nv_bfloat162 t2 = __floats2bfloat162_rn(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
-            __nv_bfloat162 t3 = __floats2bfloat162_rn(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
-            pk.x = *reinterpret_cast<uint32_t*>(&t0);
-            pk.y = *reinterpret_cast<uint32_t*>(&t1);
-            pk.z = *reinterpret_cast<uint32_t*>(&t2);
-            pk.w = *reinterpret_cast<uint32_t*>(&t3);
-            dst[c * 4 + q] = pk;
+            uint4 pkq;
+            pkq.x = bf16x2(o[8 * q + 0], o[8 * q + 1]);
+            pkq.y = bf16x2(o[8 * q + 2], o[8 * q + 3]);
+            pkq.z = bf16x2(o[8 * q + 4], o[8 * q + 5]);
+            pkq.w = bf16x2(o[8 * q + 6], o[8 * q + 7]);
+            dst[c * 4 + q] = pkq;
           }
         }
       }
-      if (write && sg == 0 && prm.lse)
-        prm.lse[orow] = valid && lrow > 0.f ? (m + __log2f(lrow)) * 0.69314718055994531f : 0.f;
+      if (write && par == 0 && prm.lse)
+        prm.lse[orow] = valid && lrow > 0.f ? (mt + __log2f(lrow)) * 0.69314718055994531f : 0.f;
       tc_fence_before();
+      mbar_arrive(bar(B_OFREE));
       mbar_arrive(bar(B_LEMPTY0 + slot));
     }
   }
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -160,6 +160,30 @@ VSA_API vsa_status vsa_tile_score(vsa_plan* plan, const void* qp, const void* kp
                           const float* proj_q, const float* proj_k, float* scores,
                           void* workspace, void* stream);
 
+/* The a2-a4 score stage of vsa_tile_score with its scratch in a fixed device
+ * array owned by the library instead of a caller workspace, for callers that
+ * may not allocate device memory while they run the layer: code under another
+ * framework's memory planner or fixed arena, plugins that must not call
+ * cudaMalloc (it can synchronise the device, or fail part-way through a step),
+ * latency-critical loops. The pages describe no such call; it has no
+ * counterpart there.
+ *  - The scratch is a 32 MiB array in device memory, held by every GPU that
+ *    loads this library until the process exits. Plans whose workspace_bytes
+ *    exceed 32 MiB are rejected with VSA_ERR_UNSUPPORTED.
+ *  - The call allocates nothing. Its first call on a device looks up the
+ *    array's device address (cudaGetSymbolAddress) with that device current;
+ *    make that first call before any stream capture.
+ *  - The current device must be the plan's device (else VSA_ERR_INVALID_ARG).
+ *  - Every call on a device shares the one array, which keeps the last
+ *    call's contents (each call writes every scratch element before reading
+ *    it, so nothing needs clearing). Calls whose kernels overlap on the GPU --
+ *    on different streams, plans or threads -- race on it.
+ * Arguments, layout and results are those of vsa_tile_score without the
+ * workspace argument. */
+VSA_API vsa_status vsa_tile_score_static(vsa_plan* plan, const void* qp, const void* kp,
+                                         const float* proj_q, const float* proj_k, float* scores,
+                                         void* stream);
+
 /* a5. For every (b, h, video query tile i) keep the k_per_head[h] video key
  * tiles with the largest scores; equal scores keep the lower tile index. The
  * kept tile indices (0-based video tile ids) are written sorted ascending to

@@ -10,6 +10,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <mutex>
+
 #include "vsa_internal.h"
 
 namespace vsa {
@@ -233,3 +235,69 @@ cudaError_t launch_score(const vsa_plan* pl, const void* qp, const void* kp, con
 }
 
 }  // namespace vsa
+
+// ---------------------------------------------------------------------------
+// vsa_tile_score_static: the same score stage with its scratch (pooled and
+// projected tiles) in a fixed device array instead of a caller workspace.
+//
+// For callers that may not allocate device memory when they run the layer:
+// code called under another framework's memory planner or fixed arena, a
+// plugin that must not call cudaMalloc (it can synchronise the device or fail
+// mid-step), or a latency-critical loop where allocation is not allowed.
+// ---------------------------------------------------------------------------
+namespace vsa {
+namespace {
+
+constexpr size_t kStaticScoreScratchBytes = size_t(32) << 20;   // 32 MiB
+
+// Held by every GPU that loads this library until the process exits. Each
+// call overwrites every element it later reads, so nothing needs clearing.
+__device__ __align__(256) unsigned char g_static_score_scratch[kStaticScoreScratchBytes];
+
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_addr[256] = {};   // device address per device ordinal
+
+// Device address of the scratch array on the current device. The host-side
+// symbol is only a stand-in: its device address comes from
+// cudaGetSymbolAddress, called once per device with that device current.
+cudaError_t static_scratch_address(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_score_scratch);
+    if (e != cudaSuccess) return e;
+    g_static_scratch_addr[dev] = ptr;
+  }
+  *out = g_static_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace vsa
+
+extern "C" vsa_status vsa_tile_score_static(vsa_plan* p, const void* qp, const void* kp, const float* proj_q,
+                                            const float* proj_k, float* scores, void* stream) {
+  auto fail = [&](vsa_status st) {
+    if (p) p->stats.errors++;
+    return st;
+  };
+  if (!p || !qp || !kp || !proj_q || !proj_k || !scores) return fail(VSA_ERR_INVALID_ARG);
+  const auto a16 = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; };
+  if (!a16(qp) || !a16(kp) || !a16(proj_q) || !a16(proj_k) || !a16(scores)) return fail(VSA_ERR_INVALID_ARG);
+  if (p->info.workspace_bytes > int64_t(vsa::kStaticScoreScratchBytes)) return fail(VSA_ERR_UNSUPPORTED);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(VSA_ERR_CUDA);
+  }
+  if (dev != p->device || dev < 0 || dev >= 256) return fail(VSA_ERR_INVALID_ARG);
+  void* ws = nullptr;
+  if (vsa::static_scratch_address(dev, &ws) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(VSA_ERR_CUDA);
+  }
+  p->stats.calls_score++;
+  if (vsa::launch_score(p, qp, kp, proj_q, proj_k, scores, ws, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(VSA_ERR_CUDA);
+  return VSA_OK;
+}

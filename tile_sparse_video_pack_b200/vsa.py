@@ -25,7 +25,7 @@ SCORE_MODES = {"meanpool_gate": 0, "tripool": 1}
 # every entry point declared in include/vsa.h
 EXPORTS = ("vsa_plan_create", "vsa_plan_destroy", "vsa_plan_query", "vsa_plan_get_stats", "vsa_k_from_sparsity",
            "vsa_tile_pack", "vsa_tile_score", "vsa_topk_select", "vsa_sparse_attn", "vsa_tile_unpack",
-           "vsa_layer_forward", "vsa_plan_check", "vsa_status_string")
+           "vsa_layer_forward", "vsa_plan_check", "vsa_status_string", "vsa_tile_score_static")
 
 
 class VsaDesc(ctypes.Structure):
@@ -88,6 +88,7 @@ def library() -> ctypes.CDLL:
         "vsa_layer_forward": (I32, [P] + [P] * 15),
         "vsa_plan_check": (I32, [P]),
         "vsa_status_string": (ctypes.c_char_p, [I32]),
+        "vsa_tile_score_static": (I32, [P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -236,6 +237,21 @@ class Plan:
             _ptr(scores, torch.float32, "scores", self.info.score_elems),
             _ptr(workspace, torch.uint8, "workspace", self.info.workspace_bytes), _stream(stream)),
             "vsa_tile_score")
+
+    def tile_score_static(self, qp, kp, proj_q, proj_k, scores, stream=None):
+        """tile_score with the library's fixed 32 MiB device scratch instead of a workspace.
+
+        For callers that may not allocate device memory while the layer runs.
+        Its first call on a device looks up the scratch address: make it before
+        any stream capture. Calls that overlap on the GPU share the scratch and race.
+        """
+        import torch
+        pe = self.info.packed_elems
+        _check(library().vsa_tile_score_static(
+            self._h, _ptr(qp, torch.bfloat16, "qp", pe), _ptr(kp, torch.bfloat16, "kp", pe),
+            _ptr(proj_q, torch.float32, "proj_q"), _ptr(proj_k, torch.float32, "proj_k"),
+            _ptr(scores, torch.float32, "scores", self.info.score_elems), _stream(stream)),
+            "vsa_tile_score_static")
 
     def topk_select(self, scores, idx, stream=None):
         import torch

@@ -659,60 +659,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 64; ++c) sv[c] = c < cnt[h] ? sv[c] : -INFINITY;
           }
         };
-        // pass 1: raw row max over both tiles
-        float mx = -INFINITY;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (cnt[h] == 0) continue;
-          float sv[64];
-          load_tile(h, sv);
-          float mq[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float t = fmax3(sv[16 * q], sv[16 * q + 1], sv[16 * q + 2]);
-#pragma unroll
-            for (int c = 3; c < 15; c += 2) t = fmax3(t, sv[16 * q + c], sv[16 * q + c + 1]);
-            mq[q] = fmaxf(t, sv[16 * q + 15]);
-          }
-          mx = fmax3(mx, fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-        }
-        mx *= prm.scale_log2;                         // the scale is positive: it commutes with max
-        float alpha = 1.f;
-        if (mx > m + kLazy) {                         // also taken when m is still -inf
-          alpha = m == -INFINITY ? 1.f : ex2(m - mx);
-          m = mx;
-        }
-        const float m_use = m == -INFINITY ? 0.f : m;
-        const uint64_t nm2 = f2pack(-m_use, -m_use);
-        // O_par holds earlier blocks of this parity at the old max: rescale it
-        // once the PV of the previous block of this parity has finished
-        if (__any_sync(0xffffffffu, j >= 2 && alpha != 1.f)) {
-          ok = wait_bar(bar(B_PEMPTY0 + par), (nb & 1) ^ 1, abort_flag, gerr);   // PV of block nb-1
-          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t orr[32];
-            tmem_ld32(tOp + 32 * c, orr);
-            tmem_wait_ld(orr);
-            float o[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]) * alpha;
-            tmem_st32(tOp + 32 * c, o);
-          }
-        }
-        // pass 2: P = 2^(s * scale * log2(e) - m) as bf16 pairs, written over
-        // consumed S columns: tile 0's P to [0,32), tile 1's to [64,96)
-        uint64_t acc[2] = {0ull, 0ull};
+        // One pass per tile: P = 2^(s * scale * log2(e) - m) with the running max m
+        // (log2 units), written as bf16 pairs over consumed S columns (tile 0 ->
+        // [0,32), tile 1 -> [64,96)). Each tile's max is checked first: if it
+        // exceeds m by more than kLazy, m is raised before the tile's
+        // exponentials, and whatever was already accumulated at the old m -- the
+        // row sum, tile 0's stored P, and O_par -- is scaled by 2^(m_old - m_new).
+        float alpha_blk = 1.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
+          float a_tile = 1.f;
           if (cnt[h] == 0) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) pk[i] = 0u;
           } else {
             float sv[64];
             load_tile(h, sv);
+            float mq[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float t = fmax3(sv[16 * q], sv[16 * q + 1], sv[16 * q + 2]);
+#pragma unroll
+              for (int c = 3; c < 15; c += 2) t = fmax3(t, sv[16 * q + c], sv[16 * q + c + 1]);
+              mq[q] = fmaxf(t, sv[16 * q + 15]);
+            }
+            const float tmx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * prm.scale_log2;
+            if (tmx > m + kLazy) {                  // also taken when m is still -inf
+              a_tile = m == -INFINITY ? 1.f : ex2(m - tmx);
+              l *= a_tile;
+              m = tmx;
+            }
+            const uint64_t nm2 = f2pack(-m, -m);
+            uint64_t acc[2] = {0ull, 0ull};
             if (cnt[h] == 64) {
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
@@ -740,12 +719,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pk[i] = bf16x2(p0, p1);
               }
             }
+            float r0, r1;
+            f2unpack(fadd2(acc[0], acc[1]), r0, r1);
+            l += r0 + r1;
+          }
+          alpha_blk *= a_tile;
+          // tile 1 raised the max after tile 0's P went out: bring tile 0's P to the new max
+          if (h == 1 && __any_sync(0xffffffffu, a_tile != 1.f)) {
+            tmem_wait_st();
+            uint32_t p0r[32];
+            tmem_ld32(tSp, p0r);
+            tmem_wait_ld(p0r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float lo = __uint_as_float(p0r[i] << 16) * a_tile;
+              const float hi = __uint_as_float(p0r[i] & 0xFFFF0000u) * a_tile;
+              p0r[i] = bf16x2(lo, hi);
+            }
+            tmem_st32u(tSp, p0r);
           }
           tmem_st32u(tSp + 64 * h, pk);
         }
-        float r0, r1;
-        f2unpack(fadd2(acc[0], acc[1]), r0, r1);
-        l = l * alpha + (r0 + r1);
+        // O_par holds earlier blocks of this parity at the old max: rescale it
+        // once the PV of the previous block of this parity has finished
+        if (__any_sync(0xffffffffu, j >= 2 && alpha_blk != 1.f)) {
+          ok = wait_bar(bar(B_PEMPTY0 + par), (nb & 1) ^ 1, abort_flag, gerr);   // PV of block nb-1
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(tOp + 32 * c, orr);
+            tmem_wait_ld(orr);
+            float o[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]) * alpha_blk;
+            tmem_st32(tOp + 32 * c, o);
+          }
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_PFULL0 + par));

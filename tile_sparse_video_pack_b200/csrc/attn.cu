@@ -12,22 +12,26 @@
 // is two query tiles of one (batch, head) -- neighbours along h on the video
 // grid, or two prefix tiles -- so the tensor core runs M = 128 MMAs. They
 // share one key list: the union of their kept tiles, each entry tagged with
-// which of the two rows-halves keeps it; a row-half masks the other's tiles to
+// which of the two row-halves keeps it; a row-half masks the other's tiles to
 // -inf. Key tiles go through smem two at a time (128 keys per step).
 //
-// Warp roles (256 threads):
-//   warp 0  TMA producer: Q pair once per item, then K tile pairs (2 stages)
-//   warp 3  TMA producer: V tile pairs (2 stages)
-//   warp 1  MMA issuer: S = Q K^T into TMEM (double buffered), O += P V
+// Warp roles (384 threads):
+//   warp 0  TMA producer: K tile pairs (3 stages)
+//   warp 3  TMA producer: V tile pairs (3 stages)
+//   warp 1  MMA issuer: S = Q K^T with Q in TMEM (two S buffers), O += P V
+//           with P in TMEM
 //   warp 2  scheduler: fetches the next block from a global counter and builds
-//           its merged key list in smem (double buffered)
-//   warps 4-11 softmax, two warpgroups: warpgroup p owns the key blocks of
-//           parity p for all 128 rows (TMEM lane = row), with its own running
-//           max, row sum and O accumulator in TMEM; P goes back to TMEM as
-//           bf16 over the consumed S columns; the epilogue merges the two
+//           its merged key list (double buffered, in a per-CTA global slice)
+//   warps 4-11 softmax, two warpgroups: row r (TMEM lane r) is shared by one
+//           thread of each; warpgroup g handles key tile g of every 128-key
+//           block and half of O's columns. They exchange the block row max and
+//           keep one lazily raised running max; P goes back to TMEM as bf16
+//           over the consumed S columns. At an item's start they put Q in TMEM.
 //
-// Shared-memory operand layouts are the canonical 128-byte-swizzled UMMA
-// layouts that TMA SWIZZLE_128B writes: Q, K and P K-major, V MN-major.
+// Shared memory holds only K and V stages, in the canonical 128-byte-swizzled
+// UMMA layouts that TMA SWIZZLE_128B writes: K K-major, V MN-major. Keeping Q
+// and P in TMEM leaves shared-memory bandwidth to the TMA writes and the two
+// B operands.
 // Every wait is bounded (about two seconds); on expiry the CTA latches a
 // timeout in the plan's error word, drains its copies and MMAs, frees TMEM and
 // returns.
@@ -46,6 +50,14 @@ constexpr float kLazy = 8.0f;  // log2 headroom before the running max is raised
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint32_t kTileBytes = 64 * 64 * 2;  // one 64 x 64 bf16 TMA box
+// K / V tile-pair stages in shared memory: a TMA load takes microseconds from
+// L2, so several must be in flight per CTA.
+#ifndef VSA_K_STAGES
+#define VSA_K_STAGES 3
+#endif
+#ifndef VSA_V_STAGES
+#define VSA_V_STAGES 3
+#endif
 
 // ------------------------------------------------------------------ PTX ----
 
@@ -91,12 +103,6 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a_tmem, uint64_t 
   asm volatile(
       "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
       "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
 #define VSA_R32(X)                                                                                            \
@@ -147,6 +153,14 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) { 
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
       "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
       "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {  // v: 16 raw words
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -234,24 +248,24 @@ struct ItemInfo {
 template <int D>
 struct Smem {
   static constexpr uint32_t kHalfBytes = 128 * 128;               // 128 rows x 128 B
-  static constexpr uint32_t kQBytes = (D / 64) * kHalfBytes;       // Q pair (K-major)
-  static constexpr uint32_t kKBytes = kQBytes;                     // K tile pair
-  static constexpr uint32_t kVBytes = kQBytes;                     // V tile pair (MN-major)
-  static constexpr uint32_t oQ = 0;
-  static constexpr uint32_t oK = oQ + kQBytes;
-  static constexpr uint32_t oV = oK + 2 * kKBytes;
-  static constexpr uint32_t oBar = oV + 2 * kVBytes;
-  static constexpr uint32_t kNumBars = 26;
+  static constexpr uint32_t kKBytes = (D / 64) * kHalfBytes;       // K tile pair (K-major)
+  static constexpr uint32_t kVBytes = kKBytes;                     // V tile pair (MN-major)
+  static constexpr int kKStages = VSA_K_STAGES;
+  static constexpr int kVStages = VSA_V_STAGES;
+  static constexpr uint32_t oK = 0;
+  static constexpr uint32_t oV = oK + kKStages * kKBytes;
+  static constexpr uint32_t oBar = oV + kVStages * kVBytes;
+  static constexpr uint32_t kNumBars = 32;
   static constexpr uint32_t oInfo = oBar + kNumBars * 8;
   static constexpr uint32_t oMisc = oInfo + 2 * sizeof(ItemInfo);  // tmem base, abort flag
   static constexpr uint32_t oXchg = oMisc + 16;                     // row max / row sum exchange
-  static constexpr uint32_t oList = oXchg + (2 * 128 + 2 * 128) * 4;
+  static constexpr uint32_t oEnd = oXchg + (2 * 2 * 128 + 2 * 128) * 4;
 };
 
 // barrier indices
 enum {
-  B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1, B_VFULL0, B_VFULL1, B_VEMPTY0, B_VEMPTY1,
-  B_SFULL0, B_SFULL1, B_PFULL0, B_PFULL1, B_PEMPTY0, B_PEMPTY1, B_LFULL0, B_LFULL1, B_LEMPTY0, B_LEMPTY1,
+  B_QREADY = 0, B_KFULL0, B_KEMPTY0 = B_KFULL0 + 4, B_VFULL0 = B_KEMPTY0 + 4, B_VEMPTY0 = B_VFULL0 + 4,
+  B_SFULL0 = B_VEMPTY0 + 4, B_SFULL1, B_PFULL, B_PDONE, B_MX0, B_MX1, B_LFULL0, B_LFULL1, B_LEMPTY0, B_LEMPTY1,
   B_OFULL, B_OFREE, B_LX, B_DRAIN
 };
 
@@ -260,11 +274,14 @@ struct AttnParams {
   const int32_t* counts;   // [heads, nt_max]
   const WorkItem* items;
   int64_t n_items;
+  const __nv_bfloat16* q;  // packed Q (its rows go to TMEM once per item)
   __nv_bfloat16* out;      // packed O
   float* lse;
   uint32_t* state;         // [0] error word, [1] work counter, [2..3] computed pairs
   int32_t heads, nt_max, ntv_max, k_max, n_pre;
   int32_t list_cap, bitmap_words;
+  uint32_t* lists;         // [CTAs][2][list_cap] merged key lists (one slice per CTA)
+  uint32_t* bitmaps;       // [CTAs][2][bitmap_words] scratch of the list builder
   float scale_log2;
   int32_t ntv[VSA_MAX_HEADS];
   int32_t k[VSA_MAX_HEADS];
@@ -307,8 +324,8 @@ __device__ __forceinline__ int warp_excl_scan(int v, int lane, int* total) {
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                const __grid_constant__ CUtensorMap tv, const __grid_constant__ AttnParams prm) {
+    attn_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                const __grid_constant__ AttnParams prm) {
   using L = Smem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzle atoms
@@ -318,27 +335,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   ItemInfo* info = reinterpret_cast<ItemInfo*>(smem + L::oInfo);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::oMisc);
   volatile uint32_t* abort_flag = misc + 1;
-  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + L::oList);
-  uint32_t* bitmaps = lists + 2 * prm.list_cap;
+  // this CTA's slice of the key-list table (global memory; written and read
+  // inside the CTA, ordered by the list mbarriers)
+  uint32_t* lists = prm.lists + size_t(blockIdx.x) * 2 * prm.list_cap;
+  uint32_t* bitmaps = prm.bitmaps + size_t(blockIdx.x) * 2 * prm.bitmap_words;
   uint32_t* gerr = prm.state;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(B_QFULL), 1);
-    mbar_init(bar(B_QEMPTY), 1);
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(bar(B_QREADY), 256);
+    for (int i = 0; i < 4; ++i) {
       mbar_init(bar(B_KFULL0 + i), 1);
       mbar_init(bar(B_KEMPTY0 + i), 1);
       mbar_init(bar(B_VFULL0 + i), 1);
       mbar_init(bar(B_VEMPTY0 + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_SFULL0 + i), 1);
+      mbar_init(bar(B_MX0 + i), 256);
       mbar_init(bar(B_LFULL0 + i), 32);
       mbar_init(bar(B_LEMPTY0 + i), 256);
-      mbar_init(bar(B_PFULL0 + i), 128);
-      mbar_init(bar(B_PEMPTY0 + i), 1);
     }
+    mbar_init(bar(B_PFULL), 256);
+    mbar_init(bar(B_PDONE), 1);
     mbar_init(bar(B_OFULL), 1);
     mbar_init(bar(B_OFREE), 256);
     mbar_init(bar(B_LX), 256);
@@ -355,15 +376,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
-  // TMEM columns: S_even [0,128), S_odd [128,256), O_even [256,256+D), O_odd [384,384+D).
-  // Even key blocks go through S_even into O_even, odd ones through S_odd into
-  // O_odd; the two partial results are merged once per work item. P (bf16
-  // pairs, two keys per 32-bit column) is written over the S columns it was
-  // computed from: keys 0-63 at columns [0,32), keys 64-127 at [64,96) of the
-  // buffer. The next S MMA into a buffer is issued after the PV MMA that reads
-  // its P, and one thread's tcgen05.mma operations execute in issue order.
+  // TMEM columns: S0 [0,128) and S1 [128,256) for alternate key blocks,
+  // O [256, 256+D), Q [384, 384+D/2) (bf16 pairs: two channels per 32-bit
+  // column; the A operand of S = Q K^T). P (bf16 pairs) is written over the S
+  // columns it was computed from: keys 0-63 at [0,32), keys 64-127 at [64,96)
+  // of the buffer. The next S MMA into a buffer is issued after the PV MMA
+  // that reads its P, and one thread's tcgen05.mma operations execute in issue
+  // order.
   const uint32_t tS = tmem;
   const uint32_t tO = tmem + 256;
+  const uint32_t tQ = tmem + 384;
 
   if (warp == 2) {
     // ------------------------------------------------ scheduler / lists ---
@@ -484,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 0 || warp == 3) {
     // --------------------------------------------------------- producers ---
-    // warp 0: the Q pair of every item and the K tile pairs; warp 3: the V tile
+    // warp 0: the K tile pairs; warp 3: the V tile
     // pairs. Separate threads, so a K load never queues behind a V load that
     // is waiting for its stage to be released by a PV MMA.
     if (lane == 0) {
@@ -492,8 +514,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const CUtensorMap* map = is_k ? &tk : &tv;
       const int full0 = is_k ? B_KFULL0 : B_VFULL0;
       const int empty0 = is_k ? B_KEMPTY0 : B_VEMPTY0;
+      const int nst = is_k ? L::kKStages : L::kVStages;
       uint32_t g = 0;          // key blocks issued
-      uint32_t issuedQ = 0;    // Q loads issued
+      int st = 0;              // stage of block g (g mod nst)
+      uint32_t ph = 0;         // phase of that stage ((g / nst) & 1)
       for (uint32_t it = 0;; ++it) {
         const int slot = it & 1;
         if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr)) break;
@@ -501,23 +525,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (inf.end) break;
         const uint32_t* list = lists + slot * prm.list_cap;
         const int row_base = inf.bh * prm.nt_max;
-        if (is_k) {
-          if (!wait_bar(bar(B_QEMPTY), (it & 1) ^ 1, abort_flag, gerr)) break;
-          mbar_expect_tx(bar(B_QFULL), 2 * (D / 64) * kTileBytes);
-          const int qb = inf.qb >= 0 ? inf.qb : inf.qa;
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(sbase + L::oQ + c * L::kHalfBytes, &tq, 64 * c, (row_base + inf.qa) * 64, bar(B_QFULL));
-            tma_load_2d(sbase + L::oQ + c * L::kHalfBytes + 8192, &tq, 64 * c, (row_base + qb) * 64, bar(B_QFULL));
-          }
-          ++issuedQ;
-        }
         const int nblk = (inf.n_entries + 1) >> 1;
         bool ok = true;
         for (int j = 0; j < nblk; ++j) {
-          const int st = g & 1;
           const int ta = int(list[2 * j] & 0xFFFFu);
           const int tb = 2 * j + 1 < inf.n_entries ? int(list[2 * j + 1] & 0xFFFFu) : ta;
-          if (!(ok = wait_bar(bar(empty0 + st), ((g >> 1) & 1) ^ 1, abort_flag, gerr))) break;
+          if (!(ok = wait_bar(bar(empty0 + st), ph ^ 1, abort_flag, gerr))) break;
           mbar_expect_tx(bar(full0 + st), 2 * (D / 64) * kTileBytes);
           if (is_k) {   // K-major: tile a rows 0-63, tile b rows 64-127 of each 64-column half
             const uint32_t sk = sbase + L::oK + st * L::kKBytes;
@@ -533,13 +546,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           ++g;
+          if (++st == nst) {
+            st = 0;
+            ph ^= 1;
+          }
         }
         if (!ok) break;
       }
       if (*abort_flag) {
         // let every copy this thread issued land before shared memory is released
-        if (is_k && issuedQ) drain_wait(bar(B_QFULL), (issuedQ - 1) & 1);
-        for (uint32_t gg = (g >= 2 ? g - 2 : 0); gg < g; ++gg) drain_wait(bar(full0 + (gg & 1)), (gg >> 1) & 1);
+        for (uint32_t gg = (g >= uint32_t(nst) ? g - nst : 0); gg < g; ++gg)
+          drain_wait(bar(full0 + int(gg % nst)), (gg / nst) & 1);
       }
     }
     __syncwarp();
@@ -548,32 +565,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idPV = idesc_bf16(128, D, 0, 1);
-      // descriptors of the stage bases; a k-step adds (byte offset >> 4) to the start address
-      const uint64_t dq = sw128_desc(sbase + L::oQ, 16, 1024);
-      const uint64_t dk[2] = {sw128_desc(sbase + L::oK, 16, 1024), sw128_desc(sbase + L::oK + L::kKBytes, 16, 1024)};
-      const uint64_t dv[2] = {sw128_desc(sbase + L::oV, 8192, 1024),
-                              sw128_desc(sbase + L::oV + L::kVBytes, 8192, 1024)};
-      uint32_t g = 0;            // key blocks so far (K / V stage ring)
-      uint32_t npv[2] = {0, 0};  // PV MMAs issued per parity (phases of P_FULL)
+      // descriptors of the first stage; a stage or k-step adds (byte offset >> 4)
+      const uint64_t dk0 = sw128_desc(sbase + L::oK, 16, 1024);
+      const uint64_t dv0 = sw128_desc(sbase + L::oV, 8192, 1024);
+      int kst = 0, vst = 0;      // K / V stage of the next S / PV MMA
+      uint32_t kph = 0, vph = 0; // their phases
+      uint32_t g = 0;            // key blocks so far
       bool ok = true;
-      // O_p += P V for block gg (global) = block jj of the item, parity p = jj & 1
+      // O += P V for block gg (global) = block jj of the item
       auto issue_pv = [&](uint32_t gg, int jj, uint32_t it) -> bool {
-        const int st = gg & 1;
-        const int p = jj & 1;
         if (jj == 0 && !wait_bar(bar(B_OFREE), (it & 1) ^ 1, abort_flag, gerr)) return false;
-        if (!wait_bar(bar(B_PFULL0 + p), npv[p] & 1, abort_flag, gerr)) return false;
-        if (!wait_bar(bar(B_VFULL0 + st), (gg >> 1) & 1, abort_flag, gerr)) return false;
-        ++npv[p];
+        if (!wait_bar(bar(B_PFULL), gg & 1, abort_flag, gerr)) return false;
+        if (!wait_bar(bar(B_VFULL0 + vst), vph, abort_flag, gerr)) return false;
         tc_fence_after();
-        const uint32_t o = tO + p * 128;
-        const uint32_t pcol = tS + p * 128;
+        const uint32_t pcol = tS + (gg & 1) * 128;
+        const uint64_t dv = dv0 + ((vst * L::kVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {   // 16 keys per step: 8 TMEM columns of P
           const uint32_t boff = ((kk >> 2) * (D / 64) * 8192 + (kk & 3) * 2048) >> 4;
-          tc_mma_ts(o, pcol + (kk >> 2) * 64 + (kk & 3) * 8, dv[st] + boff, idPV, (jj < 2 && kk == 0) ? 0u : 1u);
+          tc_mma_ts(tO, pcol + (kk >> 2) * 64 + (kk & 3) * 8, dv + boff, idPV, (jj == 0 && kk == 0) ? 0u : 1u);
         }
-        tc_commit(bar(B_VEMPTY0 + st));
-        tc_commit(bar(B_PEMPTY0 + p));
+        tc_commit(bar(B_VEMPTY0 + vst));
+        tc_commit(bar(B_PDONE));
+        if (++vst == L::kVStages) {
+          vst = 0;
+          vph ^= 1;
+        }
         return true;
       };
       for (uint32_t it = 0; ok; ++it) {
@@ -581,21 +598,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr)) break;
         const ItemInfo inf = info[slot];
         if (inf.end) break;
-        if (!wait_bar(bar(B_QFULL), it & 1, abort_flag, gerr)) break;
+        if (!wait_bar(bar(B_QREADY), it & 1, abort_flag, gerr)) break;   // Q rows in TMEM
         const int nblk = (inf.n_entries + 1) >> 1;
         for (int j = 0; j < nblk; ++j, ++g) {
-          const int st = g & 1;
-          if (!(ok = wait_bar(bar(B_KFULL0 + st), (g >> 1) & 1, abort_flag, gerr))) break;
+          if (!(ok = wait_bar(bar(B_KFULL0 + kst), kph, abort_flag, gerr))) break;
           tc_fence_after();
-          const int p = j & 1;     // S buffer of this block's parity within the item
+          const uint64_t dk = dk0 + ((kst * L::kKBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
+          for (int kk = 0; kk < D / 16; ++kk) {   // S = Q K^T, 16 channels per step
             const uint32_t off = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
-            tc_mma(tS + p * 128, dq + off, dk[st] + off, idS, kk > 0 ? 1u : 0u);
+            tc_mma_ts(tS + (g & 1) * 128, tQ + kk * 8, dk + off, idS, kk > 0 ? 1u : 0u);
           }
-          tc_commit(bar(B_SFULL0 + p));
-          tc_commit(bar(B_KEMPTY0 + st));
-          if (j == nblk - 1) tc_commit(bar(B_QEMPTY));
+          tc_commit(bar(B_SFULL0 + (g & 1)));
+          tc_commit(bar(B_KEMPTY0 + kst));
+          if (++kst == L::kKStages) {
+            kst = 0;
+            kph ^= 1;
+          }
           if (j > 0 && !(ok = issue_pv(g - 1, j - 1, it))) break;
         }
         if (!ok) break;
@@ -609,21 +628,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ----------------------------------------------------------- softmax ---
-    // Warpgroup par (0 or 1) handles the even or odd key blocks of every item
-    // for all 128 rows (row = TMEM lane), with its own running max m, row sum
-    // l and accumulator O_par. The running max is raised only when a block
-    // exceeds it by more than kLazy (log2 units), so P < 2^kLazy and O_par is
-    // rarely rescaled. The epilogue merges (m, l, O) of both warpgroups.
-    const int par = (warp - 4) >> 2;
+    // Two warpgroups share every row (row = TMEM lane): warpgroup sg handles
+    // key tile sg of each 128-key block (S columns [64 sg, 64 sg + 64)) and O
+    // columns [sg D/2, (sg+1) D/2). They exchange each block's row max through
+    // shared memory and keep the same running max m; it is raised only when a
+    // block exceeds it by more than kLazy (log2 units), so P < 2^kLazy and O
+    // is rarely rescaled. At the start of an item each thread puts its half of
+    // its Q row into TMEM.
+    const int sg = (warp - 4) >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     const uint32_t my_bit = r < 64 ? 1u : 2u;
-    const uint32_t tSp = tS + par * 128 + lane_off;
-    const uint32_t tOp = tO + par * 128 + lane_off;
-    float* xm = reinterpret_cast<float*>(smem + L::oXchg);   // [2][128] row max (log2 units)
-    float* xl = xm + 2 * 128;                               // [2][128] row sum
+    float* xm = reinterpret_cast<float*>(smem + L::oXchg);   // [2 buffers][2 groups][128] block row max
+    float* xl = xm + 2 * 2 * 128;                           // [2 groups][128] row sums
     const uint64_t c2 = f2pack(prm.scale_log2, prm.scale_log2);
-    uint32_t nb = 0;           // blocks of this parity so far (phases of S_FULL / P_FULL / P_EMPTY)
+    uint32_t g = 0;
     bool ok = true;
     for (uint32_t it = 0; ok; ++it) {
       const int slot = it & 1;
@@ -633,186 +652,178 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (inf.end) break;
       const uint32_t* list = lists + slot * prm.list_cap;
       const int nblk = (inf.n_entries + 1) >> 1;
+      {  // Q: this thread's row, channels [sg D/2, (sg+1) D/2), as bf16 pairs
+        const int tile = r < 64 ? inf.qa : inf.qb;
+        uint32_t qw[D / 4];
+        if (tile >= 0) {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              prm.q + ((size_t(inf.bh) * prm.nt_max + tile) * 64 + (r & 63)) * D + sg * (D / 2));
+#pragma unroll
+          for (int i = 0; i < D / 16; ++i) {
+            const uint4 u = src[i];
+            qw[4 * i] = u.x;
+            qw[4 * i + 1] = u.y;
+            qw[4 * i + 2] = u.z;
+            qw[4 * i + 3] = u.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < D / 4; ++i) qw[i] = 0u;
+        }
+        if constexpr (D == 128) {
+          tmem_st32u(tQ + lane_off + sg * 32, qw);
+        } else {
+          tmem_st16u(tQ + lane_off + sg * 16, qw);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_QREADY));
+      }
       float m = -INFINITY, l = 0.f;
-      for (int j = par; j < nblk; j += 2, ++nb) {
-        ok = wait_bar(bar(B_SFULL0 + par), nb & 1, abort_flag, gerr);
+      for (int j = 0; j < nblk; ++j, ++g) {
+        const int b = g & 1;
+        const uint32_t tSb = tS + b * 128 + lane_off;
+        ok = wait_bar(bar(B_SFULL0 + b), (g >> 1) & 1, abort_flag, gerr);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-        int cnt[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int ei = 2 * j + h;
-          const uint32_t e = ei < inf.n_entries ? list[ei] : 0u;
-          cnt[h] = ((e >> 16) & my_bit) ? int(e >> 24) : 0;   // valid keys of tile h for my row
-        }
-        // 64 scores of tile h (columns [64h, 64h+64)); missing keys of a partial tile -> -inf
-        auto load_tile = [&](int h, float (&sv)[64]) {
+        const int ei = 2 * j + sg;
+        const uint32_t e = ei < inf.n_entries ? list[ei] : 0u;
+        const int cnt = ((e >> 16) & my_bit) ? int(e >> 24) : 0;   // valid keys of my tile for my row
+        float sv[64];
+        float tmx = -INFINITY;
+        if (cnt > 0) {
           uint32_t sr[2][32];
-          tmem_ld32(tSp + 64 * h, sr[0]);
-          tmem_ld32(tSp + 64 * h + 32, sr[1]);
+          tmem_ld32(tSb + 64 * sg, sr[0]);
+          tmem_ld32(tSb + 64 * sg + 32, sr[1]);
           tmem_wait_ld(sr[0]);
           reg_fence(sr[1]);
 #pragma unroll
           for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
-          if (cnt[h] < 64) {
+          if (cnt < 64) {                          // partial tile: missing keys -> -inf
 #pragma unroll
-            for (int c = 0; c < 64; ++c) sv[c] = c < cnt[h] ? sv[c] : -INFINITY;
+            for (int c = 0; c < 64; ++c) sv[c] = c < cnt ? sv[c] : -INFINITY;
           }
-        };
-        // One pass per tile: P = 2^(s * scale * log2(e) - m) with the running max m
-        // (log2 units), written as bf16 pairs over consumed S columns (tile 0 ->
-        // [0,32), tile 1 -> [64,96)). Each tile's max is checked first: if it
-        // exceeds m by more than kLazy, m is raised before the tile's
-        // exponentials, and whatever was already accumulated at the old m -- the
-        // row sum, tile 0's stored P, and O_par -- is scaled by 2^(m_old - m_new).
-        float alpha_blk = 1.f;
+          float mq[4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-          float a_tile = 1.f;
-          if (cnt[h] == 0) {
+          for (int q = 0; q < 4; ++q) {
+            float t = fmax3(sv[16 * q], sv[16 * q + 1], sv[16 * q + 2]);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) pk[i] = 0u;
-          } else {
-            float sv[64];
-            load_tile(h, sv);
-            float mq[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float t = fmax3(sv[16 * q], sv[16 * q + 1], sv[16 * q + 2]);
-#pragma unroll
-              for (int c = 3; c < 15; c += 2) t = fmax3(t, sv[16 * q + c], sv[16 * q + c + 1]);
-              mq[q] = fmaxf(t, sv[16 * q + 15]);
-            }
-            const float tmx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * prm.scale_log2;
-            if (tmx > m + kLazy) {                  // also taken when m is still -inf
-              a_tile = m == -INFINITY ? 1.f : ex2(m - tmx);
-              l *= a_tile;
-              m = tmx;
-            }
-            const uint64_t nm2 = f2pack(-m, -m);
-            uint64_t acc[2] = {0ull, 0ull};
-            if (cnt[h] == 64) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                float x0, x1, p0, p1;
-                f2unpack(ffma2(f2pack(sv[2 * i], sv[2 * i + 1]), c2, nm2), x0, x1);
-                constexpr int kPoly = VSA_EXP_POLY_EVERY;
-                bool on_fma = false;
-                if constexpr (kPoly > 0) on_fma = i % kPoly == kPoly - 1;
-                if (on_fma) {
-                  ex2_fma_pipe(x0, x1, p0, p1);
-                } else {
-                  p0 = ex2(x0);
-                  p1 = ex2(x1);
-                }
-                acc[i & 1] = fadd2(acc[i & 1], f2pack(p0, p1));
-                pk[i] = bf16x2(p0, p1);
-              }
-            } else {                                   // partial tile: masked keys give exactly 0
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                float x0, x1;
-                f2unpack(ffma2(f2pack(sv[2 * i], sv[2 * i + 1]), c2, nm2), x0, x1);
-                const float p0 = ex2(x0), p1 = ex2(x1);   // ex2(-inf) = 0
-                acc[i & 1] = fadd2(acc[i & 1], f2pack(p0, p1));
-                pk[i] = bf16x2(p0, p1);
-              }
-            }
-            float r0, r1;
-            f2unpack(fadd2(acc[0], acc[1]), r0, r1);
-            l += r0 + r1;
+            for (int c = 3; c < 15; c += 2) t = fmax3(t, sv[16 * q + c], sv[16 * q + c + 1]);
+            mq[q] = fmaxf(t, sv[16 * q + 15]);
           }
-          alpha_blk *= a_tile;
-          // tile 1 raised the max after tile 0's P went out: bring tile 0's P to the new max
-          if (h == 1 && __any_sync(0xffffffffu, a_tile != 1.f)) {
-            tmem_wait_st();
-            uint32_t p0r[32];
-            tmem_ld32(tSp, p0r);
-            tmem_wait_ld(p0r);
+          tmx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+        }
+        // the block's row max from both warpgroups (raw scores; the scale is positive)
+        xm[(b * 2 + sg) * 128 + r] = tmx;
+        mbar_arrive(bar(B_MX0 + b));
+        ok = wait_bar(bar(B_MX0 + b), (g >> 1) & 1, abort_flag, gerr);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        const float bmx = fmaxf(xm[(b * 2) * 128 + r], xm[(b * 2 + 1) * 128 + r]) * prm.scale_log2;
+        float alpha = 1.f;
+        if (bmx > m + kLazy) {                     // also taken when m is still -inf
+          alpha = m == -INFINITY ? 1.f : ex2(m - bmx);
+          m = bmx;
+        }
+        l *= alpha;
+        uint32_t pk[32];
+        if (cnt > 0) {
+          const uint64_t nm2 = f2pack(-m, -m);
+          uint64_t acc[2] = {0ull, 0ull};
+          if (cnt == 64) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float lo = __uint_as_float(p0r[i] << 16) * a_tile;
-              const float hi = __uint_as_float(p0r[i] & 0xFFFF0000u) * a_tile;
-              p0r[i] = bf16x2(lo, hi);
+              float x0, x1, p0, p1;
+              f2unpack(ffma2(f2pack(sv[2 * i], sv[2 * i + 1]), c2, nm2), x0, x1);
+              constexpr int kPoly = VSA_EXP_POLY_EVERY;
+              bool on_fma = false;
+              if constexpr (kPoly > 0) on_fma = i % kPoly == kPoly - 1;
+              if (on_fma) {
+                ex2_fma_pipe(x0, x1, p0, p1);
+              } else {
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+              }
+              acc[i & 1] = fadd2(acc[i & 1], f2pack(p0, p1));
+              pk[i] = bf16x2(p0, p1);
             }
-            tmem_st32u(tSp, p0r);
+          } else {                                 // partial tile: masked keys give exactly 0
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              float x0, x1;
+              f2unpack(ffma2(f2pack(sv[2 * i], sv[2 * i + 1]), c2, nm2), x0, x1);
+              const float p0 = ex2(x0), p1 = ex2(x1);   // ex2(-inf) = 0
+              acc[i & 1] = fadd2(acc[i & 1], f2pack(p0, p1));
+              pk[i] = bf16x2(p0, p1);
+            }
           }
-          tmem_st32u(tSp + 64 * h, pk);
+          float r0, r1;
+          f2unpack(fadd2(acc[0], acc[1]), r0, r1);
+          l += r0 + r1;
+        } else {                                   // my row-half does not keep this tile
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pk[i] = 0u;
         }
-        // O_par holds earlier blocks of this parity at the old max: rescale it
-        // once the PV of the previous block of this parity has finished
-        if (__any_sync(0xffffffffu, j >= 2 && alpha_blk != 1.f)) {
-          ok = wait_bar(bar(B_PEMPTY0 + par), (nb & 1) ^ 1, abort_flag, gerr);   // PV of block nb-1
+        // P over my tile's consumed S columns: [64 sg, 64 sg + 32)
+        tmem_st32u(tSb + 64 * sg, pk);
+        // earlier blocks of this item sit in O at the old max: rescale my half of
+        // O once the previous PV has finished accumulating into it
+        if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
+          ok = wait_bar(bar(B_PDONE), (g - 1) & 1, abort_flag, gerr);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < D / 64; ++c) {
             uint32_t orr[32];
-            tmem_ld32(tOp + 32 * c, orr);
+            const uint32_t col = tO + lane_off + sg * (D / 2) + 32 * c;
+            tmem_ld32(col, orr);
             tmem_wait_ld(orr);
             float o[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]) * alpha_blk;
-            tmem_st32(tOp + 32 * c, o);
+            for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]) * alpha;
+            tmem_st32(col, o);
           }
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_PFULL0 + par));
+        mbar_arrive(bar(B_PFULL));
       }
       if (!ok) break;
-      // epilogue: both partial results are final once the item's last PV is done
+      // epilogue: O is final once the item's last PV is done; the row sum is the two groups' sum
       ok = wait_bar(bar(B_OFULL), it & 1, abort_flag, gerr);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      xm[par * 128 + r] = m;
-      xl[par * 128 + r] = l;
+      xl[sg * 128 + r] = l;
       mbar_arrive(bar(B_LX));
       ok = wait_bar(bar(B_LX), it & 1, abort_flag, gerr);
       if (!__all_sync(0xffffffffu, ok)) break;
-      const float m0 = xm[r], m1 = xm[128 + r], l0 = xl[r], l1 = xl[128 + r];
-      const float mt = fmaxf(m0, m1);
-      const bool has_odd = nblk >= 2;
-      const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - mt);
-      const float f1 = (!has_odd || m1 == -INFINITY) ? 0.f : ex2(m1 - mt);
-      const float lrow = l0 * f0 + l1 * f1;
+      const float lrow = xl[r] + xl[128 + r];
       const int tile = r < 64 ? inf.qa : inf.qb;
       const int slot_r = r & 63;
       const int rows = r < 64 ? inf.rows_a : inf.rows_b;
       const bool write = tile >= 0 && !inf.bad;
       const bool valid = write && slot_r < rows;
       const float inv = (valid && lrow > 0.f) ? 1.f / lrow : 0.f;
-      const float w0 = f0 * inv, w1 = f1 * inv;
       const size_t orow = (size_t(inf.bh) * prm.nt_max + (tile >= 0 ? tile : 0)) * 64 + slot_r;
-      // this warpgroup writes O columns [par D/2, (par+1) D/2) of its rows
-      uint4* dst = reinterpret_cast<uint4*>(prm.out + orow * D + par * (D / 2));
+      uint4* dst = reinterpret_cast<uint4*>(prm.out + orow * D + sg * (D / 2));
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
-        const uint32_t col = lane_off + par * (D / 2) + 32 * c;
-        uint32_t a0[32], a1[32];
-        tmem_ld32(tO + col, a0);
-        if (has_odd) tmem_ld32(tO + 128 + col, a1);
-        tmem_wait_ld(a0);
-        if (has_odd) reg_fence(a1);
-        float o[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          o[i] = __uint_as_float(a0[i]) * w0 + (has_odd ? __uint_as_float(a1[i]) * w1 : 0.f);
+        uint32_t orr[32];
+        tmem_ld32(tO + lane_off + sg * (D / 2) + 32 * c, orr);
+        tmem_wait_ld(orr);
         if (write) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint4 pkq;
-            pkq.x = bf16x2(o[8 * q + 0], o[8 * q + 1]);
-            pkq.y = bf16x2(o[8 * q + 2], o[8 * q + 3]);
-            pkq.z = bf16x2(o[8 * q + 4], o[8 * q + 5]);
-            pkq.w = bf16x2(o[8 * q + 6], o[8 * q + 7]);
+            pkq.x = bf16x2(__uint_as_float(orr[8 * q + 0]) * inv, __uint_as_float(orr[8 * q + 1]) * inv);
+            pkq.y = bf16x2(__uint_as_float(orr[8 * q + 2]) * inv, __uint_as_float(orr[8 * q + 3]) * inv);
+            pkq.z = bf16x2(__uint_as_float(orr[8 * q + 4]) * inv, __uint_as_float(orr[8 * q + 5]) * inv);
+            pkq.w = bf16x2(__uint_as_float(orr[8 * q + 6]) * inv, __uint_as_float(orr[8 * q + 7]) * inv);
             dst[c * 4 + q] = pkq;
           }
         }
       }
-      if (write && par == 0 && prm.lse)
-        prm.lse[orow] = valid && lrow > 0.f ? (mt + __log2f(lrow)) * 0.69314718055994531f : 0.f;
+      if (write && sg == 0 && prm.lse)
+        prm.lse[orow] = valid && lrow > 0.f ? (m + __log2f(lrow)) * 0.69314718055994531f : 0.f;
       tc_fence_before();
       mbar_arrive(bar(B_OFREE));
       mbar_arrive(bar(B_LEMPTY0 + slot));
@@ -859,23 +870,23 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int d) {
 }  // namespace
 
 int attn_smem_bytes(int list_cap) {
-  using L = Smem<128>;
-  const int bitmap_words = (list_cap / 32) + 2;
-  return 1024 + int(L::oList) + 2 * list_cap * 4 + 2 * bitmap_words * 4;
+  (void)list_cap;   // key lists live in global memory
+  static_assert(Smem<64>::oEnd <= Smem<128>::oEnd, "the d=64 layout fits the d=128 allocation");
+  return 1024 + int(Smem<128>::oEnd);
 }
 
 cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp, const int32_t* idx, void* op,
                         float* lse, cudaStream_t s) {
   const Geometry& g = p->geo;
   const int64_t rows = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE;
-  CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, qp, rows, g.d) || !make_map(&tk, kp, rows, g.d) || !make_map(&tv, vp, rows, g.d))
-    return cudaErrorInvalidValue;
+  CUtensorMap tk, tv;
+  if (!make_map(&tk, kp, rows, g.d) || !make_map(&tv, vp, rows, g.d)) return cudaErrorInvalidValue;
   AttnParams prm;
   prm.idx = idx;
   prm.counts = p->d_tile_count;
   prm.items = p->d_items;
   prm.n_items = p->n_items;
+  prm.q = static_cast<const __nv_bfloat16*>(qp);
   prm.out = static_cast<__nv_bfloat16*>(op);
   prm.lse = lse;
   prm.state = p->d_state;
@@ -886,6 +897,8 @@ cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void*
   prm.n_pre = g.n_pre_tiles;
   prm.list_cap = p->list_cap;
   prm.bitmap_words = (p->list_cap / 32) + 2;
+  prm.lists = p->d_lists;
+  prm.bitmaps = p->d_lists + size_t(p->num_sms) * 2 * p->list_cap;
   prm.scale_log2 = p->desc.softmax_scale * 1.4426950408889634f;
   for (int h = 0; h < VSA_MAX_HEADS; ++h) {
     prm.ntv[h] = h < g.Hh ? g.ntv[h] : 0;
@@ -899,11 +912,11 @@ cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void*
   if (g.d == 128) {
     e = cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel<128><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm);
+    attn_kernel<128><<<grid, kThreads, smem, s>>>(tk, tv, prm);
   } else {
     e = cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel<64><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm);
+    attn_kernel<64><<<grid, kThreads, smem, s>>>(tk, tv, prm);
   }
   return cudaGetLastError();
 }

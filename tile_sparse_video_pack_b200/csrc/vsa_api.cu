@@ -153,7 +153,8 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
   }
   g.nt_max = g.n_pre_tiles + g.ntv_max;
 
-  // the attention kernel keeps one item's key list in shared memory
+  // the attention kernel builds each item's merged key list (at most every
+  // tile of a head, 16-bit tile ids) in a per-CTA slice of global memory
   p->list_cap = g.nt_max;
   p->attn_smem_bytes = vsa::attn_smem_bytes(p->list_cap);
   if (p->attn_smem_bytes > 227 * 1024 || g.nt_max >= 65536) {
@@ -219,6 +220,10 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
   if (e == cudaSuccess) e = cudaMalloc(&p->d_tile_count, counts.size() * sizeof(int32_t));
   if (e == cudaSuccess) e = cudaMalloc(&p->d_items, items.size() * sizeof(WorkItem));
   if (e == cudaSuccess) e = cudaMalloc(&p->d_state, 64);
+  if (e == cudaSuccess) {
+    const size_t words = size_t(p->num_sms) * 2 * (size_t(p->list_cap) + size_t(p->list_cap / 32 + 2));
+    e = cudaMalloc(&p->d_lists, words * sizeof(uint32_t));
+  }
   if (e == cudaSuccess)
     e = cudaMemcpy(p->d_tile_count, counts.data(), counts.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess)
@@ -236,10 +241,11 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
 
 vsa_status vsa_plan_destroy(vsa_plan* p) {
   if (!p) return VSA_OK;
-  if (p->d_tile_count || p->d_items || p->d_state) cudaDeviceSynchronize();
+  if (p->d_tile_count || p->d_items || p->d_state || p->d_lists) cudaDeviceSynchronize();
   if (p->d_tile_count) cudaFree(p->d_tile_count);
   if (p->d_items) cudaFree(p->d_items);
   if (p->d_state) cudaFree(p->d_state);
+  if (p->d_lists) cudaFree(p->d_lists);
   delete p;
   return VSA_OK;
 }

@@ -52,6 +52,7 @@ struct vsa_plan {
   vsa::WorkItem* d_items;  // attention work list, heaviest first
   int64_t n_items;
   uint32_t* d_state;       // [0] error word, [1] work counter
+  uint32_t* d_lists;       // attention key lists and bitmaps, one slice per CTA
   int attn_smem_bytes;
   int list_cap;            // entries of one key-list buffer in the attention kernel
 };

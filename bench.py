@@ -75,7 +75,7 @@ def attn_source_sha1() -> str:
         return hashlib.sha1(f.read()).hexdigest()
 
 
-def measured_traffic(config: str, heads: int):
+def measured_traffic(config: str, sparsity: float, heads: int):
     """DRAM bytes per attention launch from the committed ncu capture, if it is of this kernel source.
 
     The capture runs a smaller case (fewer heads) of the same workload; bytes grow
@@ -90,7 +90,8 @@ def measured_traffic(config: str, heads: int):
             if "=" in ln and not ln.startswith("#"):
                 a, b = ln.split("=", 1)
                 kv[a.strip()] = b.strip()
-    if kv.get("attn_source_sha1") != attn_source_sha1() or kv.get("config") != config:
+    if (kv.get("attn_source_sha1") != attn_source_sha1() or kv.get("config") != config
+            or float(kv.get("sparsity", "nan")) != sparsity):
         return None
     per_head = (float(kv["dram_bytes_read"]) + float(kv["dram_bytes_write"])) / float(kv["heads"])
     return int(per_head * heads)
@@ -99,8 +100,8 @@ def measured_traffic(config: str, heads: int):
 # --------------------------------------------------------------- work counts --
 
 def k_list(cfg, s):
-    import oracle.vsa_oracle as O  # the k rule only; no attention work
-    return [O.k_from_sparsity(s, -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw))
+    from tile_sparse_video_pack_b200 import vsa
+    return [vsa.k_from_sparsity(s, -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw))
             for (pt, ph, pw) in cfg.tile_shapes]
 
 
@@ -193,7 +194,8 @@ class OracleSample:
         self.inp = make_layer_inputs(self.sub)
         f = lambda b: bf16_bits_to_f32(b).astype(np.float64)
         self.q, self.k, self.v = f(self.inp.q), f(self.inp.k), f(self.inp.v)
-        self.ks = k_list(self.sub, sparsity)
+        self.ks = [O.k_from_sparsity(sparsity, -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw))
+                   for (pt, ph, pw) in self.sub.tile_shapes]
         self.til = O.head_tiling(self.sub, 0)
         self.rng = np.random.default_rng(0)
 
@@ -373,7 +375,7 @@ def run_ours(args, rank, world, local_rank):
     achieved = flops / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": measured_traffic(args.config, cfg.heads),
+                "frac": round(achieved / peak, 4), "traffic": measured_traffic(args.config, args.sparsity, cfg.heads),
                 "kernel": "attn_kernel (vsa_sparse_attn)",
                 "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
                 "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),

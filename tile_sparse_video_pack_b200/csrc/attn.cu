@@ -16,22 +16,25 @@
 // -inf. Key tiles go through smem two at a time (128 keys per step).
 //
 // Warp roles (384 threads):
-//   warp 0  TMA producer: K tile pairs (3 stages)
-//   warp 3  TMA producer: V tile pairs (3 stages)
-//   warp 1  MMA issuer: S = Q K^T with Q in TMEM (two S buffers), O += P V
-//           with P in TMEM
+//   warp 0  TMA producers: lane 0 the Q pair of every block of rows and the K
+//           tile pairs (2 stages), lane 1 the V tile pairs (3 stages)
+//   warp 1  MMA issuer for S = Q K^T (Q and K in smem) into one of three TMEM
+//           S buffers
+//   warp 3  MMA issuer for O += P V (P in TMEM over the S columns it came
+//           from, V in smem)
 //   warp 2  scheduler: fetches the next block from a global counter and builds
 //           its merged key list (double buffered, in a per-CTA global slice)
 //   warps 4-11 softmax, two warpgroups: row r (TMEM lane r) is shared by one
 //           thread of each; warpgroup g handles key tile g of every 128-key
 //           block and half of O's columns. They exchange the block row max and
 //           keep one lazily raised running max; P goes back to TMEM as bf16
-//           over the consumed S columns. At an item's start they put Q in TMEM.
+//           over the consumed S columns.
 //
-// Shared memory holds only K and V stages, in the canonical 128-byte-swizzled
-// UMMA layouts that TMA SWIZZLE_128B writes: K K-major, V MN-major. Keeping Q
-// and P in TMEM leaves shared-memory bandwidth to the TMA writes and the two
-// B operands.
+// One thread can have only one tcgen05.mma in execution at a time, and an
+// M = 128, K = 16 MMA takes about as long for N = 128 as for N = 256; S and PV
+// therefore come from two issuing threads, and three S buffers let S for the
+// next blocks run while PV drains the previous one.
+//
 // Every wait is bounded (about two seconds); on expiry the CTA latches a
 // timeout in the plan's error word, drains its copies and MMAs, frees TMEM and
 // returns.
@@ -46,6 +49,9 @@ namespace vsa {
 namespace {
 
 constexpr int kThreads = 384;
+constexpr int kSBuf = 2;        // TMEM S buffers
+constexpr int kPvWarp = 3;      // the PV MMA issuer
+constexpr int kSmWarps = 8;     // softmax warps (4-11); each arrives once on their barriers
 constexpr float kLazy = 8.0f;  // log2 headroom before the running max is raised
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
@@ -53,7 +59,7 @@ constexpr uint32_t kTileBytes = 64 * 64 * 2;  // one 64 x 64 bf16 TMA box
 // K / V tile-pair stages in shared memory: a TMA load takes microseconds from
 // L2, so several must be in flight per CTA.
 #ifndef VSA_K_STAGES
-#define VSA_K_STAGES 3
+#define VSA_K_STAGES 2
 #endif
 #ifndef VSA_V_STAGES
 #define VSA_V_STAGES 3
@@ -74,6 +80,13 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// One arrival for the whole warp: every lane's earlier shared-memory writes and
+// completed TMEM stores are ordered before it by the warp barrier, and the
+// arrival (a release) publishes them to the thread that waits on the mbarrier.
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
@@ -97,6 +110,13 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+// A and B from shared memory (descriptors).
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
 }
 // A from TMEM (K-major, 16-bit elements packed two per 32-bit column), B from smem.
 __device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -153,14 +173,6 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) { 
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
       "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
       "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {  // v: 16 raw words
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
-      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -252,29 +264,32 @@ struct Smem {
   static constexpr uint32_t kVBytes = kKBytes;                     // V tile pair (MN-major)
   static constexpr int kKStages = VSA_K_STAGES;
   static constexpr int kVStages = VSA_V_STAGES;
-  static constexpr uint32_t oK = 0;
+  static constexpr uint32_t kQBytes = kKBytes;                     // the Q pair (K-major)
+  static constexpr uint32_t oQ = 0;
+  static constexpr uint32_t oK = oQ + kQBytes;
   static constexpr uint32_t oV = oK + kKStages * kKBytes;
   static constexpr uint32_t oBar = oV + kVStages * kVBytes;
-  static constexpr uint32_t kNumBars = 32;
+  static constexpr uint32_t kNumBars = 40;
   static constexpr uint32_t oInfo = oBar + kNumBars * 8;
   static constexpr uint32_t oMisc = oInfo + 2 * sizeof(ItemInfo);  // tmem base, abort flag
   static constexpr uint32_t oXchg = oMisc + 16;                     // row max / row sum exchange
-  static constexpr uint32_t oEnd = oXchg + (2 * 2 * 128 + 2 * 128) * 4;
+  static constexpr uint32_t oEnd = oXchg + (2 * 128 + 2 * 128) * 4;
 };
 
 // barrier indices
 enum {
-  B_QREADY = 0, B_KFULL0, B_KEMPTY0 = B_KFULL0 + 4, B_VFULL0 = B_KEMPTY0 + 4, B_VEMPTY0 = B_VFULL0 + 4,
-  B_SFULL0 = B_VEMPTY0 + 4, B_SFULL1, B_PFULL, B_PDONE, B_MX0, B_MX1, B_LFULL0, B_LFULL1, B_LEMPTY0, B_LEMPTY1,
-  B_OFULL, B_OFREE, B_LX, B_DRAIN
+  B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KEMPTY0 = B_KFULL0 + 4, B_VFULL0 = B_KEMPTY0 + 4, B_VEMPTY0 = B_VFULL0 + 4,
+  // P_FULL / P_DONE: [softmax warpgroup][S buffer]
+  B_SFULL0 = B_VEMPTY0 + 4, B_PFULL0 = B_SFULL0 + kSBuf, B_PDONE0 = B_PFULL0 + 2 * kSBuf,
+  B_LFULL0 = B_PDONE0 + 2 * kSBuf, B_LFULL1, B_LEMPTY0, B_LEMPTY1, B_OFULL, B_OFREE, B_LX, B_DRAIN, B_COUNT
 };
+static_assert(B_COUNT <= 40, "barrier slots");
 
 struct AttnParams {
   const int32_t* idx;      // [B, heads, ntv_max, k_max]
   const int32_t* counts;   // [heads, nt_max]
   const WorkItem* items;
   int64_t n_items;
-  const __nv_bfloat16* q;  // packed Q (its rows go to TMEM once per item)
   __nv_bfloat16* out;      // packed O
   float* lse;
   uint32_t* state;         // [0] error word, [1] work counter, [2..3] computed pairs
@@ -324,7 +339,8 @@ __device__ __forceinline__ int warp_excl_scan(int v, int lane, int* total) {
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+    attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                const __grid_constant__ CUtensorMap tv,
                 const __grid_constant__ AttnParams prm) {
   using L = Smem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -345,25 +361,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(B_QREADY), 256);
+    mbar_init(bar(B_QFULL), 1);
+    mbar_init(bar(B_QEMPTY), 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(bar(B_KFULL0 + i), 1);
       mbar_init(bar(B_KEMPTY0 + i), 1);
       mbar_init(bar(B_VFULL0 + i), 1);
       mbar_init(bar(B_VEMPTY0 + i), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(B_SFULL0 + i), 1);
-      mbar_init(bar(B_MX0 + i), 256);
-      mbar_init(bar(B_LFULL0 + i), 32);
-      mbar_init(bar(B_LEMPTY0 + i), 256);
+    for (int i = 0; i < kSBuf; ++i) mbar_init(bar(B_SFULL0 + i), 1);
+    for (int i = 0; i < 2 * kSBuf; ++i) {
+      mbar_init(bar(B_PFULL0 + i), kSmWarps / 2);   // the four warps of one softmax warpgroup
+      mbar_init(bar(B_PDONE0 + i), 1);
     }
-    mbar_init(bar(B_PFULL), 256);
-    mbar_init(bar(B_PDONE), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_LFULL0 + i), 32);
+      mbar_init(bar(B_LEMPTY0 + i), kSmWarps);
+    }
     mbar_init(bar(B_OFULL), 1);
-    mbar_init(bar(B_OFREE), 256);
-    mbar_init(bar(B_LX), 256);
-    mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_OFREE), kSmWarps);
+    mbar_init(bar(B_LX), kSmWarps);
+    mbar_init(bar(B_DRAIN), 2);   // both MMA issuers
     misc[1] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -376,16 +394,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
-  // TMEM columns: S0 [0,128) and S1 [128,256) for alternate key blocks,
-  // O [256, 256+D), Q [384, 384+D/2) (bf16 pairs: two channels per 32-bit
-  // column; the A operand of S = Q K^T). P (bf16 pairs) is written over the S
-  // columns it was computed from: keys 0-63 at [0,32), keys 64-127 at [64,96)
-  // of the buffer. The next S MMA into a buffer is issued after the PV MMA
-  // that reads its P, and one thread's tcgen05.mma operations execute in issue
-  // order.
+  // TMEM columns: S buffers [0,128) and [128,256) for alternate key blocks;
+  // O_0 [256, 256+D) and O_1 [384, 384+D), the partial outputs of the two
+  // softmax warpgroups (keys of tile 0 / tile 1 of every block). P (bf16
+  // pairs) is written over the S columns it was computed from: keys 0-63 at
+  // [0,32), keys 64-127 at [64,96) of the buffer. S for block g + 2 is issued
+  // only after both PV MMAs that read P of block g have completed.
   const uint32_t tS = tmem;
-  const uint32_t tO = tmem + 256;
-  const uint32_t tQ = tmem + 384;
+  const uint32_t tO0 = tmem + 256;
+  static_assert(D <= 128, "each O fits 128 columns");
 
   if (warp == 2) {
     // ------------------------------------------------ scheduler / lists ---
@@ -504,13 +521,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       mbar_arrive(bar(B_LFULL0 + slot));
     }
-  } else if (warp == 0 || warp == 3) {
+  } else if (warp == 0) {
     // --------------------------------------------------------- producers ---
-    // warp 0: the K tile pairs; warp 3: the V tile
-    // pairs. Separate threads, so a K load never queues behind a V load that
-    // is waiting for its stage to be released by a PV MMA.
-    if (lane == 0) {
-      const bool is_k = warp == 0;
+    // lane 0: the Q pair of every item and the K tile pairs; lane 1: the V tile
+    // pairs. Separate threads (diverged lanes make independent progress), so a
+    // K load never queues behind a V load that is waiting for its stage to be
+    // released by a PV MMA.
+    if (lane < 2) {
+      const bool is_k = lane == 0;
       const CUtensorMap* map = is_k ? &tk : &tv;
       const int full0 = is_k ? B_KFULL0 : B_VFULL0;
       const int empty0 = is_k ? B_KEMPTY0 : B_VEMPTY0;
@@ -518,6 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t g = 0;          // key blocks issued
       int st = 0;              // stage of block g (g mod nst)
       uint32_t ph = 0;         // phase of that stage ((g / nst) & 1)
+      uint32_t issuedQ = 0;    // Q loads issued
       for (uint32_t it = 0;; ++it) {
         const int slot = it & 1;
         if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr)) break;
@@ -525,6 +544,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (inf.end) break;
         const uint32_t* list = lists + slot * prm.list_cap;
         const int row_base = inf.bh * prm.nt_max;
+        if (is_k) {   // rows 0-63: tile qa, rows 64-127: tile qb (qa again when there is none)
+          if (!wait_bar(bar(B_QEMPTY), (it & 1) ^ 1, abort_flag, gerr)) break;
+          mbar_expect_tx(bar(B_QFULL), 2 * (D / 64) * kTileBytes);
+          const int qb = inf.qb >= 0 ? inf.qb : inf.qa;
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(sbase + L::oQ + c * L::kHalfBytes, &tq, 64 * c, (row_base + inf.qa) * 64, bar(B_QFULL));
+            tma_load_2d(sbase + L::oQ + c * L::kHalfBytes + 8192, &tq, 64 * c, (row_base + qb) * 64, bar(B_QFULL));
+          }
+          ++issuedQ;
+        }
         const int nblk = (inf.n_entries + 1) >> 1;
         bool ok = true;
         for (int j = 0; j < nblk; ++j) {
@@ -555,92 +584,130 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*abort_flag) {
         // let every copy this thread issued land before shared memory is released
+        if (is_k && issuedQ) drain_wait(bar(B_QFULL), (issuedQ - 1) & 1);
         for (uint32_t gg = (g >= uint32_t(nst) ? g - nst : 0); gg < g; ++gg)
           drain_wait(bar(full0 + int(gg % nst)), (gg / nst) & 1);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // --------------------------------------------------------------- MMA ---
+    // ------------------------------------------------------------- S MMA ---
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t idPV = idesc_bf16(128, D, 0, 1);
-      // descriptors of the first stage; a stage or k-step adds (byte offset >> 4)
+      // descriptors of the stage bases; a stage or k-step adds (byte offset >> 4)
+      const uint64_t dq = sw128_desc(sbase + L::oQ, 16, 1024);
       const uint64_t dk0 = sw128_desc(sbase + L::oK, 16, 1024);
-      const uint64_t dv0 = sw128_desc(sbase + L::oV, 8192, 1024);
-      int kst = 0, vst = 0;      // K / V stage of the next S / PV MMA
-      uint32_t kph = 0, vph = 0; // their phases
-      uint32_t g = 0;            // key blocks so far
+      int kst = 0;               // K stage of the next S MMA
+      uint32_t kph = 0;          // its phase
+      int sb = 0;                // S buffer of block g (g mod kSBuf)
+      uint32_t su = 0;           // uses of that buffer before block g (g / kSBuf)
       bool ok = true;
-      // O += P V for block gg (global) = block jj of the item
-      auto issue_pv = [&](uint32_t gg, int jj, uint32_t it) -> bool {
-        if (jj == 0 && !wait_bar(bar(B_OFREE), (it & 1) ^ 1, abort_flag, gerr)) return false;
-        if (!wait_bar(bar(B_PFULL), gg & 1, abort_flag, gerr)) return false;
-        if (!wait_bar(bar(B_VFULL0 + vst), vph, abort_flag, gerr)) return false;
-        tc_fence_after();
-        const uint32_t pcol = tS + (gg & 1) * 128;
-        const uint64_t dv = dv0 + ((vst * L::kVBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // 16 keys per step: 8 TMEM columns of P
-          const uint32_t boff = ((kk >> 2) * (D / 64) * 8192 + (kk & 3) * 2048) >> 4;
-          tc_mma_ts(tO, pcol + (kk >> 2) * 64 + (kk & 3) * 8, dv + boff, idPV, (jj == 0 && kk == 0) ? 0u : 1u);
-        }
-        tc_commit(bar(B_VEMPTY0 + vst));
-        tc_commit(bar(B_PDONE));
-        if (++vst == L::kVStages) {
-          vst = 0;
-          vph ^= 1;
-        }
-        return true;
-      };
       for (uint32_t it = 0; ok; ++it) {
         const int slot = it & 1;
         if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr)) break;
         const ItemInfo inf = info[slot];
         if (inf.end) break;
-        if (!wait_bar(bar(B_QREADY), it & 1, abort_flag, gerr)) break;   // Q rows in TMEM
+        if (!wait_bar(bar(B_QFULL), it & 1, abort_flag, gerr)) break;
         const int nblk = (inf.n_entries + 1) >> 1;
-        for (int j = 0; j < nblk; ++j, ++g) {
+        if (nblk == 0) tc_commit(bar(B_QEMPTY));   // a rejected item without prefix tiles
+        for (int j = 0; j < nblk; ++j) {
           if (!(ok = wait_bar(bar(B_KFULL0 + kst), kph, abort_flag, gerr))) break;
+          // the buffer's previous P has been read by both PV MMAs
+          if (su > 0 && !(ok = wait_bar(bar(B_PDONE0 + sb), (su - 1) & 1, abort_flag, gerr))) break;
+          if (su > 0 && !(ok = wait_bar(bar(B_PDONE0 + kSBuf + sb), (su - 1) & 1, abort_flag, gerr))) break;
           tc_fence_after();
           const uint64_t dk = dk0 + ((kst * L::kKBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {   // S = Q K^T, 16 channels per step
+          for (int kk = 0; kk < D / 16; ++kk) {   // 16 channels per step
             const uint32_t off = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
-            tc_mma_ts(tS + (g & 1) * 128, tQ + kk * 8, dk + off, idS, kk > 0 ? 1u : 0u);
+            tc_mma(tS + sb * 128, dq + off, dk + off, idS, kk > 0 ? 1u : 0u);
           }
-          tc_commit(bar(B_SFULL0 + (g & 1)));
+          tc_commit(bar(B_SFULL0 + sb));
           tc_commit(bar(B_KEMPTY0 + kst));
+          if (j == nblk - 1) tc_commit(bar(B_QEMPTY));
           if (++kst == L::kKStages) {
             kst = 0;
             kph ^= 1;
           }
-          if (j > 0 && !(ok = issue_pv(g - 1, j - 1, it))) break;
+          if (++sb == kSBuf) {
+            sb = 0;
+            ++su;
+          }
         }
-        if (!ok) break;
-        if (!(ok = issue_pv(g - 1, nblk - 1, it))) break;
-        tc_commit(bar(B_OFULL));
       }
       // nothing of ours may still run on the tensor core when TMEM is freed
       tc_commit(bar(B_DRAIN));
       drain_wait(bar(B_DRAIN), 0);
     }
     __syncwarp();
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------ PV MMA ---
+    if (lane == 0) {
+      constexpr uint32_t idPV = idesc_bf16(128, D, 0, 1);
+      const uint64_t dv0 = sw128_desc(sbase + L::oV, 8192, 1024);
+      int vst = 0;               // V stage of the next PV MMA
+      uint32_t vph = 0;
+      int sb = 0;                // S buffer holding P of block g
+      uint32_t su = 0;
+      bool ok = true;
+      for (uint32_t it = 0; ok; ++it) {
+        const int slot = it & 1;
+        if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr)) break;
+        const ItemInfo inf = info[slot];
+        if (inf.end) break;
+        const int nblk = (inf.n_entries + 1) >> 1;
+        // O is free once the previous item's epilogue has read it
+        if (!wait_bar(bar(B_OFREE), (it & 1) ^ 1, abort_flag, gerr)) break;
+        if (nblk == 0) tc_commit(bar(B_OFULL));    // nothing to accumulate; the epilogue skips it
+        for (int j = 0; j < nblk; ++j) {
+          if (!(ok = wait_bar(bar(B_VFULL0 + vst), vph, abort_flag, gerr))) break;
+          const uint64_t dv = dv0 + ((vst * L::kVBytes) >> 4);
+          // O_w += P_w V_w: keys of tile w (64) against tile w of the V pair
+          for (int w = 0; w < 2 && ok; ++w) {
+            if (!(ok = wait_bar(bar(B_PFULL0 + w * kSBuf + sb), su & 1, abort_flag, gerr))) break;
+            tc_fence_after();
+            const uint32_t pcol = tS + sb * 128 + w * 64;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {   // 16 keys per step: 8 TMEM columns of P
+              const uint32_t boff = (w * (D / 64) * 8192 + kk * 2048) >> 4;
+              tc_mma_ts(tO0 + w * 128, pcol + kk * 8, dv + boff, idPV, (j == 0 && kk == 0) ? 0u : 1u);
+            }
+            tc_commit(bar(B_PDONE0 + w * kSBuf + sb));
+          }
+          if (!ok) break;
+          tc_commit(bar(B_VEMPTY0 + vst));
+          if (j == nblk - 1) tc_commit(bar(B_OFULL));
+          if (++vst == L::kVStages) {
+            vst = 0;
+            vph ^= 1;
+          }
+          if (++sb == kSBuf) {
+            sb = 0;
+            ++su;
+          }
+        }
+      }
+      tc_commit(bar(B_DRAIN));
+      drain_wait(bar(B_DRAIN), 0);
+    }
+    __syncwarp();
   } else if (warp >= 4) {
     // ----------------------------------------------------------- softmax ---
-    // Two warpgroups share every row (row = TMEM lane): warpgroup sg handles
-    // key tile sg of each 128-key block (S columns [64 sg, 64 sg + 64)) and O
-    // columns [sg D/2, (sg+1) D/2). They exchange each block's row max through
-    // shared memory and keep the same running max m; it is raised only when a
-    // block exceeds it by more than kLazy (log2 units), so P < 2^kLazy and O
-    // is rarely rescaled. At the start of an item each thread puts its half of
-    // its Q row into TMEM.
+    // Warpgroup sg owns key tile sg of every 128-key block (S columns
+    // [64 sg, 64 sg + 64)) for all 128 rows (row = TMEM lane) and keeps its own
+    // online softmax: running max m, row sum l and partial output O_sg. The
+    // two warpgroups never wait for each other inside an item, so one can
+    // compute exponentials while the other loads and reduces its scores. The
+    // running max is raised only when a tile exceeds it by more than kLazy
+    // (log2 units), so P < 2^kLazy and O_sg is rarely rescaled. The epilogue
+    // merges the two partial softmaxes of each row.
     const int sg = (warp - 4) >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     const uint32_t my_bit = r < 64 ? 1u : 2u;
-    float* xm = reinterpret_cast<float*>(smem + L::oXchg);   // [2 buffers][2 groups][128] block row max
-    float* xl = xm + 2 * 2 * 128;                           // [2 groups][128] row sums
+    const uint32_t tOw = tO0 + sg * 128 + lane_off;          // my warpgroup's O, my row
+    float* xm = reinterpret_cast<float*>(smem + L::oXchg);   // [2 groups][128] row max
+    float* xl = xm + 2 * 128;                               // [2 groups][128] row sums
     const uint64_t c2 = f2pack(prm.scale_log2, prm.scale_log2);
     uint32_t g = 0;
     bool ok = true;
@@ -652,49 +719,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (inf.end) break;
       const uint32_t* list = lists + slot * prm.list_cap;
       const int nblk = (inf.n_entries + 1) >> 1;
-      {  // Q: this thread's row, channels [sg D/2, (sg+1) D/2), as bf16 pairs
-        const int tile = r < 64 ? inf.qa : inf.qb;
-        uint32_t qw[D / 4];
-        if (tile >= 0) {
-          const uint4* src = reinterpret_cast<const uint4*>(
-              prm.q + ((size_t(inf.bh) * prm.nt_max + tile) * 64 + (r & 63)) * D + sg * (D / 2));
-#pragma unroll
-          for (int i = 0; i < D / 16; ++i) {
-            const uint4 u = src[i];
-            qw[4 * i] = u.x;
-            qw[4 * i + 1] = u.y;
-            qw[4 * i + 2] = u.z;
-            qw[4 * i + 3] = u.w;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < D / 4; ++i) qw[i] = 0u;
-        }
-        if constexpr (D == 128) {
-          tmem_st32u(tQ + lane_off + sg * 32, qw);
-        } else {
-          tmem_st16u(tQ + lane_off + sg * 16, qw);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(B_QREADY));
-      }
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < nblk; ++j, ++g) {
-        const int b = g & 1;
-        const uint32_t tSb = tS + b * 128 + lane_off;
-        ok = wait_bar(bar(B_SFULL0 + b), (g >> 1) & 1, abort_flag, gerr);
+        const int sbuf = int(g % kSBuf);           // S / P buffer
+        const uint32_t sph = (g / kSBuf) & 1;      // its phase
+        const uint32_t tSb = tS + sbuf * 128 + lane_off + 64 * sg;
+        ok = wait_bar(bar(B_SFULL0 + sbuf), sph, abort_flag, gerr);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
         const int ei = 2 * j + sg;
         const uint32_t e = ei < inf.n_entries ? list[ei] : 0u;
         const int cnt = ((e >> 16) & my_bit) ? int(e >> 24) : 0;   // valid keys of my tile for my row
-        float sv[64];
-        float tmx = -INFINITY;
+        float alpha = 1.f;
+        uint32_t pk[32];
         if (cnt > 0) {
+          float sv[64];
           uint32_t sr[2][32];
-          tmem_ld32(tSb + 64 * sg, sr[0]);
-          tmem_ld32(tSb + 64 * sg + 32, sr[1]);
+          tmem_ld32(tSb, sr[0]);
+          tmem_ld32(tSb + 32, sr[1]);
           tmem_wait_ld(sr[0]);
           reg_fence(sr[1]);
 #pragma unroll
@@ -711,22 +753,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 3; c < 15; c += 2) t = fmax3(t, sv[16 * q + c], sv[16 * q + c + 1]);
             mq[q] = fmaxf(t, sv[16 * q + 15]);
           }
-          tmx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-        }
-        // the block's row max from both warpgroups (raw scores; the scale is positive)
-        xm[(b * 2 + sg) * 128 + r] = tmx;
-        mbar_arrive(bar(B_MX0 + b));
-        ok = wait_bar(bar(B_MX0 + b), (g >> 1) & 1, abort_flag, gerr);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        const float bmx = fmaxf(xm[(b * 2) * 128 + r], xm[(b * 2 + 1) * 128 + r]) * prm.scale_log2;
-        float alpha = 1.f;
-        if (bmx > m + kLazy) {                     // also taken when m is still -inf
-          alpha = m == -INFINITY ? 1.f : ex2(m - bmx);
-          m = bmx;
-        }
-        l *= alpha;
-        uint32_t pk[32];
-        if (cnt > 0) {
+          // raw scores; the scale is positive
+          const float bmx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * prm.scale_log2;
+          if (bmx > m + kLazy) {                   // also taken when m is still -inf
+            alpha = m == -INFINITY ? 1.f : ex2(m - bmx);
+            m = bmx;
+          }
           const uint64_t nm2 = f2pack(-m, -m);
           uint64_t acc[2] = {0ull, 0ull};
           if (cnt == 64) {
@@ -758,75 +790,90 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           float r0, r1;
           f2unpack(fadd2(acc[0], acc[1]), r0, r1);
-          l += r0 + r1;
+          l = l * alpha + (r0 + r1);
         } else {                                   // my row-half does not keep this tile
 #pragma unroll
           for (int i = 0; i < 32; ++i) pk[i] = 0u;
         }
-        // P over my tile's consumed S columns: [64 sg, 64 sg + 32)
-        tmem_st32u(tSb + 64 * sg, pk);
-        // earlier blocks of this item sit in O at the old max: rescale my half of
-        // O once the previous PV has finished accumulating into it
+        // P over the first half of my consumed S columns
+        tmem_st32u(tSb, pk);
+        // earlier blocks of this item sit in O_sg at the old max: rescale it
+        // once my previous PV has finished accumulating into it
         if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
-          ok = wait_bar(bar(B_PDONE), (g - 1) & 1, abort_flag, gerr);
+          const uint32_t gp = g - 1;
+          ok = wait_bar(bar(B_PDONE0 + sg * kSBuf + int(gp % kSBuf)), (gp / kSBuf) & 1, abort_flag, gerr);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < D / 64; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t orr[32];
-            const uint32_t col = tO + lane_off + sg * (D / 2) + 32 * c;
-            tmem_ld32(col, orr);
+            tmem_ld32(tOw + 32 * c, orr);
             tmem_wait_ld(orr);
             float o[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(orr[i]) * alpha;
-            tmem_st32(col, o);
+            tmem_st32(tOw + 32 * c, o);
           }
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_PFULL));
+        warp_arrive(bar(B_PFULL0 + sg * kSBuf + sbuf));
       }
       if (!ok) break;
-      // epilogue: O is final once the item's last PV is done; the row sum is the two groups' sum
+      // epilogue: both partial outputs are final once the item's last PV is
+      // done. Row r's two partial softmaxes (m_0, l_0, O_0) and (m_1, l_1, O_1)
+      // merge as O = sum_w 2^(m_w - M) O_w / sum_w 2^(m_w - M) l_w, M = max m_w;
+      // warpgroup sg writes channels [sg D/2, (sg+1) D/2).
       ok = wait_bar(bar(B_OFULL), it & 1, abort_flag, gerr);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
+      xm[sg * 128 + r] = m;
       xl[sg * 128 + r] = l;
-      mbar_arrive(bar(B_LX));
+      warp_arrive(bar(B_LX));
       ok = wait_bar(bar(B_LX), it & 1, abort_flag, gerr);
       if (!__all_sync(0xffffffffu, ok)) break;
-      const float lrow = xl[r] + xl[128 + r];
+      const float m0 = xm[r], m1 = xm[128 + r];
+      const float mrow = fmaxf(m0, m1);
+      const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - mrow);
+      const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - mrow);
+      const float lrow = xl[r] * a0 + xl[128 + r] * a1;
       const int tile = r < 64 ? inf.qa : inf.qb;
       const int slot_r = r & 63;
       const int rows = r < 64 ? inf.rows_a : inf.rows_b;
       const bool write = tile >= 0 && !inf.bad;
       const bool valid = write && slot_r < rows;
       const float inv = (valid && lrow > 0.f) ? 1.f / lrow : 0.f;
+      const float w0 = a0 * inv, w1 = a1 * inv;
       const size_t orow = (size_t(inf.bh) * prm.nt_max + (tile >= 0 ? tile : 0)) * 64 + slot_r;
       uint4* dst = reinterpret_cast<uint4*>(prm.out + orow * D + sg * (D / 2));
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
-        uint32_t orr[32];
-        tmem_ld32(tO + lane_off + sg * (D / 2) + 32 * c, orr);
-        tmem_wait_ld(orr);
+        uint32_t o0[32], o1[32];
+        tmem_ld32(tO0 + lane_off + sg * (D / 2) + 32 * c, o0);
+        tmem_ld32(tO0 + 128 + lane_off + sg * (D / 2) + 32 * c, o1);
+        tmem_wait_ld(o0);
+        reg_fence(o1);
         if (write) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              v[i] = __uint_as_float(o0[8 * q + i]) * w0 + __uint_as_float(o1[8 * q + i]) * w1;
             uint4 pkq;
-            pkq.x = bf16x2(__uint_as_float(orr[8 * q + 0]) * inv, __uint_as_float(orr[8 * q + 1]) * inv);
-            pkq.y = bf16x2(__uint_as_float(orr[8 * q + 2]) * inv, __uint_as_float(orr[8 * q + 3]) * inv);
-            pkq.z = bf16x2(__uint_as_float(orr[8 * q + 4]) * inv, __uint_as_float(orr[8 * q + 5]) * inv);
-            pkq.w = bf16x2(__uint_as_float(orr[8 * q + 6]) * inv, __uint_as_float(orr[8 * q + 7]) * inv);
+            pkq.x = bf16x2(v[0], v[1]);
+            pkq.y = bf16x2(v[2], v[3]);
+            pkq.z = bf16x2(v[4], v[5]);
+            pkq.w = bf16x2(v[6], v[7]);
             dst[c * 4 + q] = pkq;
           }
         }
       }
       if (write && sg == 0 && prm.lse)
-        prm.lse[orow] = valid && lrow > 0.f ? (m + __log2f(lrow)) * 0.69314718055994531f : 0.f;
+        prm.lse[orow] = valid && lrow > 0.f ? (mrow + __log2f(lrow)) * 0.69314718055994531f : 0.f;
       tc_fence_before();
-      mbar_arrive(bar(B_OFREE));
-      mbar_arrive(bar(B_LEMPTY0 + slot));
+      warp_arrive(bar(B_OFREE));
+      warp_arrive(bar(B_LEMPTY0 + slot));
     }
   }
 
@@ -879,14 +926,14 @@ cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void*
                         float* lse, cudaStream_t s) {
   const Geometry& g = p->geo;
   const int64_t rows = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE;
-  CUtensorMap tk, tv;
-  if (!make_map(&tk, kp, rows, g.d) || !make_map(&tv, vp, rows, g.d)) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, qp, rows, g.d) || !make_map(&tk, kp, rows, g.d) || !make_map(&tv, vp, rows, g.d))
+    return cudaErrorInvalidValue;
   AttnParams prm;
   prm.idx = idx;
   prm.counts = p->d_tile_count;
   prm.items = p->d_items;
   prm.n_items = p->n_items;
-  prm.q = static_cast<const __nv_bfloat16*>(qp);
   prm.out = static_cast<__nv_bfloat16*>(op);
   prm.lse = lse;
   prm.state = p->d_state;
@@ -912,11 +959,11 @@ cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void*
   if (g.d == 128) {
     e = cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel<128><<<grid, kThreads, smem, s>>>(tk, tv, prm);
+    attn_kernel<128><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm);
   } else {
     e = cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_kernel<64><<<grid, kThreads, smem, s>>>(tk, tv, prm);
+    attn_kernel<64><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm);
   }
   return cudaGetLastError();
 }

@@ -15,26 +15,29 @@
 // which of the two row-halves keeps it; a row-half masks the other's tiles to
 // -inf. Key tiles go through smem two at a time (128 keys per step).
 //
-// Warp roles (384 threads):
+// Warp roles (416 threads):
 //   warp 0  TMA producers: lane 0 the Q pair of every block of rows and the K
 //           tile pairs (2 stages), lane 1 the V tile pairs (3 stages)
-//   warp 1  MMA issuer for S = Q K^T (Q and K in smem) into one of three TMEM
+//   warp 1  MMA issuer for S = Q K^T (Q and K in smem) into one of two TMEM
 //           S buffers
-//   warp 3  MMA issuer for O += P V (P in TMEM over the S columns it came
-//           from, V in smem)
+//   warps 3, 12  MMA issuers for O_0 += P_0 V_0 and O_1 += P_1 V_1 (P in
+//           TMEM over the S columns it came from, V in smem)
 //   warp 2  scheduler: fetches the next block from a global counter and builds
 //           its merged key list (double buffered, in a per-CTA global slice)
-//   warps 4-11 softmax, two warpgroups: row r (TMEM lane r) is shared by one
-//           thread of each; warpgroup g handles key tile g of every 128-key
-//           block and half of O's columns. They exchange the block row max and
-//           keep one lazily raised running max; P goes back to TMEM as bf16
-//           over the consumed S columns.
+//   warps 4-11 softmax, two warpgroups: warpgroup w owns key tile w of every
+//           128-key block for all 128 rows (row = TMEM lane) with its own
+//           online softmax (running max, row sum, partial output O_w); the
+//           epilogue merges the two partial softmaxes of each row.
 //
-// One thread can have only one tcgen05.mma in execution at a time, and an
-// M = 128, K = 16 MMA takes about as long for N = 128 as for N = 256; S and PV
-// therefore come from two issuing threads, and three S buffers let S for the
-// next blocks run while PV drains the previous one.
+// One thread's tcgen05.mma stream runs one M = 128, K = 16 instruction at a
+// time, about as long for N = 128 as for N = 256, so S and the two PV halves
+// come from three issuing threads. The softmax warpgroups never wait for each
+// other inside an item, so one computes exponentials while the other loads
+// and reduces its scores.
 //
+// TMEM holds the two S buffers and the two partial outputs; shared memory the
+// Q pair and the K and V stages, in the canonical 128-byte-swizzled UMMA
+// layouts that TMA SWIZZLE_128B writes (Q and K K-major, V MN-major).
 // Every wait is bounded (about two seconds); on expiry the CTA latches a
 // timeout in the plan's error word, drains its copies and MMAs, frees TMEM and
 // returns.
@@ -48,9 +51,10 @@
 namespace vsa {
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 416;
 constexpr int kSBuf = 2;        // TMEM S buffers
-constexpr int kPvWarp = 3;      // the PV MMA issuer
+constexpr int kPvWarp0 = 3;     // PV MMA issuer for softmax warpgroup 0's keys
+constexpr int kPvWarp1 = 12;    // ... and for warpgroup 1's
 constexpr int kSmWarps = 8;     // softmax warps (4-11); each arrives once on their barriers
 constexpr float kLazy = 8.0f;  // log2 headroom before the running max is raised
 constexpr uint32_t kTmemCols = 512;
@@ -367,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_KFULL0 + i), 1);
       mbar_init(bar(B_KEMPTY0 + i), 1);
       mbar_init(bar(B_VFULL0 + i), 1);
-      mbar_init(bar(B_VEMPTY0 + i), 1);
+      mbar_init(bar(B_VEMPTY0 + i), 2);   // both PV issuers
     }
     for (int i = 0; i < kSBuf; ++i) mbar_init(bar(B_SFULL0 + i), 1);
     for (int i = 0; i < 2 * kSBuf; ++i) {
@@ -378,10 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_LFULL0 + i), 32);
       mbar_init(bar(B_LEMPTY0 + i), kSmWarps);
     }
-    mbar_init(bar(B_OFULL), 1);
+    mbar_init(bar(B_OFULL), 2);
     mbar_init(bar(B_OFREE), kSmWarps);
     mbar_init(bar(B_LX), kSmWarps);
-    mbar_init(bar(B_DRAIN), 2);   // both MMA issuers
+    mbar_init(bar(B_DRAIN), 3);   // the three MMA issuers
     misc[1] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -640,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(bar(B_DRAIN), 0);
     }
     __syncwarp();
-  } else if (warp == kPvWarp) {
+  } else if (warp == kPvWarp0 || warp == kPvWarp1) {
     // ------------------------------------------------------------ PV MMA ---
     if (lane == 0) {
       constexpr uint32_t idPV = idesc_bf16(128, D, 0, 1);
@@ -649,6 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t vph = 0;
       int sb = 0;                // S buffer holding P of block g
       uint32_t su = 0;
+      const int w = warp == kPvWarp0 ? 0 : 1;   // O_w += P_w V_w: keys of tile w of every block
       bool ok = true;
       for (uint32_t it = 0; ok; ++it) {
         const int slot = it & 1;
@@ -662,19 +667,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < nblk; ++j) {
           if (!(ok = wait_bar(bar(B_VFULL0 + vst), vph, abort_flag, gerr))) break;
           const uint64_t dv = dv0 + ((vst * L::kVBytes) >> 4);
-          // O_w += P_w V_w: keys of tile w (64) against tile w of the V pair
-          for (int w = 0; w < 2 && ok; ++w) {
-            if (!(ok = wait_bar(bar(B_PFULL0 + w * kSBuf + sb), su & 1, abort_flag, gerr))) break;
-            tc_fence_after();
-            const uint32_t pcol = tS + sb * 128 + w * 64;
+          if (!(ok = wait_bar(bar(B_PFULL0 + w * kSBuf + sb), su & 1, abort_flag, gerr))) break;
+          tc_fence_after();
+          const uint32_t pcol = tS + sb * 128 + w * 64;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {   // 16 keys per step: 8 TMEM columns of P
-              const uint32_t boff = (w * (D / 64) * 8192 + kk * 2048) >> 4;
-              tc_mma_ts(tO0 + w * 128, pcol + kk * 8, dv + boff, idPV, (j == 0 && kk == 0) ? 0u : 1u);
-            }
-            tc_commit(bar(B_PDONE0 + w * kSBuf + sb));
+          for (int kk = 0; kk < 4; ++kk) {   // 16 keys per step: 8 TMEM columns of P
+            const uint32_t boff = (w * (D / 64) * 8192 + kk * 2048) >> 4;
+            tc_mma_ts(tO0 + w * 128, pcol + kk * 8, dv + boff, idPV, (j == 0 && kk == 0) ? 0u : 1u);
           }
-          if (!ok) break;
+          tc_commit(bar(B_PDONE0 + w * kSBuf + sb));
           tc_commit(bar(B_VEMPTY0 + vst));
           if (j == nblk - 1) tc_commit(bar(B_OFULL));
           if (++vst == L::kVStages) {
@@ -691,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(bar(B_DRAIN), 0);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 12) {
     // ----------------------------------------------------------- softmax ---
     // Warpgroup sg owns key tile sg of every 128-key block (S columns
     // [64 sg, 64 sg + 64)) for all 128 rows (row = TMEM lane) and keeps its own

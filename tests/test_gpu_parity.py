@@ -156,3 +156,26 @@ def test_argument_errors():
     st = T.vsa.library().vsa_tile_unpack(r.plan._h, T.vsa.ctypes.c_void_p(bad.data_ptr()),
                                          T.vsa.ctypes.c_void_p(r.out.data_ptr()), None)
     assert st == 1
+
+
+def test_running_max_jumps_late_in_the_row():
+    """Keys of the last video frames scaled by 6: their scores exceed every earlier
+    block's by far more than the lazy threshold, so the running max is raised late in
+    the row and the partial outputs are rescaled (prefix rows see every key)."""
+    import dataclasses
+    from vsa_synth import bf16_bits_to_f32, f32_to_bf16_bits
+    from vsa_synth.generate import make_layer_inputs
+    cfg = ragged_gpu_config(128)
+    inp = make_layer_inputs(cfg)
+    k = bf16_bits_to_f32(inp.k).reshape(cfg.batch, -1, cfg.heads, cfg.head_dim)
+    n_last = cfg.H * cfg.W * 2                       # tokens of the last two frames
+    k[:, -n_last:] *= 6.0
+    inp = dataclasses.replace(inp, k=f32_to_bf16_bits(k).reshape(inp.k.shape))
+    r = GpuRun(cfg, 0.5, inputs=inp).run()
+    q, kk, v = oracle_inputs_f64(r.inp)
+    kept = {(b, h): r.kept(b, h) for b in range(cfg.batch) for h in range(cfg.heads)}
+    res = O.run_layer(cfg, q, kk, v, r.k, gate=r.inp.gate, w_q=r.inp.w_q, w_k=r.inp.w_k, kept=kept)
+    # the jump is real: some prefix row's largest logit comes from the scaled keys
+    s = np.einsum("nd,md->nm", q[0, :64, 0], kk[0, :, 0]) * scale_of(cfg)
+    assert np.any(np.argmax(s, axis=1) >= s.shape[1] - n_last)
+    check_close(bf16_to_f64(r.out), res.out)

@@ -35,7 +35,7 @@ if ROOT not in sys.path:
 CONFIG = "full"
 SPARSITY = 0.75
 SECONDARY_SPARSITY = 0.9
-KERNELS_PER_STEP = 8  # pack 1, score 4 (pool, 2 projections, scores), select 1, attention 1, unpack 1
+KERNELS_PER_STEP = 7  # pack + pool 1, score 3 (2 projections, scores), select 1, attention 1, unpack 1
 
 
 def parse():
@@ -347,9 +347,9 @@ def run_ours(args, rank, world, local_rank):
         for i in range(steps):
             e = ev[i]
             e[0].record(stream)
-            p.tile_pack(q, k, v, b["qp"], b["kp"], b["vp"])
+            p.tile_pack_pool(q, k, v, b["qp"], b["kp"], b["vp"], b["workspace"])
             e[1].record(stream)
-            p.tile_score(b["qp"], b["kp"], pq, pk, b["scores"], b["workspace"])
+            p.tile_score_pooled(pq, pk, b["scores"], b["workspace"])
             e[2].record(stream)
             p.topk_select(b["scores"], b["idx"])
             e[3].record(stream)
@@ -363,7 +363,7 @@ def run_ours(args, rank, world, local_rank):
         layer.plan.check()
         total = sum(ev[i][0].elapsed_time(ev[i][5]) for i in range(steps))
         stages = {name: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps)) / steps
-                  for j, name in enumerate(("pack", "score", "select", "attn", "unpack"))}
+                  for j, name in enumerate(("pack_pool", "score", "select", "attn", "unpack"))}
         ms_step = max_over_ranks(total / steps)
         stats = layer.plan.stats()
         return layer, out, ms_step, stages, clocks, stats

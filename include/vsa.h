@@ -160,6 +160,24 @@ VSA_API vsa_status vsa_tile_score(vsa_plan* plan, const void* qp, const void* kp
                           const float* proj_q, const float* proj_k, float* scores,
                           void* workspace, void* stream);
 
+/* a1 + a2 in one pass (the fused form of the first two steps): pack Q, K and V
+ * exactly as vsa_tile_pack and, while each video tile's Q and K rows pass
+ * through, pool them as vsa_tile_score does (fp32 mean over the tile's valid
+ * tokens; TripPool adds max and min), writing the descriptors into
+ * `workspace` (>= workspace_bytes, 256-byte aligned). Follow with
+ * vsa_tile_score_pooled on the same workspace. q, k and v are all required.
+ * This saves the score stage's second read of packed Q and K. Same sources as
+ * vsa_tile_pack and vsa_tile_score (Ref2VA VSA README: mean-pooled gate score;
+ * BSAI VedaSparse README "Core Technology: TripPool", eq. 5). */
+VSA_API vsa_status vsa_tile_pack_pool(vsa_plan* plan, const void* q, const void* k, const void* v,
+                              void* qp, void* kp, void* vp, void* workspace, void* stream);
+
+/* a3-a4 of vsa_tile_score from the descriptors vsa_tile_pack_pool left in
+ * `workspace`: projection and tile scores, same arguments (less qp, kp),
+ * layout and results as vsa_tile_score. */
+VSA_API vsa_status vsa_tile_score_pooled(vsa_plan* plan, const float* proj_q, const float* proj_k,
+                                 float* scores, void* workspace, void* stream);
+
 /* The a2-a4 score stage of vsa_tile_score with its scratch in a fixed device
  * array owned by the library instead of a caller workspace, for callers that
  * may not allocate device memory while they run the layer: code under another
@@ -211,8 +229,10 @@ VSA_API vsa_status vsa_sparse_attn(vsa_plan* plan, const void* qp, const void* k
 /* a7. Inverse of the pack permutation: [B, heads, nt_max, 64, d] -> [B, N, heads, d]. */
 VSA_API vsa_status vsa_tile_unpack(vsa_plan* plan, const void* op, void* o, void* stream);
 
-/* All five calls in order on one stream, on caller-provided buffers (sizes
- * from vsa_plan_query). Returns the first failing call's status. */
+/* The whole layer in order on one stream, on caller-provided buffers (sizes
+ * from vsa_plan_query): vsa_tile_pack_pool, vsa_tile_score_pooled,
+ * vsa_topk_select, vsa_sparse_attn, vsa_tile_unpack. Returns the first
+ * failing call's status. */
 VSA_API vsa_status vsa_layer_forward(vsa_plan* plan, const void* q, const void* k, const void* v,
                              const float* proj_q, const float* proj_k,
                              void* qp, void* kp, void* vp, float* scores, int32_t* idx,

@@ -73,11 +73,17 @@ class GpuRun:
             self.proj_k = torch.from_numpy(self.inp.w_k).cuda()
         self.out = torch.empty_like(self.q)
 
-    def run(self, stages=True):
+    def run(self, stages=True, fused=False):
+        """The layer as separate calls (fused: pack and pooling in one call), or as one
+        vsa_layer_forward call (stages=False), which takes the fused path."""
         b, p = self.bufs, self.plan
         if stages:
-            p.tile_pack(self.q, self.k_t, self.v, b["qp"], b["kp"], b["vp"])
-            p.tile_score(b["qp"], b["kp"], self.proj_q, self.proj_k, b["scores"], b["workspace"])
+            if fused:
+                p.tile_pack_pool(self.q, self.k_t, self.v, b["qp"], b["kp"], b["vp"], b["workspace"])
+                p.tile_score_pooled(self.proj_q, self.proj_k, b["scores"], b["workspace"])
+            else:
+                p.tile_pack(self.q, self.k_t, self.v, b["qp"], b["kp"], b["vp"])
+                p.tile_score(b["qp"], b["kp"], self.proj_q, self.proj_k, b["scores"], b["workspace"])
             p.topk_select(b["scores"], b["idx"])
             p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], b["lse"])
             p.tile_unpack(b["op"], self.out)

@@ -37,6 +37,23 @@ def test_header_declares_binding_exports():
     assert header_functions() == sorted(V.EXPORTS)
 
 
+def header_arity():
+    """Parameter count of every function the header declares."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"^VSA_API\s+[\w\s\*]+?\b(vsa_\w+)\s*\(([^)]*)\)", text, re.M):
+        params = [x for x in m.group(2).split(",") if x.strip() and x.strip() != "void"]
+        out[m.group(1)] = len(params)
+    return out
+
+
+def test_binding_argument_counts_match_header(lib):
+    ar = header_arity()
+    assert sorted(ar) == header_functions()
+    for name, n in ar.items():
+        assert len(getattr(lib, name).argtypes) == n, name
+
+
 def test_library_exports_every_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", V.LIB_PATH], capture_output=True, text=True, check=True)
     syms = {ln.split()[-1] for ln in out.stdout.splitlines() if " T " in ln}

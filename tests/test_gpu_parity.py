@@ -25,16 +25,17 @@ CASES = {
 _runs = {}
 
 
-def gpu_run(name):
-    if name not in _runs:
+def gpu_run(name, fused=False):
+    if (name, fused) not in _runs:
         make, s = CASES[name]
-        _runs[name] = GpuRun(make(), s).run()
-    return _runs[name]
+        _runs[name, fused] = GpuRun(make(), s).run(fused=fused)
+    return _runs[name, fused]
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["pack", "pack_pool"])
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_pack_bit_exact(name):
-    r = gpu_run(name)
+def test_pack_bit_exact(name, fused):
+    r = gpu_run(name, fused)
     q, k, v = oracle_inputs_f64(r.inp)
     for src, packed in ((q, r.bufs["qp"]), (k, r.bufs["kp"]), (v, r.bufs["vp"])):
         want, counts = O.pack(src, r.cfg)
@@ -49,9 +50,10 @@ def test_pack_bit_exact(name):
     assert torch.equal(back.view(torch.int16), r.q.view(torch.int16))
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["pool", "pack_pool"])
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_scores_and_topk(name):
-    r = gpu_run(name)
+def test_scores_and_topk(name, fused):
+    r = gpu_run(name, fused)
     q, k, v = oracle_inputs_f64(r.inp)
     for b in range(r.cfg.batch):
         for h in range(r.cfg.heads):
@@ -67,9 +69,10 @@ def test_scores_and_topk(name):
                 assert np.array_equal(kept[i], O.topk_row(s_gpu[i], r.k[h]))
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["pack", "pack_pool"])
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_attention_matches_oracle(name):
-    r = gpu_run(name)
+def test_attention_matches_oracle(name, fused):
+    r = gpu_run(name, fused)
     q, k, v = oracle_inputs_f64(r.inp)
     kept = {(b, h): r.kept(b, h) for b in range(r.cfg.batch) for h in range(r.cfg.heads)}
     res = O.run_layer(r.cfg, q, k, v, r.k, gate=r.inp.gate, w_q=r.inp.w_q, w_k=r.inp.w_k, kept=kept)
@@ -104,12 +107,31 @@ def test_dense_when_k_is_all(name):
 
 def test_layer_forward_equals_stages_and_is_deterministic():
     import torch
-    r = gpu_run("ragged128_batch2")
+    r = gpu_run("ragged128_batch2", fused=True)
     first = r.out.clone()
-    r.run(stages=False)
+    r.run(stages=False)                    # vsa_layer_forward takes the fused path
     assert torch.equal(first.view(torch.int16), r.out.view(torch.int16))
-    r.run(stages=True)
+    r.run(stages=True, fused=True)
     assert torch.equal(first.view(torch.int16), r.out.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_pack_pool_descriptors_match_pool_stage(name):
+    """The fused pass writes the score stage's pooled descriptors: same layout, values equal
+    up to fp32 summation order (the separate pool sums rows in order, the fused one in a tree)."""
+    import torch
+    r0, r1 = gpu_run(name, False), gpu_run(name, True)
+    n = r0.cfg.batch * r0.cfg.heads * r0.plan.info.ntv_max
+    kd = 3 * r0.cfg.head_dim if r0.cfg.score_mode == "tripool" else r0.cfg.head_dim
+    off = ((n * kd * 4 + 255) // 256) * 256
+    for base in (0, off):                  # pooled Q, then pooled K
+        a = r0.bufs["workspace"][base:base + n * kd * 4].view(torch.float32).view(n, kd)
+        b = r1.bufs["workspace"][base:base + n * kd * 4].view(torch.float32).view(n, kd)
+        for bh in range(r0.cfg.batch * r0.cfg.heads):
+            h = bh % r0.cfg.heads
+            rows = slice(bh * r0.plan.info.ntv_max, bh * r0.plan.info.ntv_max + n_video_tiles(r0.cfg, h))
+            x, y = a[rows].double().cpu().numpy(), b[rows].double().cpu().numpy()
+            assert np.max(np.abs(x - y)) <= 1e-5 * max(1.0, np.max(np.abs(x)))
 
 
 def test_k_one_and_edges():

@@ -5,6 +5,7 @@
 // segment-pure prefix tiles) and BSAI VedaSparse README ("Core Technology:
 // Head-Aware Tiling", per-head (pt, ph, pw) with product 64).
 #include <cuda_runtime.h>
+#include <math.h>
 
 #include "vsa_internal.h"
 
@@ -100,6 +101,138 @@ __global__ void __launch_bounds__(256) unpack_kernel(Geometry g, const uint4* __
   }
 }
 
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float (&x)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// Pack fused with pooling (a1 + a2 in one pass over Q and K): one CTA per
+// (b, h, packed tile). Thread t moves chunk t mod CPR of rows t / CPR + RG*i of
+// Q, K and V, and for a video tile also sums (TripPool: max, min) its 8
+// channels of Q and K over those rows in fp32; the warps' partials are
+// combined through shared memory into the tile's descriptor, written in the
+// score stage's pooled layout [B*heads*ntv_max][KD]: mean (sum / valid
+// tokens), then max and min for TripPool. The pooling itself is that of the
+// score stage (Ref2VA VSA README: mean-pooled Q, K for the gate score; BSAI
+// VedaSparse README "Core Technology: TripPool", eq. 5).
+template <int CPR, bool TRIP>
+__global__ void __launch_bounds__(256) pack_pool_kernel(Geometry g, const uint4* __restrict__ q,
+                                                        const uint4* __restrict__ k,
+                                                        const uint4* __restrict__ v, uint4* __restrict__ qp,
+                                                        uint4* __restrict__ kp, uint4* __restrict__ vp,
+                                                        const int32_t* __restrict__ counts,
+                                                        float* __restrict__ pq, float* __restrict__ pk) {
+  constexpr int D = CPR * 8;
+  constexpr int KD = TRIP ? 3 * D : D;
+  constexpr int RG = 256 / CPR;       // row groups: 16 (d = 128) or 32 (d = 64)
+  constexpr int RPT = 64 / RG;        // rows per thread: 4 or 2
+  constexpr int NS = TRIP ? 3 : 1;    // statistics: sum (, max, min)
+  __shared__ float part[NS][2][8][D];
+  const int64_t tile = blockIdx.x;    // bh * nt_max + n
+  const int n = int(tile % g.nt_max);
+  const int bh = int(tile / g.nt_max);
+  const int h = bh % g.Hh, b = bh / g.Hh;
+  const int c = threadIdx.x % CPR;
+  const int rg = threadIdx.x / CPR;
+  const int vt = n - g.n_pre_tiles;
+  const bool pool = vt >= 0 && vt < g.ntv[h];   // uniform over the CTA
+  float st[NS][2][8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      st[0][t][e] = 0.f;
+      if (TRIP) {
+        st[NS - 2][t][e] = -INFINITY;
+        st[NS - 1][t][e] = INFINITY;
+      }
+    }
+  }
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const int s = rg + RG * i;
+    const int tok = src_token(g, h, n, s);
+    const int64_t dst = (tile * VSA_TILE + s) * CPR + c;
+    uint4 a = zero, bb = zero, cc = zero;
+    if (tok >= 0) {
+      const int64_t src = ((int64_t(b) * g.n_tokens + tok) * g.Hh + h) * CPR + c;
+      a = ld_stream(q + src);
+      bb = ld_stream(k + src);
+      cc = ld_stream(v + src);
+    }
+    qp[dst] = a;
+    kp[dst] = bb;
+    vp[dst] = cc;
+    if (pool && tok >= 0) {
+      float xq[8], xk[8];
+      bf16x8_to_f32(a, xq);
+      bf16x8_to_f32(bb, xk);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        st[0][0][e] += xq[e];
+        st[0][1][e] += xk[e];
+        if (TRIP) {
+          st[NS - 2][0][e] = fmaxf(st[NS - 2][0][e], xq[e]);
+          st[NS - 2][1][e] = fmaxf(st[NS - 2][1][e], xk[e]);
+          st[NS - 1][0][e] = fminf(st[NS - 1][0][e], xq[e]);
+          st[NS - 1][1][e] = fminf(st[NS - 1][1][e], xk[e]);
+        }
+      }
+    }
+  }
+  if (!pool) return;
+  // lanes l and l ^ CPR (and l ^ 2 CPR for d = 64) hold the same chunk of
+  // different rows: fold them so that lanes < CPR hold the warp's partials
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = CPR; o < 32; o <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        st[0][t][e] += __shfl_xor_sync(0xffffffffu, st[0][t][e], o);
+        if (TRIP) {
+          st[NS - 2][t][e] = fmaxf(st[NS - 2][t][e], __shfl_xor_sync(0xffffffffu, st[NS - 2][t][e], o));
+          st[NS - 1][t][e] = fminf(st[NS - 1][t][e], __shfl_xor_sync(0xffffffffu, st[NS - 1][t][e], o));
+        }
+      }
+    }
+  }
+  if (lane < CPR) {
+#pragma unroll
+    for (int z = 0; z < NS; ++z)
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) part[z][t][warp][8 * lane + e] = st[z][t][e];
+  }
+  __syncthreads();
+  if (threadIdx.x < 2 * D) {
+    const int t = threadIdx.x / D, ch = threadIdx.x % D;
+    float sum = 0.f, mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      sum += part[0][t][w][ch];
+      if (TRIP) {
+        mx = fmaxf(mx, part[NS - 2][t][w][ch]);
+        mn = fminf(mn, part[NS - 1][t][w][ch]);
+      }
+    }
+    const float cnt = float(counts[h * g.nt_max + n]);
+    float* out = (t ? pk : pq) + (int64_t(bh) * g.ntv_max + vt) * KD;
+    out[ch] = sum / cnt;
+    if (TRIP) {
+      out[D + ch] = mx;
+      out[2 * D + ch] = mn;
+    }
+  }
+}
+
 int grid_for(const vsa_plan* p, int64_t total) {
   const int64_t want = (total + 255) / 256;
   const int64_t cap = int64_t(p->num_sms) * 8;  // 8 blocks of 256 threads per SM
@@ -124,6 +257,28 @@ cudaError_t launch_pack(const vsa_plan* p, const void* q, const void* k, const v
     pack_kernel<16><<<grid, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4);
   else
     pack_kernel<8><<<grid, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_pool(const vsa_plan* p, const void* q, const void* k, const void* v, void* qp,
+                             void* kp, void* vp, float* pooled_q, float* pooled_k, cudaStream_t s) {
+  const Geometry& g = p->geo;
+  const int64_t tiles = int64_t(g.B) * g.Hh * g.nt_max;
+  const bool trip = p->desc.score_mode == VSA_SCORE_TRIPPOOL;
+  auto* q4 = static_cast<const uint4*>(q);
+  auto* k4 = static_cast<const uint4*>(k);
+  auto* v4 = static_cast<const uint4*>(v);
+  auto* qp4 = static_cast<uint4*>(qp);
+  auto* kp4 = static_cast<uint4*>(kp);
+  auto* vp4 = static_cast<uint4*>(vp);
+  const int32_t* cnt = p->d_tile_count;
+  if (g.d == 128) {
+    if (trip) pack_pool_kernel<16, true><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k);
+    else pack_pool_kernel<16, false><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k);
+  } else {
+    if (trip) pack_pool_kernel<8, true><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k);
+    else pack_pool_kernel<8, false><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k);
+  }
   return cudaGetLastError();
 }
 

@@ -189,8 +189,16 @@ __global__ void __launch_bounds__(256) sgemm_kernel(Geometry g, const float* __r
 
 int64_t score_workspace_bytes(const Geometry& g, int mode, int p) { return score_layout(g, mode, p).total; }
 
-cudaError_t launch_score(const vsa_plan* pl, const void* qp, const void* kp, const float* proj_q,
-                         const float* proj_k, float* scores, void* workspace, cudaStream_t s) {
+void score_pooled_ptrs(const vsa_plan* pl, void* workspace, float** pooled_q, float** pooled_k) {
+  const ScoreLayout L = score_layout(pl->geo, pl->desc.score_mode, pl->desc.proj_dim);
+  char* ws = static_cast<char*>(workspace);
+  *pooled_q = reinterpret_cast<float*>(ws + L.off_pq);
+  *pooled_k = reinterpret_cast<float*>(ws + L.off_pk);
+}
+
+// a3-a4 from the pooled descriptors already in the workspace.
+cudaError_t launch_project_score(const vsa_plan* pl, const float* proj_q, const float* proj_k, float* scores,
+                                 void* workspace, cudaStream_t s) {
   const Geometry& g = pl->geo;
   const int mode = pl->desc.score_mode;
   const int p = pl->desc.proj_dim;
@@ -202,6 +210,30 @@ cudaError_t launch_score(const vsa_plan* pl, const void* qp, const void* kp, con
   float* hk = reinterpret_cast<float*>(ws + L.off_hk);
   const bool trip = mode == VSA_SCORE_TRIPPOOL;
 
+  // projection: [ntv, kd] x [kd, p]; the gate is shared by all heads, TripPool weights are per head
+  const int Z = g.B * g.Hh;
+  const int64_t sW = trip ? int64_t(L.kd) * p : 0;
+  dim3 gp((p + 127) / 128, (g.ntv_max + 127) / 128, Z);
+  sgemm_kernel<false><<<gp, 256, 0, s>>>(g, pq, int64_t(g.ntv_max) * L.kd, L.kd, proj_q, 0, sW, p, hq,
+                                         int64_t(g.ntv_max) * p, p, L.kd, p, 1.0f);
+  sgemm_kernel<false><<<gp, 256, 0, s>>>(g, pk, int64_t(g.ntv_max) * L.kd, L.kd, proj_k, 0, sW, p, hk,
+                                         int64_t(g.ntv_max) * p, p, L.kd, p, 1.0f);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  // scores: q_hat k_hat^T / sqrt(p)
+  dim3 gs((g.ntv_max + 127) / 128, (g.ntv_max + 127) / 128, Z);
+  sgemm_kernel<true><<<gs, 256, 0, s>>>(g, hq, int64_t(g.ntv_max) * p, p, hk, int64_t(g.ntv_max) * p, 0, p, scores,
+                                        int64_t(g.ntv_max) * g.ntv_max, g.ntv_max, p, 0, 1.0f / sqrtf(float(p)));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_score(const vsa_plan* pl, const void* qp, const void* kp, const float* proj_q,
+                         const float* proj_k, float* scores, void* workspace, cudaStream_t s) {
+  const Geometry& g = pl->geo;
+  const bool trip = pl->desc.score_mode == VSA_SCORE_TRIPPOOL;
+  float *pq, *pk;
+  score_pooled_ptrs(pl, workspace, &pq, &pk);
   const int64_t tasks = int64_t(g.B) * g.Hh * g.ntv_max * 2;
   const int blocks = int((tasks + 7) / 8);
   auto* q16 = static_cast<const uint16_t*>(qp);
@@ -215,23 +247,7 @@ cudaError_t launch_score(const vsa_plan* pl, const void* qp, const void* kp, con
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-
-  // projection: [ntv, kd] x [kd, p]; the gate is shared by all heads, TripPool weights are per head
-  const int Z = g.B * g.Hh;
-  const int64_t sW = trip ? int64_t(L.kd) * p : 0;
-  dim3 gp((p + 127) / 128, (g.ntv_max + 127) / 128, Z);
-  sgemm_kernel<false><<<gp, 256, 0, s>>>(g, pq, int64_t(g.ntv_max) * L.kd, L.kd, proj_q, 0, sW, p, hq,
-                                         int64_t(g.ntv_max) * p, p, L.kd, p, 1.0f);
-  sgemm_kernel<false><<<gp, 256, 0, s>>>(g, pk, int64_t(g.ntv_max) * L.kd, L.kd, proj_k, 0, sW, p, hk,
-                                         int64_t(g.ntv_max) * p, p, L.kd, p, 1.0f);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-
-  // scores: q_hat k_hat^T / sqrt(p)
-  dim3 gs((g.ntv_max + 127) / 128, (g.ntv_max + 127) / 128, Z);
-  sgemm_kernel<true><<<gs, 256, 0, s>>>(g, hq, int64_t(g.ntv_max) * p, p, hk, int64_t(g.ntv_max) * p, 0, p, scores,
-                                        int64_t(g.ntv_max) * g.ntv_max, g.ntv_max, p, 0, 1.0f / sqrtf(float(p)));
-  return cudaGetLastError();
+  return launch_project_score(pl, proj_q, proj_k, scores, workspace, s);
 }
 
 }  // namespace vsa

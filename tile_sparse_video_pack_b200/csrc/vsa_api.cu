@@ -287,6 +287,31 @@ vsa_status vsa_tile_pack(vsa_plan* p, const void* q, const void* k, const void* 
   return VSA_OK;
 }
 
+vsa_status vsa_tile_pack_pool(vsa_plan* p, const void* q, const void* k, const void* v, void* qp, void* kp,
+                              void* vp, void* ws, void* stream) {
+  if (!p || !q || !k || !v || !qp || !kp || !vp || !ws) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qp) || !aligned16(kp) || !aligned16(vp) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_pack++;
+  float *pq, *pk;
+  vsa::score_pooled_ptrs(p, ws, &pq, &pk);
+  if (vsa::launch_pack_pool(p, q, k, v, qp, kp, vp, pq, pk, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_tile_score_pooled(vsa_plan* p, const float* proj_q, const float* proj_k, float* scores, void* ws,
+                                 void* stream) {
+  if (!p || !proj_q || !proj_k || !scores || !ws) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!aligned16(proj_q) || !aligned16(proj_k) || !aligned16(scores) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_score++;
+  if (vsa::launch_project_score(p, proj_q, proj_k, scores, ws, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
 vsa_status vsa_tile_unpack(vsa_plan* p, const void* op, void* o, void* stream) {
   if (!p || !op || !o || !aligned16(op) || !aligned16(o)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_unpack++;
@@ -332,8 +357,8 @@ vsa_status vsa_layer_forward(vsa_plan* p, const void* q, const void* k, const vo
                              const float* proj_q, const float* proj_k, void* qp, void* kp, void* vp,
                              float* scores, int32_t* idx, void* op, float* lse, void* ws, void* o,
                              void* stream) {
-  vsa_status s = vsa_tile_pack(p, q, k, v, qp, kp, vp, stream);
-  if (s == VSA_OK) s = vsa_tile_score(p, qp, kp, proj_q, proj_k, scores, ws, stream);
+  vsa_status s = vsa_tile_pack_pool(p, q, k, v, qp, kp, vp, ws, stream);
+  if (s == VSA_OK) s = vsa_tile_score_pooled(p, proj_q, proj_k, scores, ws, stream);
   if (s == VSA_OK) s = vsa_topk_select(p, scores, idx, stream);
   if (s == VSA_OK) s = vsa_sparse_attn(p, qp, kp, vp, idx, op, lse, stream);
   if (s == VSA_OK) s = vsa_tile_unpack(p, op, o, stream);

@@ -62,10 +62,16 @@ namespace vsa {
 // Launchers (return cudaGetLastError()).
 cudaError_t launch_pack(const vsa_plan* p, const void* q, const void* k, const void* v, void* qp,
                         void* kp, void* vp, cudaStream_t s);
+cudaError_t launch_pack_pool(const vsa_plan* p, const void* q, const void* k, const void* v, void* qp,
+                             void* kp, void* vp, float* pooled_q, float* pooled_k, cudaStream_t s);
 cudaError_t launch_unpack(const vsa_plan* p, const void* op, void* o, cudaStream_t s);
 cudaError_t launch_score(const vsa_plan* p, const void* qp, const void* kp, const float* proj_q,
                          const float* proj_k, float* scores, void* workspace, cudaStream_t s);
 int64_t score_workspace_bytes(const Geometry& g, int score_mode, int proj_dim);
+// Where the score stage keeps the pooled Q and K descriptors in a workspace.
+void score_pooled_ptrs(const vsa_plan* p, void* workspace, float** pooled_q, float** pooled_k);
+cudaError_t launch_project_score(const vsa_plan* p, const float* proj_q, const float* proj_k, float* scores,
+                                 void* workspace, cudaStream_t s);
 cudaError_t launch_topk(const vsa_plan* p, const float* scores, int32_t* idx, cudaStream_t s);
 cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp,
                         const int32_t* idx, void* op, float* lse, cudaStream_t s);

@@ -35,8 +35,8 @@ class TileSparseAttention:
     def stages(self, q, k, v, out, stream=None):
         """The five calls one by one (same result as :meth:`forward`)."""
         b, p = self.bufs, self.plan
-        p.tile_pack(q, k, v, b["qp"], b["kp"], b["vp"], stream)
-        p.tile_score(b["qp"], b["kp"], self.proj_q, self.proj_k, b["scores"], b["workspace"], stream)
+        p.tile_pack_pool(q, k, v, b["qp"], b["kp"], b["vp"], b["workspace"], stream)
+        p.tile_score_pooled(self.proj_q, self.proj_k, b["scores"], b["workspace"], stream)
         p.topk_select(b["scores"], b["idx"], stream)
         p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], b["lse"], stream)
         p.tile_unpack(b["op"], out, stream)

@@ -25,7 +25,8 @@ SCORE_MODES = {"meanpool_gate": 0, "tripool": 1}
 # every entry point declared in include/vsa.h
 EXPORTS = ("vsa_plan_create", "vsa_plan_destroy", "vsa_plan_query", "vsa_plan_get_stats", "vsa_k_from_sparsity",
            "vsa_tile_pack", "vsa_tile_score", "vsa_topk_select", "vsa_sparse_attn", "vsa_tile_unpack",
-           "vsa_layer_forward", "vsa_plan_check", "vsa_status_string", "vsa_tile_score_static")
+           "vsa_layer_forward", "vsa_plan_check", "vsa_status_string", "vsa_tile_score_static",
+           "vsa_tile_pack_pool", "vsa_tile_score_pooled")
 
 
 class VsaDesc(ctypes.Structure):
@@ -89,6 +90,8 @@ def library() -> ctypes.CDLL:
         "vsa_plan_check": (I32, [P]),
         "vsa_status_string": (ctypes.c_char_p, [I32]),
         "vsa_tile_score_static": (I32, [P, P, P, P, P, P, P]),
+        "vsa_tile_pack_pool": (I32, [P] * 9),
+        "vsa_tile_score_pooled": (I32, [P] * 6),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -237,6 +240,26 @@ class Plan:
             _ptr(scores, torch.float32, "scores", self.info.score_elems),
             _ptr(workspace, torch.uint8, "workspace", self.info.workspace_bytes), _stream(stream)),
             "vsa_tile_score")
+
+    def tile_pack_pool(self, q, k, v, qp, kp, vp, workspace, stream=None):
+        """tile_pack fused with the pooling of tile_score; follow with tile_score_pooled."""
+        import torch
+        n_tok = self.desc.batch * self.info.n_tokens * self.desc.heads * self.desc.head_dim
+        pe, bf = self.info.packed_elems, torch.bfloat16
+        _check(library().vsa_tile_pack_pool(
+            self._h, _ptr(q, bf, "q", n_tok), _ptr(k, bf, "k", n_tok), _ptr(v, bf, "v", n_tok),
+            _ptr(qp, bf, "qp", pe), _ptr(kp, bf, "kp", pe), _ptr(vp, bf, "vp", pe),
+            _ptr(workspace, torch.uint8, "workspace", self.info.workspace_bytes), _stream(stream)),
+            "vsa_tile_pack_pool")
+
+    def tile_score_pooled(self, proj_q, proj_k, scores, workspace, stream=None):
+        """Projection and scores from the descriptors tile_pack_pool left in the workspace."""
+        import torch
+        _check(library().vsa_tile_score_pooled(
+            self._h, _ptr(proj_q, torch.float32, "proj_q"), _ptr(proj_k, torch.float32, "proj_k"),
+            _ptr(scores, torch.float32, "scores", self.info.score_elems),
+            _ptr(workspace, torch.uint8, "workspace", self.info.workspace_bytes), _stream(stream)),
+            "vsa_tile_score_pooled")
 
     def tile_score_static(self, qp, kp, proj_q, proj_k, scores, stream=None):
         """tile_score with the library's fixed 32 MiB device scratch instead of a workspace.

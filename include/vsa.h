@@ -229,6 +229,32 @@ VSA_API vsa_status vsa_sparse_attn(vsa_plan* plan, const void* qp, const void* k
 /* a7. Inverse of the pack permutation: [B, heads, nt_max, 64, d] -> [B, N, heads, d]. */
 VSA_API vsa_status vsa_tile_unpack(vsa_plan* plan, const void* op, void* o, void* stream);
 
+/* Teacher tile map (row f3; the first stage of the Veda method: full attention,
+ * max-pooled per tile pair, is the teacher distribution at tile level -- Veda
+ * news page, "Что делает Veda"). For video query tile i and video key tile j
+ * of every (batch, head):
+ *   teacher[b][h][i][j] = max over valid rows r of tile i and valid keys c of
+ *                         tile j of exp(scale * q_r . k_c - lse[r]),
+ * the largest full-attention weight a token of tile i puts on a token of tile
+ * j. lse ([B, heads, nt_max, 64] fp32, natural log) must be the row
+ * log-sum-exp over EVERY key: the lse output of vsa_sparse_attn on a plan
+ * with k = every video tile. qp, kp: packed bf16 as from vsa_tile_pack.
+ * teacher: fp32 [B, heads, ntv_max, ntv_max] (the layout of the scores of
+ * vsa_tile_score, so vsa_topk_select ranks it); entries past a head's own
+ * ntv are left untouched. Cost: a dense Q K^T over all video tile pairs. */
+VSA_API vsa_status vsa_teacher_tiles(vsa_plan* plan, const void* qp, const void* kp, const float* lse,
+                             float* teacher, void* stream);
+
+/* For every (batch, head, video query tile) row of two index tables
+ * ([B, heads, ntv_max, k_max] int32, ascending rows of the head's k, as
+ * vsa_topk_select writes them): the number of indices the rows share, in
+ * counts [B, heads, ntv_max] (0 for rows past a head's ntv). With a = the
+ * scorer's selection and b = the teacher's top-k, counts / k is the tile
+ * recall of the scorer (BSAI VedaSparse README, "Core Technology": TripPool
+ * tile recall against full attention). */
+VSA_API vsa_status vsa_index_overlap(vsa_plan* plan, const int32_t* idx_a, const int32_t* idx_b,
+                             int32_t* counts, void* stream);
+
 /* The whole layer in order on one stream, on caller-provided buffers (sizes
  * from vsa_plan_query): vsa_tile_pack_pool, vsa_tile_score_pooled,
  * vsa_topk_select, vsa_sparse_attn, vsa_tile_unpack. Returns the first

@@ -373,3 +373,34 @@ def attention_flops(cfg, k_per_head) -> int:
         kh = int(k_per_head[h])
         total_pairs += sum(sizes) * (n_pre_tok + kh * TILE)
     return 4 * cfg.head_dim * total_pairs * cfg.batch
+
+
+# ---------------------------------------------------------------------------
+# teacher tile map and tile recall (the Veda method's first stage)
+# ---------------------------------------------------------------------------
+
+
+def teacher_tiles(q_h: np.ndarray, k_h: np.ndarray, til: HeadTiling, scale: float) -> np.ndarray:
+    """Teacher map of one head, fp64: T[i, j] is the largest weight that any token of video
+    tile i gives any token of video tile j in FULL softmax attention, i.e. over every token of
+    the sequence, prefix included (Veda news page, "Что делает Veda": full attention,
+    max-pooled per tile pair, is the tile-level teacher distribution that the scorer learns).
+    """
+    keys = np.concatenate(til.all)
+    start = np.cumsum([0] + [len(t) for t in til.all])       # tile t occupies keys[start[t]:start[t+1]]
+    n_pre, n_vid = til.n_prefix, til.n_video
+    T = np.zeros((n_vid, n_vid))
+    for i, rows in enumerate(til.video):
+        x = scale * (q_h[rows] @ k_h[keys].T)
+        a = np.exp(x - x.max(axis=1, keepdims=True))
+        a /= a.sum(axis=1, keepdims=True)                     # each row: weights over every key
+        for j in range(n_vid):
+            T[i, j] = a[:, start[n_pre + j]:start[n_pre + j + 1]].max()
+    return T
+
+
+def tile_recall(kept_row: np.ndarray, teacher_row: np.ndarray, k: int) -> float:
+    """Share of the teacher's k best key tiles (ranked by :func:`topk_row`) that a selection
+    keeps: the tile recall by which the BSAI VedaSparse README ("Core Technology") compares
+    TripPool with mean pooling."""
+    return len(np.intersect1d(kept_row, topk_row(teacher_row, k))) / k

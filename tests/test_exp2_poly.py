@@ -17,7 +17,8 @@ ATTN = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
 
 def kernel_coefficients():
     src = open(ATTN).read()
-    body = src[src.index("void ex2_fma_pipe"):src.index("__device__ __forceinline__ uint32_t bf16x2")]
+    start = src.index("void ex2_fma_pipe")
+    body = src[start:src.index("\n}\n", start)]
     vals = [float(v) for v in re.findall(r"f2pack\(([0-9.e-]+)f, \1f\)", body)]
     return np.array(vals[::-1], dtype=np.float32)   # written highest degree first
 

@@ -346,3 +346,99 @@ def test_mutation_video_rows_lose_prefix(monkeypatch):
 def test_mutation_pool_over_64(monkeypatch):
     monkeypatch.setattr(O, "mean_pool", lambda x: x.sum(axis=0) / 64.0)
     _expect_pin_failure(pin_constant_tiles_pool, ragged_config(batch=1))
+
+
+# ------------------------------------------------ teacher map and recall ---
+
+def _teacher_case(h=1):
+    cfg = ragged_config(batch=1)
+    inp, q, k, v = inputs_f64(cfg)
+    return cfg, O.head_tiling(cfg, h), q[0, :, h], k[0, :, h]
+
+
+def pin_teacher_uniform_when_q_zero():
+    """Q = 0: every row attends uniformly to all N tokens, prefix included, so every
+    entry of the teacher map is exactly 1 / N."""
+    cfg, til, q, k = _teacher_case()
+    T = O.teacher_tiles(np.zeros_like(q), k, til, 1 / math.sqrt(cfg.head_dim))
+    assert T.shape == (til.n_video, til.n_video)
+    assert np.max(np.abs(T - 1.0 / cfg.n_tokens)) <= 1e-15
+
+
+def test_teacher_uniform_when_q_zero():
+    pin_teacher_uniform_when_q_zero()
+
+
+def pin_teacher_dominant_token():
+    """One query token r0 of video tile i0 aligned with one key token c0 of tile j0 (far
+    larger logit than anything else): T[i0, j0] ~ 1 and j0 is the teacher's top tile of
+    row i0, while a row-mean pooling would give about 1/64. Rows of other tiles are
+    unaffected."""
+    cfg, til, q, k = _teacher_case()
+    i0, j0 = 2, 5
+    r0, c0 = til.video[i0][7], til.video[j0][11]
+    q, k = q.copy() * 0.1, k.copy() * 0.1
+    q[r0] = 0.0
+    q[r0, 3] = 40.0
+    k[c0] = 0.0
+    k[c0, 3] = 40.0
+    scale = 1 / math.sqrt(cfg.head_dim)
+    T = O.teacher_tiles(q, k, til, scale)
+    assert T[i0, j0] > 0.999
+    assert list(O.topk_row(T[i0], 1)) == [j0]
+    # the same rows without the planted pair stay far below
+    assert np.max(np.delete(T[i0], j0)) < 0.05
+
+
+def test_teacher_dominant_token():
+    pin_teacher_dominant_token()
+
+
+def test_teacher_is_a_max_of_probabilities():
+    cfg, til, q, k = _teacher_case(h=3)
+    T = O.teacher_tiles(q, k, til, 1 / math.sqrt(cfg.head_dim))
+    assert np.all(T > 0) and np.all(T <= 1)   # softmax weights
+
+
+def test_recall_identities():
+    rng = np.random.default_rng(5)
+    T = rng.random((6, 12))
+    for i in range(6):
+        best = O.topk_row(T[i], 4)
+        assert O.tile_recall(best, T[i], 4) == 1.0
+        rest = np.setdiff1d(np.arange(12), best)[:4]
+        assert O.tile_recall(rest, T[i], 4) == 0.0
+        assert O.tile_recall(np.arange(12), T[i], 12) == 1.0
+        assert O.tile_recall(np.sort(np.r_[best[:2], rest[:2]]), T[i], 4) == 0.5
+
+
+def test_mutation_teacher_mean_over_rows(monkeypatch):
+    def bad(q_h, k_h, til, scale):         # pools rows by their mean instead of the max
+        keys = np.concatenate(til.all)
+        start = np.cumsum([0] + [len(t) for t in til.all])
+        T = np.zeros((til.n_video, til.n_video))
+        for i, rows in enumerate(til.video):
+            x = scale * (q_h[rows] @ k_h[keys].T)
+            a = np.exp(x - x.max(axis=1, keepdims=True))
+            a /= a.sum(axis=1, keepdims=True)
+            for j in range(til.n_video):
+                T[i, j] = a[:, start[til.n_prefix + j]:start[til.n_prefix + j + 1]].max(axis=1).mean()
+        return T
+    monkeypatch.setattr(O, "teacher_tiles", bad)
+    _expect_pin_failure(pin_teacher_dominant_token)
+
+
+def test_mutation_teacher_softmax_over_video_keys_only(monkeypatch):
+    def bad(q_h, k_h, til, scale):         # normalises each row over video keys only
+        keys = np.concatenate(til.video)
+        start = np.cumsum([0] + [len(t) for t in til.video])
+        T = np.zeros((til.n_video, til.n_video))
+        for i, rows in enumerate(til.video):
+            x = scale * (q_h[rows] @ k_h[keys].T)
+            a = np.exp(x - x.max(axis=1, keepdims=True))
+            a /= a.sum(axis=1, keepdims=True)
+            for j in range(til.n_video):
+                T[i, j] = a[:, start[j]:start[j + 1]].max()
+        return T
+    monkeypatch.setattr(O, "teacher_tiles", bad)
+    _expect_pin_failure(pin_teacher_uniform_when_q_zero)

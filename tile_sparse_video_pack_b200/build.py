@@ -13,8 +13,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libvsa.so")
-SOURCES = ["vsa_api.cu", "pack.cu", "score.cu", "topk.cu", "attn.cu"]
-HEADERS = ["vsa_internal.h"]
+SOURCES = ["vsa_api.cu", "pack.cu", "score.cu", "topk.cu", "attn.cu", "teacher.cu"]
+HEADERS = ["vsa_internal.h", "tc_sm100.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

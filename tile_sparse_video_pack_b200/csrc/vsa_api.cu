@@ -365,6 +365,25 @@ vsa_status vsa_layer_forward(vsa_plan* p, const void* q, const void* k, const vo
   return s;
 }
 
+vsa_status vsa_teacher_tiles(vsa_plan* p, const void* qp, const void* kp, const float* lse, float* teacher,
+                             void* stream) {
+  if (!p || !qp || !kp || !lse || !teacher || !aligned16(qp) || !aligned16(kp) || !aligned16(lse) ||
+      !aligned16(teacher))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  if (vsa::launch_teacher(p, qp, kp, lse, teacher, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_index_overlap(vsa_plan* p, const int32_t* idx_a, const int32_t* idx_b, int32_t* counts,
+                             void* stream) {
+  if (!p || !idx_a || !idx_b || !counts || !aligned16(idx_a) || !aligned16(idx_b) || !aligned16(counts))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  if (vsa::launch_overlap(p, idx_a, idx_b, counts, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
 vsa_status vsa_plan_check(vsa_plan* p) {
   if (!p) return VSA_ERR_INVALID_ARG;
   cudaError_t e = cudaDeviceSynchronize();

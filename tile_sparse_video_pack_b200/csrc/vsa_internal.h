@@ -76,5 +76,8 @@ cudaError_t launch_topk(const vsa_plan* p, const float* scores, int32_t* idx, cu
 cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp,
                         const int32_t* idx, void* op, float* lse, cudaStream_t s);
 int attn_smem_bytes(int list_cap);
+cudaError_t launch_teacher(vsa_plan* p, const void* qp, const void* kp, const float* lse, float* teacher,
+                           cudaStream_t s);
+cudaError_t launch_overlap(vsa_plan* p, const int32_t* a, const int32_t* b, int32_t* counts, cudaStream_t s);
 
 }  // namespace vsa

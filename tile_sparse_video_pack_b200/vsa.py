@@ -26,7 +26,7 @@ SCORE_MODES = {"meanpool_gate": 0, "tripool": 1}
 EXPORTS = ("vsa_plan_create", "vsa_plan_destroy", "vsa_plan_query", "vsa_plan_get_stats", "vsa_k_from_sparsity",
            "vsa_tile_pack", "vsa_tile_score", "vsa_topk_select", "vsa_sparse_attn", "vsa_tile_unpack",
            "vsa_layer_forward", "vsa_plan_check", "vsa_status_string", "vsa_tile_score_static",
-           "vsa_tile_pack_pool", "vsa_tile_score_pooled")
+           "vsa_tile_pack_pool", "vsa_tile_score_pooled", "vsa_teacher_tiles", "vsa_index_overlap")
 
 
 class VsaDesc(ctypes.Structure):
@@ -92,6 +92,8 @@ def library() -> ctypes.CDLL:
         "vsa_tile_score_static": (I32, [P, P, P, P, P, P, P]),
         "vsa_tile_pack_pool": (I32, [P] * 9),
         "vsa_tile_score_pooled": (I32, [P] * 6),
+        "vsa_teacher_tiles": (I32, [P] * 6),
+        "vsa_index_overlap": (I32, [P] * 5),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -260,6 +262,24 @@ class Plan:
             _ptr(scores, torch.float32, "scores", self.info.score_elems),
             _ptr(workspace, torch.uint8, "workspace", self.info.workspace_bytes), _stream(stream)),
             "vsa_tile_score_pooled")
+
+    def teacher_tiles(self, qp, kp, lse, teacher, stream=None):
+        """Max-pooled full-attention weights per video tile pair; lse from a dense sparse_attn."""
+        import torch
+        pe = self.info.packed_elems
+        _check(library().vsa_teacher_tiles(
+            self._h, _ptr(qp, torch.bfloat16, "qp", pe), _ptr(kp, torch.bfloat16, "kp", pe),
+            _ptr(lse, torch.float32, "lse", self.info.lse_elems),
+            _ptr(teacher, torch.float32, "teacher", self.info.score_elems), _stream(stream)), "vsa_teacher_tiles")
+
+    def index_overlap(self, idx_a, idx_b, counts, stream=None):
+        """Shared indices per row of two ascending top-k tables."""
+        import torch
+        n = self.desc.batch * self.desc.heads * self.info.ntv_max
+        _check(library().vsa_index_overlap(
+            self._h, _ptr(idx_a, torch.int32, "idx_a", self.info.index_elems),
+            _ptr(idx_b, torch.int32, "idx_b", self.info.index_elems),
+            _ptr(counts, torch.int32, "counts", n), _stream(stream)), "vsa_index_overlap")
 
     def tile_score_static(self, qp, kp, proj_q, proj_k, scores, stream=None):
         """tile_score with the library's fixed 32 MiB device scratch instead of a workspace.

@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
+    ap.add_argument("--teacher", action="store_true",
+                    help="also time the teacher tile map and report the selection's tile recall")
     return ap.parse_args()
 
 
@@ -368,6 +370,48 @@ def run_ours(args, rank, world, local_rank):
         stats = layer.plan.stats()
         return layer, out, ms_step, stages, clocks, stats
 
+    def teacher_measure(layer, ks):
+        """The teacher tile map of this workload and the tile recall of the layer's selection.
+
+        A dense plan (k = every video tile) runs the layer once for the rows' full
+        log-sum-exp; the teacher kernel is then timed on its own; its top-k (same k as
+        the layer) is overlapped with the layer's selection.
+        """
+        ntv = [layer.plan.info.ntv[h] for h in range(cfg.heads)]
+        dense = T.TileSparseAttention.from_config(cfg, 0.0, pq, pk, k_per_head=ntv)
+        db = dense.bufs
+        dp = dense.plan
+        dp.tile_pack_pool(q, k, v, db["qp"], db["kp"], db["vp"], db["workspace"])
+        dp.tile_score_pooled(pq, pk, db["scores"], db["workspace"])
+        dp.topk_select(db["scores"], db["idx"])
+        lse = torch.empty(dp.info.lse_elems, dtype=torch.float32, device=dev)
+        dp.sparse_attn(db["qp"], db["kp"], db["vp"], db["idx"], db["op"], lse)
+        teacher = torch.zeros_like(db["scores"])
+        iters = 3
+        dp.teacher_tiles(db["qp"], db["kp"], lse, teacher)            # warm-up
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            dp.teacher_tiles(db["qp"], db["kp"], lse, teacher)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / iters
+        lp = layer.plan
+        t_idx = torch.empty_like(layer.bufs["idx"])
+        lp.topk_select(teacher, t_idx)
+        counts = torch.empty(cfg.batch * cfg.heads * lp.info.ntv_max, dtype=torch.int32, device=dev)
+        lp.index_overlap(layer.bufs["idx"], t_idx, counts)
+        dp.check()
+        lp.check()
+        c = counts.view(cfg.batch, cfg.heads, lp.info.ntv_max).cpu().numpy()
+        recall = float(np.mean([c[b, h, :ntv[h]].mean() / ks[h] for b in range(cfg.batch) for h in range(cfg.heads)]))
+        flops = 2 * cfg.head_dim * cfg.batch * cfg.heads * cfg.n_video_tokens ** 2
+        tf = flops / (ms * 1e-3) / 1e12
+        return {"kernel": "teacher_kernel (vsa_teacher_tiles)", "ms": round(ms, 3), "tflops": round(tf, 1),
+                "bound": "tensor", "peak": peaks["bf16_tflops"], "frac": round(tf / peaks["bf16_tflops"], 4),
+                "peak_kind": f"bf16 dense, burst, {peaks['source']}", "algorithmic_flops": flops,
+                "recall": round(recall, 4), "recall_of": f"{cfg.score_mode} selection, k={ks[0]}, vs the teacher's top-k"}
+
     ks = k_list(cfg, args.sparsity)
     layer, out, ms_step, stages, clocks, stats = timed_layer(args.sparsity, args.steps, args.warmup, True)
     flops = attention_flops(cfg, ks)
@@ -394,6 +438,8 @@ def run_ours(args, rank, world, local_rank):
                      "attn_tflops": round(f2 / (st2["attn"] * 1e-3) / 1e12, 1),
                      "layer_tflops": round(f2 / (ms2 * 1e-3) / 1e12, 1)}
 
+    teacher = teacher_measure(layer, ks) if args.teacher else None
+
     value = job_ms_per_layer(ms_step, 1, world)
     line = {
         "metric": "ms per attention layer at 107k video tokens, 75% video sparsity (90% in secondary); effective TFLOP/s",
@@ -417,6 +463,8 @@ def run_ours(args, rank, world, local_rank):
         "attention_computed_pct": round(100.0 * stats["computed_pairs"] / stats["dense_pairs"], 2),
         "secondary": secondary,
     }
+    if teacher is not None:
+        line["teacher"] = teacher
     return line
 
 

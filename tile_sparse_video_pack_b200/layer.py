@@ -19,8 +19,8 @@ class TileSparseAttention:
         self.bufs = plan.allocate(device, with_lse=with_lse)
 
     @classmethod
-    def from_config(cls, cfg, sparsity, proj_q, proj_k, **kw):
-        return cls(Plan.from_config(cfg, sparsity), proj_q, proj_k, **kw)
+    def from_config(cls, cfg, sparsity, proj_q, proj_k, k_per_head=None, **kw):
+        return cls(Plan.from_config(cfg, sparsity, k_per_head=k_per_head), proj_q, proj_k, **kw)
 
     def forward(self, q, k, v, out=None, stream=None):
         """Token-major ``[B, N, heads, d]`` bf16 CUDA tensors -> output of the same shape."""

@@ -180,26 +180,45 @@ def tripool(x: np.ndarray) -> np.ndarray:
 
 
 def tile_scores(q_h: np.ndarray, k_h: np.ndarray, til: HeadTiling, cfg, h: int,
-                gate=None, w_q=None, w_k=None) -> np.ndarray:
+                gate=None, w_q=None, w_k=None, key_tiles=None) -> np.ndarray:
     """Scores S[i, j] for video query tile i and video key tile j of head h (fp64).
 
     ``q_h``/``k_h`` are the head's token rows ``[N, d]``. Prefix tiles are not
-    scored: they are never pruned.
+    scored: they are never pruned. ``key_tiles`` (a list of token-index arrays)
+    replaces the video key tiles on the key side: the reference tiles of the
+    R2VA budget variant are scored this way, against the same video query tiles.
     """
+    key_tiles = til.video if key_tiles is None else key_tiles
     if cfg.score_mode == "meanpool_gate":
         g = np.asarray(gate, dtype=np.float64)
         qd = np.stack([mean_pool(q_h[t]) for t in til.video]) @ g
-        kd = np.stack([mean_pool(k_h[t]) for t in til.video]) @ g
+        kd = np.stack([mean_pool(k_h[t]) for t in key_tiles]) @ g
         width = g.shape[1]
     elif cfg.score_mode == "tripool":
         wq = np.asarray(w_q[h], dtype=np.float64)
         wk = np.asarray(w_k[h], dtype=np.float64)
         qd = np.stack([tripool(q_h[t]) for t in til.video]) @ wq
-        kd = np.stack([tripool(k_h[t]) for t in til.video]) @ wk
+        kd = np.stack([tripool(k_h[t]) for t in key_tiles]) @ wk
         width = wq.shape[1]
     else:
         raise ValueError(cfg.score_mode)
     return (qd @ kd.T) / math.sqrt(width)
+
+
+def ref_tiles(cfg) -> np.ndarray:
+    """Indices (into the prefix tile list) of the tiles of reference segments: the
+    prefix streams that the R2VA budget variant prunes with their own top-k (BSAI
+    VedaSparse README, v3.4.2 notes on the R2VA predictor: 32 reference tiles and 32
+    video tiles per query, text / VLM / audio conditioning always dense). Empty when
+    no segment is marked."""
+    flags = tuple(cfg.seg_ref) or (0,) * len(cfg.segments)
+    out, t = [], 0
+    for length, f in zip(cfg.segments, flags):
+        n = -(-length // TILE)
+        if f:
+            out.extend(range(t, t + n))
+        t += n
+    return np.asarray(out, dtype=np.int64)
 
 
 # ---------------------------------------------------------------------------
@@ -239,16 +258,22 @@ def softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float)
     return p @ v, (m + np.log(s))[:, 0], p.sum(axis=1)
 
 
-def query_key_tokens(til: HeadTiling, tile_id: int, kept_video) -> np.ndarray:
+def query_key_tokens(til: HeadTiling, tile_id: int, kept_video, ref=None, kept_ref=None) -> np.ndarray:
     """Key tokens that query tile ``tile_id`` (index into ``til.all``) attends to.
 
     Prefix query tiles see every token (BSAI README "cond rows always dense";
     Ref2VA README item 1). Video query tiles see every prefix tile plus their
-    kept video tiles (Ref2VA README items 1-2).
+    kept video tiles (Ref2VA README items 1-2). With reference tiles ``ref``
+    (prefix tile indices) a video query tile sees, of those, only ``kept_ref``
+    (positions into ``ref``); the other prefix tiles stay dense.
     """
     if tile_id < til.n_prefix:
         return np.concatenate(til.all)
-    return np.concatenate(til.prefix + [til.video[j] for j in kept_video])
+    prefix = til.prefix
+    if ref is not None and len(ref):
+        drop = set(int(ref[r]) for r in range(len(ref))) - set(int(ref[r]) for r in kept_ref)
+        prefix = [t for i, t in enumerate(til.prefix) if i not in drop]
+    return np.concatenate(prefix + [til.video[j] for j in kept_video])
 
 
 @dataclasses.dataclass
@@ -259,11 +284,13 @@ class LayerResult:
     lse: np.ndarray              # [B, N, heads] fp64
     row_sum: np.ndarray          # [B, N, heads] fp64
     computed_pairs: int          # sum over computed query rows of their key count
+    ref_scores: list = None      # per head [NTv_h, n_ref] fp64 (reference tiles of the R2VA variant)
+    ref_kept: list = None        # per head [NTv_h, k_ref] positions into ref_tiles(cfg), ascending
 
 
 def run_layer(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, k_per_head,
               gate=None, w_q=None, w_k=None, query_tiles=None,
-              heads=None, kept=None) -> LayerResult:
+              heads=None, kept=None, kept_ref=None) -> LayerResult:
     """The whole layer, in fp64: tile, score, select, attend.
 
     ``q``, ``k``, ``v``: ``[B, N, heads, d]`` (any float dtype; widened to fp64).
@@ -272,7 +299,9 @@ def run_layer(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, k_per_head,
     attention rows; the others stay NaN. ``heads`` restricts the heads computed.
     ``kept``: optional {head: [NTv_h, k_h] array} (or {(b, head): ...}) of kept
     video tiles to attend with instead of the oracle's own top-k (the scores
-    are still computed and returned).
+    are still computed and returned). With reference segments (``cfg.seg_ref``),
+    each video query tile also keeps its ``cfg.k_ref`` best reference tiles by the
+    same scorer; ``kept_ref`` overrides that choice like ``kept``.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -284,6 +313,8 @@ def run_layer(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, k_per_head,
     lse = np.full((B, N, Hh), np.nan)
     row_sum = np.full((B, N, Hh), np.nan)
     all_scores, all_kept = [None] * Hh, [None] * Hh
+    all_rs, all_rk = [None] * Hh, [None] * Hh
+    ref = ref_tiles(cfg)
     pairs = 0
     for h in heads:
         til = head_tiling(cfg, h)
@@ -295,15 +326,28 @@ def run_layer(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, k_per_head,
                 kept_bh = np.asarray(kept[(b, h)] if (b, h) in kept else kept[h])
             else:
                 kept_bh = np.stack([topk_row(s[i], kh) for i in range(til.n_video)])
+            rs = rk = None
+            if len(ref):
+                rs = tile_scores(q[b, :, h], k[b, :, h], til, cfg, h, gate, w_q, w_k,
+                                 key_tiles=[til.prefix[r] for r in ref])
+                if kept_ref is not None:
+                    rk = np.asarray(kept_ref[(b, h)] if (b, h) in kept_ref else kept_ref[h])
+                else:
+                    rk = np.stack([topk_row(rs[i], int(cfg.k_ref)) for i in range(til.n_video)])
             if b == 0:
                 all_scores[h], all_kept[h] = s, kept_bh
+                all_rs[h], all_rk[h] = rs, rk
             for t in tiles_h:
                 qt = til.all[t]
-                kv = query_key_tokens(til, t, None if t < til.n_prefix else kept_bh[t - til.n_prefix])
+                if t < til.n_prefix:
+                    kv = query_key_tokens(til, t, None)
+                else:
+                    kv = query_key_tokens(til, t, kept_bh[t - til.n_prefix], ref,
+                                          None if rk is None else rk[t - til.n_prefix])
                 o, l, rs = softmax_attention(q[b, qt, h], k[b, kv, h], v[b, kv, h], scale)
                 out[b, qt, h], lse[b, qt, h], row_sum[b, qt, h] = o, l, rs
                 pairs += len(qt) * len(kv)
-    return LayerResult(all_scores, all_kept, out, lse, row_sum, pairs)
+    return LayerResult(all_scores, all_kept, out, lse, row_sum, pairs, all_rs, all_rk)
 
 
 # ---------------------------------------------------------------------------

@@ -335,7 +335,7 @@ def test_mutation_wrong_scale(monkeypatch):
 
 
 def test_mutation_video_rows_lose_prefix(monkeypatch):
-    def bad(til, tile_id, kept):
+    def bad(til, tile_id, kept, ref=None, kept_ref=None):
         if tile_id < til.n_prefix:
             return np.concatenate(til.all)
         return np.concatenate([til.video[j] for j in kept])
@@ -442,3 +442,78 @@ def test_mutation_teacher_softmax_over_video_keys_only(monkeypatch):
         return T
     monkeypatch.setattr(O, "teacher_tiles", bad)
     _expect_pin_failure(pin_teacher_uniform_when_q_zero)
+
+
+# ------------------------------------- R2VA budgets: reference tiles pruned ---
+
+def ragged_r2va_config(score_mode="meanpool_gate"):
+    """Text, a reference segment of 130 tokens (tiles of 64, 64 and 2 tokens), audio."""
+    cfg = ragged_config(batch=1).with_(name="ragged_r2va", segments=(100, 130, 30), seg_ref=(0, 1, 0),
+                                       k_ref=2, seed=13)
+    if score_mode == "tripool":
+        cfg = cfg.with_(name="ragged_r2va_tp", score_mode="tripool", proj_dim=8, seed=14)
+    return cfg
+
+
+def prefix_tile_of_token(cfg, x):
+    t, base = 0, 0
+    for length in cfg.segments:
+        if x < base + length:
+            return t + (x - base) // 64
+        t += -(-length // 64)
+        base += length
+    raise ValueError(x)
+
+
+def pin_r2va_explicit_mask(cfg):
+    """Video rows see the dense prefix segments, their k_ref kept reference tiles and
+    their k kept video tiles; prefix rows see everything: one N x N masked softmax."""
+    inp, q, k, v = inputs_f64(cfg)
+    kk = k_list(cfg, 0.5)
+    res = O.run_layer(cfg, q, k, v, kk, gate=inp.gate, w_q=inp.w_q, w_k=inp.w_k)
+    ref = O.ref_tiles(cfg)
+    assert list(ref) == [2, 3, 4]
+    N, n_pre = cfg.n_tokens, cfg.n_prefix_tokens
+    pt = np.array([prefix_tile_of_token(cfg, x) for x in range(n_pre)])
+    for h in range(cfg.heads):
+        vt = np.array([video_tile_of_token(cfg, h, x) for x in range(cfg.n_video_tokens)])
+        allowed = np.zeros((N, N), dtype=bool)
+        allowed[:n_pre, :] = True
+        for r in range(n_pre, N):
+            i = vt[r - n_pre]
+            kept_pre = [t for t in range(pt.max() + 1) if t not in ref] + [int(ref[j]) for j in res.ref_kept[h][i]]
+            allowed[r, :n_pre] = np.isin(pt, kept_pre)
+            allowed[r, n_pre:] = np.isin(vt, res.kept[h][i])
+            assert len(res.ref_kept[h][i]) == cfg.k_ref
+        want = O.masked_dense_attention(q[0, :, h], k[0, :, h], v[0, :, h], allowed, 1.0 / math.sqrt(cfg.head_dim))
+        assert np.max(np.abs(want - res.out[0, :, h])) <= 1e-12
+
+
+@pytest.mark.parametrize("mode", ["meanpool_gate", "tripool"])
+def test_r2va_equals_explicit_mask(mode):
+    pin_r2va_explicit_mask(ragged_r2va_config(mode))
+
+
+def test_r2va_all_reference_tiles_is_the_dense_prefix_layer():
+    cfg = ragged_r2va_config().with_(k_ref=3)
+    inp, q, k, v = inputs_f64(cfg)
+    kk = k_list(cfg, 0.5)
+    a = O.run_layer(cfg, q, k, v, kk, gate=inp.gate)
+    b = O.run_layer(cfg.with_(seg_ref=(), k_ref=0), q, k, v, kk, gate=inp.gate)
+    assert np.array_equal(a.out, b.out) and a.computed_pairs == b.computed_pairs
+
+
+def test_r2va_zero_gate_keeps_lowest_reference_tiles():
+    cfg = ragged_r2va_config()
+    inp, q, k, v = inputs_f64(cfg)
+    res = O.run_layer(cfg, q, k, v, k_list(cfg, 0.5), gate=np.zeros_like(inp.gate))
+    for h in range(cfg.heads):
+        assert np.all(res.ref_kept[h] == np.array([0, 1]))
+
+
+def test_mutation_r2va_drops_reference_tiles(monkeypatch):
+    good = O.query_key_tokens
+    monkeypatch.setattr(O, "query_key_tokens",
+                        lambda til, t, kept, ref=None, kept_ref=None:
+                        good(til, t, kept, ref, kept_ref[:0] if kept_ref is not None else None))
+    _expect_pin_failure(pin_r2va_explicit_mask, ragged_r2va_config())

@@ -31,6 +31,11 @@ class LayerConfig:
     sparsity: tuple            # video-key sparsity levels this workload is run at
     seed: int
     note: str = ""
+    # Reference segments (R2VA budget variant): seg_ref[s] = 1 marks prefix segment s as a
+    # reference stream whose tiles each video query tile selects with its own budget k_ref;
+    # the other segments stay dense. Empty: every prefix tile is kept (the default layer).
+    seg_ref: tuple = ()
+    k_ref: int = 0
 
     @property
     def n_prefix_tokens(self) -> int:
@@ -77,6 +82,12 @@ CONFIGS = {
         segments=(512, 3840, 640), tile_shapes=_veda(24), score_mode="tripool",
         proj_dim=64, sparsity=(0.9, 0.95), seed=3,
         note="head-aware tiling, TripPool scoring"),
+    "r2va": LayerConfig(
+        name="r2va", batch=1, heads=24, head_dim=128, T=28, H=48, W=80,
+        segments=(512, 3840, 640), tile_shapes=_uniform(24), score_mode="meanpool_gate",
+        proj_dim=128, sparsity=(1.0 - 32 / 1680,), seed=5, seg_ref=(0, 1, 0), k_ref=32,
+        note="R2VA budgets: 32 of the 60 reference-image tiles + 32 of 1680 video tiles per query "
+             "tile; text and audio tiles dense"),
     "long": LayerConfig(
         name="long", batch=1, heads=24, head_dim=128, T=60, H=48, W=80,
         segments=(512, 3840, 1280), tile_shapes=_uniform(24), score_mode="meanpool_gate",

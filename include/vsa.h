@@ -83,6 +83,15 @@ typedef struct {
   int32_t score_mode;                   /* vsa_score_mode */
   int32_t proj_dim;                     /* mean-pool gate: == head_dim; TripPool: 16..128, %16 == 0 */
   float softmax_scale;                  /* 0 -> 1/sqrt(head_dim) */
+  /* R2VA budget variant (BSAI VedaSparse README, v3.4.2 notes on the R2VA
+   * predictor: per query, 32 reference tiles and 32 video tiles; text / VLM /
+   * audio conditioning stays dense). seg_ref[s] = 1 marks prefix segment s as
+   * a reference stream: each video query tile keeps only k_ref_per_head[h] of
+   * the reference segments' tiles, chosen by the layer's scorer
+   * (vsa_ref_score, vsa_topk_select_ref, vsa_sparse_attn_ref). All zero: every
+   * prefix tile is kept by every query tile, as in the default layer. */
+  int32_t seg_ref[VSA_MAX_SEGMENTS];    /* 0 or 1 per segment */
+  int32_t k_ref_per_head[VSA_MAX_HEADS];/* 1 .. reference tiles, when any seg_ref is set */
 } vsa_desc;
 
 /* Sizes a caller needs to allocate buffers for a plan. */
@@ -99,6 +108,10 @@ typedef struct {
   int64_t workspace_bytes;              /* scratch for vsa_tile_score */
   int64_t lse_elems;                    /* batch*heads*nt_max*64 (fp32) */
   int64_t attn_work_items;              /* 128-row blocks the attention kernel schedules */
+  int32_t n_ref_tiles;                  /* tiles of the reference segments (0: none) */
+  int32_t k_ref_max;                    /* max over heads of k_ref_per_head (0: none) */
+  int64_t ref_score_elems;              /* batch*heads*ntv_max*n_ref_tiles (fp32) */
+  int64_t ref_index_elems;              /* batch*heads*ntv_max*k_ref_max (int32) */
 } vsa_plan_info;
 
 typedef struct vsa_plan vsa_plan;
@@ -229,6 +242,33 @@ VSA_API vsa_status vsa_sparse_attn(vsa_plan* plan, const void* qp, const void* k
 /* a7. Inverse of the pack permutation: [B, heads, nt_max, 64, d] -> [B, N, heads, d]. */
 VSA_API vsa_status vsa_tile_unpack(vsa_plan* plan, const void* op, void* o, void* stream);
 
+/* R2VA budgets, scores of the reference tiles: for video query tile i and
+ * reference tile r (the r-th tile of the segments marked in seg_ref, in
+ * sequence order), scores_ref[b][h][i][r] = the layer's tile score of query
+ * tile i against reference tile r (pooled K of tile r, projected with proj_k,
+ * against the projected pooled Q of tile i), fp32 [B, heads, ntv_max,
+ * n_ref_tiles]. `workspace` must hold the projected pooled Q that
+ * vsa_tile_score or vsa_tile_score_pooled just wrote into it; this call adds
+ * the reference tiles' pooled and projected K behind it (workspace_bytes
+ * covers both). kp: packed K. Same scorer and sources as vsa_tile_score. */
+VSA_API vsa_status vsa_ref_score(vsa_plan* plan, const void* kp, const float* proj_k, float* scores_ref,
+                         void* workspace, void* stream);
+
+/* R2VA budgets, a5 for the reference tiles: the k_ref_per_head[h] best
+ * reference tiles of each video query tile, ties to the lower index, written
+ * ascending into idx_ref [B, heads, ntv_max, k_ref_max] (positions 0 ..
+ * n_ref_tiles - 1). As vsa_topk_select. */
+VSA_API vsa_status vsa_topk_select_ref(vsa_plan* plan, const float* scores_ref, int32_t* idx_ref,
+                               void* stream);
+
+/* R2VA budgets, a6: vsa_sparse_attn in which a video query tile keeps, of the
+ * reference segments' tiles, only those idx_ref lists for it; the other
+ * prefix tiles stay dense and prefix query rows still see every key. Indices
+ * out of range or not ascending are rejected as in vsa_sparse_attn. */
+VSA_API vsa_status vsa_sparse_attn_ref(vsa_plan* plan, const void* qp, const void* kp, const void* vp,
+                               const int32_t* idx, const int32_t* idx_ref, void* op, float* lse,
+                               void* stream);
+
 /* Teacher tile map (row f3; the first stage of the Veda method: full attention,
  * max-pooled per tile pair, is the teacher distribution at tile level -- Veda
  * news page, "Что делает Veda"). For video query tile i and video key tile j
@@ -258,7 +298,9 @@ VSA_API vsa_status vsa_index_overlap(vsa_plan* plan, const int32_t* idx_a, const
 /* The whole layer in order on one stream, on caller-provided buffers (sizes
  * from vsa_plan_query): vsa_tile_pack_pool, vsa_tile_score_pooled,
  * vsa_topk_select, vsa_sparse_attn, vsa_tile_unpack. Returns the first
- * failing call's status. */
+ * failing call's status. Plans with reference segments (seg_ref) return
+ * VSA_ERR_UNSUPPORTED: their layer adds vsa_ref_score and
+ * vsa_topk_select_ref and attends with vsa_sparse_attn_ref. */
 VSA_API vsa_status vsa_layer_forward(vsa_plan* plan, const void* q, const void* k, const void* v,
                              const float* proj_q, const float* proj_k,
                              void* qp, void* kp, void* vp, float* scores, int32_t* idx,

@@ -27,6 +27,13 @@ def ragged_gpu_config(d=128, score_mode="meanpool_gate", batch=1, seed=21):
         sparsity=(0.5,), seed=seed)
 
 
+def r2va_gpu_config(d=128, score_mode="meanpool_gate", k_ref=2, seed=23):
+    """Text, a reference segment of 130 tokens (tiles of 64, 64 and 2 tokens), audio; the
+    reference tiles are selected per video query tile with their own budget."""
+    return ragged_gpu_config(d, score_mode, seed=seed).with_(
+        name=f"r2va{d}", segments=(100, 130, 30), seg_ref=(0, 1, 0), k_ref=k_ref)
+
+
 def no_prefix_config():
     return LayerConfig(name="noprefix", batch=1, heads=2, head_dim=128, T=8, H=8, W=8,
                        segments=(), tile_shapes=((4, 4, 4), (2, 4, 8)), score_mode="meanpool_gate",
@@ -85,12 +92,25 @@ class GpuRun:
                 p.tile_pack(self.q, self.k_t, self.v, b["qp"], b["kp"], b["vp"])
                 p.tile_score(b["qp"], b["kp"], self.proj_q, self.proj_k, b["scores"], b["workspace"])
             p.topk_select(b["scores"], b["idx"])
-            p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], b["lse"])
+            if p.info.n_ref_tiles:       # R2VA budgets
+                p.ref_score(b["kp"], self.proj_k, b["scores_ref"], b["workspace"])
+                p.topk_select_ref(b["scores_ref"], b["idx_ref"])
+                p.sparse_attn_ref(b["qp"], b["kp"], b["vp"], b["idx"], b["idx_ref"], b["op"], b["lse"])
+            else:
+                p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], b["lse"])
             p.tile_unpack(b["op"], self.out)
         else:
             p.layer_forward(self.q, self.k_t, self.v, self.proj_q, self.proj_k, b, self.out)
         p.check()
         return self
+
+    def ref_kept(self, b, h):
+        ntv, kr = n_video_tiles(self.cfg, h), int(self.cfg.k_ref)
+        return self.bufs["idx_ref"][b, h, :ntv, :kr].cpu().numpy().astype(np.int64)
+
+    def ref_scores(self, b, h):
+        ntv = n_video_tiles(self.cfg, h)
+        return self.bufs["scores_ref"][b, h, :ntv, :].double().cpu().numpy()
 
     def kept(self, b, h):
         ntv, kh = n_video_tiles(self.cfg, h), self.k[h]

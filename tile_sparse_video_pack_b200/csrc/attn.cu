@@ -160,6 +160,9 @@ static_assert(B_COUNT <= 40, "barrier slots");
 
 struct AttnParams {
   const int32_t* idx;      // [B, heads, ntv_max, k_max]
+  const int32_t* idx_ref;  // [B, heads, ntv_max, k_ref_max] kept reference tiles, or null (all prefix dense)
+  const int32_t* ref_tiles;   // [n_ref] prefix tile id of each reference tile
+  const int32_t* prefix_ref;  // [n_pre] position among the reference tiles, or -1
   const int32_t* counts;   // [heads, nt_max]
   const WorkItem* items;
   int64_t n_items;
@@ -173,6 +176,8 @@ struct AttnParams {
   float scale_log2;
   int32_t ntv[VSA_MAX_HEADS];
   int32_t k[VSA_MAX_HEADS];
+  int32_t n_ref, k_ref_max;
+  int32_t k_ref[VSA_MAX_HEADS];
 };
 
 __device__ __forceinline__ int warp_excl_scan(int v, int lane, int* total) {
@@ -286,57 +291,77 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = lane; t < nt; t += 32) list[t] = uint32_t(t) | (maskab << 16) | (uint32_t(cnt[t]) << 24);
         n_entries = nt;
       } else {
-        for (int t = lane; t < prm.n_pre; t += 32)
-          list[t] = uint32_t(t) | (maskab << 16) | (uint32_t(cnt[t]) << 24);
-        uint32_t* bmA = bitmaps;
-        uint32_t* bmB = bitmaps + prm.bitmap_words;
-        const int words = (ntv + 31) >> 5;
-        for (int w = lane; w < words; w += 32) {
-          bmA[w] = 0u;
-          bmB[w] = 0u;
-        }
-        __syncwarp();
-        const int kh = prm.k[h];
-        for (int side = 0; side < 2; ++side) {
-          const int qt = side == 0 ? wi.qa : wi.qb;
-          if (qt < 0) continue;
-          const int32_t* row = prm.idx + ((size_t(b) * prm.heads + h) * prm.ntv_max + (qt - prm.n_pre)) * prm.k_max;
-          uint32_t* bm = side == 0 ? bmA : bmB;
-          for (int e = lane; e < kh; e += 32) {
-            const int j = row[e];
-            const int jp = e > 0 ? row[e - 1] : -1;
-            if (j < 0 || j >= ntv || j <= jp) {
-              bad = true;
-            } else {
-              atomicOr(bm + (j >> 5), 1u << (j & 31));
-            }
-          }
-        }
-        bad = __any_sync(0xffffffffu, bad);
-        __syncwarp();
-        int base = prm.n_pre;
-        if (!bad) {
-          for (int w0 = 0; w0 < words; w0 += 32) {
-            const int w = w0 + lane;
-            const uint32_t a = w < words ? bmA[w] : 0u;
-            const uint32_t bb = w < words ? bmB[w] : 0u;
-            uint32_t u = a | bb;
+        int base = 0;
+        if (prm.idx_ref) {   // reference segments: the dense prefix tiles first, compacted
+          for (int t0 = 0; t0 < prm.n_pre; t0 += 32) {
+            const int t = t0 + lane;
+            const int keep = (t < prm.n_pre && prm.prefix_ref[t] < 0) ? 1 : 0;
             int total;
-            int pos = base + warp_excl_scan(__popc(u), lane, &total);
-            while (u) {
-              const int bit = __ffs(u) - 1;
-              u &= u - 1;
-              const int j = (w << 5) + bit;
-              const uint32_t m = ((a >> bit) & 1u) | (((bb >> bit) & 1u) << 1);
-              const int t = prm.n_pre + j;
-              list[pos++] = uint32_t(t) | (m << 16) | (uint32_t(cnt[t]) << 24);
-            }
+            const int pos = base + warp_excl_scan(keep, lane, &total);
+            if (keep) list[pos] = uint32_t(t) | (maskab << 16) | (uint32_t(cnt[t]) << 24);
             base += total;
           }
-        } else if (lane == 0) {
-          atomicOr(gerr, kErrBadIndex);
+        } else {             // every prefix tile
+          for (int t = lane; t < prm.n_pre; t += 32)
+            list[t] = uint32_t(t) | (maskab << 16) | (uint32_t(cnt[t]) << 24);
+          base = prm.n_pre;
         }
-        n_entries = base;
+        // The kept tiles of both query tiles, merged: each selection row (ascending
+        // positions among nbits candidate tiles) sets bits of its row-half's
+        // bitmap; the union is appended in ascending order, each entry tagged with
+        // the row-halves that keep it. A row out of range or not ascending marks
+        // the item bad (warp-uniform after the vote).
+        auto merge = [&](const int32_t* sel, int stride, int kcount, int nbits, bool is_ref) {
+          uint32_t* bmA = bitmaps;
+          uint32_t* bmB = bitmaps + prm.bitmap_words;
+          const int words = (nbits + 31) >> 5;
+          for (int w = lane; w < words; w += 32) {
+            bmA[w] = 0u;
+            bmB[w] = 0u;
+          }
+          __syncwarp();
+          for (int side = 0; side < 2; ++side) {
+            const int qt = side == 0 ? wi.qa : wi.qb;
+            if (qt < 0) continue;
+            const int32_t* row = sel + ((size_t(b) * prm.heads + h) * prm.ntv_max + (qt - prm.n_pre)) * stride;
+            uint32_t* bm = side == 0 ? bmA : bmB;
+            for (int e = lane; e < kcount; e += 32) {
+              const int j = row[e];
+              const int jp = e > 0 ? row[e - 1] : -1;
+              if (j < 0 || j >= nbits || j <= jp) {
+                bad = true;
+              } else {
+                atomicOr(bm + (j >> 5), 1u << (j & 31));
+              }
+            }
+          }
+          bad = __any_sync(0xffffffffu, bad);
+          __syncwarp();
+          if (!bad) {
+            for (int w0 = 0; w0 < words; w0 += 32) {
+              const int w = w0 + lane;
+              const uint32_t a = w < words ? bmA[w] : 0u;
+              const uint32_t bb = w < words ? bmB[w] : 0u;
+              uint32_t u = a | bb;
+              int total;
+              int pos = base + warp_excl_scan(__popc(u), lane, &total);
+              while (u) {
+                const int bit = __ffs(u) - 1;
+                u &= u - 1;
+                const int j = (w << 5) + bit;
+                const uint32_t m = ((a >> bit) & 1u) | (((bb >> bit) & 1u) << 1);
+                const int t = is_ref ? prm.ref_tiles[j] : prm.n_pre + j;
+                list[pos++] = uint32_t(t) | (m << 16) | (uint32_t(cnt[t]) << 24);
+              }
+              base += total;
+            }
+          }
+          __syncwarp();
+        };
+        if (prm.idx_ref) merge(prm.idx_ref, prm.k_ref_max, prm.k_ref[h], prm.n_ref, true);
+        if (!bad) merge(prm.idx, prm.k_max, prm.k[h], ntv, false);
+        if (bad && lane == 0) atomicOr(gerr, kErrBadIndex);
+        n_entries = base;   // a bad item keeps only entries already validated; its rows are not written
       }
       __syncwarp();
       // valid-pair count for the stats: rows x keys each row-half keeps
@@ -739,8 +764,8 @@ int attn_smem_bytes(int list_cap) {
   return 1024 + int(Smem<128>::oEnd);
 }
 
-cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp, const int32_t* idx, void* op,
-                        float* lse, cudaStream_t s) {
+cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp, const int32_t* idx,
+                        const int32_t* idx_ref, void* op, float* lse, cudaStream_t s) {
   const Geometry& g = p->geo;
   const int64_t rows = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE;
   CUtensorMap tq, tk, tv;
@@ -748,6 +773,11 @@ cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void*
     return cudaErrorInvalidValue;
   AttnParams prm;
   prm.idx = idx;
+  prm.idx_ref = idx_ref;
+  prm.ref_tiles = p->d_ref_tiles;
+  prm.prefix_ref = p->d_prefix_ref;
+  prm.n_ref = g.n_ref;
+  prm.k_ref_max = g.k_ref_max;
   prm.counts = p->d_tile_count;
   prm.items = p->d_items;
   prm.n_items = p->n_items;
@@ -767,6 +797,7 @@ cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void*
   for (int h = 0; h < VSA_MAX_HEADS; ++h) {
     prm.ntv[h] = h < g.Hh ? g.ntv[h] : 0;
     prm.k[h] = h < g.Hh ? g.k[h] : 0;
+    prm.k_ref[h] = h < g.Hh ? g.k_ref[h] : 0;
   }
   // reset the work counter and the pair count
   cudaError_t e = cudaMemsetAsync(p->d_state + 1, 0, 12, s);

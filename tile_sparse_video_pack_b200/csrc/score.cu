@@ -24,7 +24,9 @@ struct ScoreLayout {
   int p;                  // projected width
   int64_t pooled_elems;   // per tensor: B*heads*ntv_max*kd
   int64_t proj_elems;     // per tensor: B*heads*ntv_max*p
-  int64_t off_pq, off_pk, off_hq, off_hk, total;
+  int64_t off_pq, off_pk, off_hq, off_hk;
+  int64_t off_pr, off_hr;  // reference tiles (R2VA budgets): pooled and projected K, [B*heads*n_ref][..]
+  int64_t total;
 };
 
 ScoreLayout score_layout(const Geometry& g, int mode, int p) {
@@ -38,7 +40,10 @@ ScoreLayout score_layout(const Geometry& g, int mode, int p) {
   L.off_pk = L.off_pq + align256(L.pooled_elems * 4);
   L.off_hq = L.off_pk + align256(L.pooled_elems * 4);
   L.off_hk = L.off_hq + align256(L.proj_elems * 4);
-  L.total = L.off_hk + align256(L.proj_elems * 4);
+  const int64_t ref_rows = int64_t(g.B) * g.Hh * g.n_ref;
+  L.off_pr = L.off_hk + align256(L.proj_elems * 4);
+  L.off_hr = L.off_pr + align256(ref_rows * L.kd * 4);
+  L.total = L.off_hr + align256(ref_rows * p * 4);
   return L;
 }
 
@@ -107,19 +112,76 @@ __global__ void __launch_bounds__(256) pool_kernel(Geometry g, const uint16_t* _
   }
 }
 
+// Pooled K of the reference tiles (R2VA budgets): one warp per (b, h,
+// reference tile); the pooling of pool_kernel, over packed tile ref_tiles[r].
+template <int D, bool TRIP>
+__global__ void __launch_bounds__(256) pool_ref_kernel(Geometry g, const uint16_t* __restrict__ kp,
+                                                       const int32_t* __restrict__ counts,
+                                                       const int32_t* __restrict__ ref_tiles, float* __restrict__ pr) {
+  constexpr int CH = D / 32;
+  constexpr int KD = TRIP ? 3 * D : D;
+  const int64_t task = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (task >= int64_t(g.B) * g.Hh * g.n_ref) return;
+  const int r = int(task % g.n_ref);
+  const int bh = int(task / g.n_ref);
+  const int h = bh % g.Hh;
+  const int n = ref_tiles[r];
+  const int cnt = counts[h * g.nt_max + n];
+  const uint16_t* src = kp + ((int64_t(bh) * g.nt_max + n) * VSA_TILE) * D + CH * lane;
+  float sum[CH], mx[CH], mn[CH];
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    sum[c] = 0.f;
+    mx[c] = -INFINITY;
+    mn[c] = INFINITY;
+  }
+  for (int s = 0; s < cnt; ++s) {
+    float x[CH];
+    if (CH == 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(src + int64_t(s) * D);
+      x[0] = bf16_lo(u.x);
+      x[1] = bf16_hi(u.x);
+      x[2] = bf16_lo(u.y);
+      x[3] = bf16_hi(u.y);
+    } else {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(src + int64_t(s) * D);
+      x[0] = bf16_lo(u);
+      x[1] = bf16_hi(u);
+    }
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      sum[c] += x[c];
+      if (TRIP) {
+        mx[c] = fmaxf(mx[c], x[c]);
+        mn[c] = fminf(mn[c], x[c]);
+      }
+    }
+  }
+  float* dst = pr + task * KD + CH * lane;
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    dst[c] = sum[c] / float(cnt);
+    if (TRIP) {
+      dst[D + c] = mx[c];
+      dst[2 * D + c] = mn[c];
+    }
+  }
+}
+
 // C[z] (+)= alpha * A[z] * op(B[z]); z = b * heads + h; 128 x 128 tiles, 8 x 8 per thread.
 // A: [M][K] row-major (lda). B: [K][N] (ldb) or, with BT, [N][K] (ldb).
-// M = ntv[h]; N = n_fixed if > 0 else ntv[h]. K % 8 == 0, rows 16-byte aligned.
+// M = m_fixed if > 0 else ntv[h]; N = n_fixed if > 0 else ntv[h]. K % 8 == 0, rows 16-byte aligned.
 template <bool BT>
 __global__ void __launch_bounds__(256) sgemm_kernel(Geometry g, const float* __restrict__ A, int64_t sA, int lda,
                                                     const float* __restrict__ Bm, int64_t sBz, int64_t sBh,
                                                     int ldb, float* __restrict__ C, int64_t sC, int ldc, int K,
-                                                    int n_fixed, float alpha) {
+                                                    int n_fixed, float alpha, int m_fixed = 0) {
   __shared__ __align__(16) float As[8][128];
   __shared__ __align__(16) float Bs[8][128];
   const int z = blockIdx.z;
   const int h = z % g.Hh;
-  const int M = g.ntv[h];
+  const int M = m_fixed > 0 ? m_fixed : g.ntv[h];
   const int N = n_fixed > 0 ? n_fixed : g.ntv[h];
   const int m0 = blockIdx.y * 128, n0 = blockIdx.x * 128;
   if (m0 >= M || n0 >= N) return;
@@ -248,6 +310,44 @@ cudaError_t launch_score(const vsa_plan* pl, const void* qp, const void* kp, con
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_project_score(pl, proj_q, proj_k, scores, workspace, s);
+}
+
+// R2VA budgets: scores of every video query tile against the reference tiles,
+// from the projected pooled Q already in the workspace.
+cudaError_t launch_ref_score(const vsa_plan* pl, const void* kp, const float* proj_k, float* scores_ref,
+                             void* workspace, cudaStream_t s) {
+  const Geometry& g = pl->geo;
+  const int mode = pl->desc.score_mode;
+  const int p = pl->desc.proj_dim;
+  const ScoreLayout L = score_layout(g, mode, p);
+  const bool trip = mode == VSA_SCORE_TRIPPOOL;
+  char* ws = static_cast<char*>(workspace);
+  const float* hq = reinterpret_cast<const float*>(ws + L.off_hq);
+  float* pr = reinterpret_cast<float*>(ws + L.off_pr);
+  float* hr = reinterpret_cast<float*>(ws + L.off_hr);
+  const int64_t tasks = int64_t(g.B) * g.Hh * g.n_ref;
+  const int blocks = int((tasks + 7) / 8);
+  auto* k16 = static_cast<const uint16_t*>(kp);
+  if (g.d == 128) {
+    if (trip) pool_ref_kernel<128, true><<<blocks, 256, 0, s>>>(g, k16, pl->d_tile_count, pl->d_ref_tiles, pr);
+    else pool_ref_kernel<128, false><<<blocks, 256, 0, s>>>(g, k16, pl->d_tile_count, pl->d_ref_tiles, pr);
+  } else {
+    if (trip) pool_ref_kernel<64, true><<<blocks, 256, 0, s>>>(g, k16, pl->d_tile_count, pl->d_ref_tiles, pr);
+    else pool_ref_kernel<64, false><<<blocks, 256, 0, s>>>(g, k16, pl->d_tile_count, pl->d_ref_tiles, pr);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int Z = g.B * g.Hh;
+  const int64_t sW = trip ? int64_t(L.kd) * p : 0;
+  dim3 gp((p + 127) / 128, (g.n_ref + 127) / 128, Z);
+  sgemm_kernel<false><<<gp, 256, 0, s>>>(g, pr, int64_t(g.n_ref) * L.kd, L.kd, proj_k, 0, sW, p, hr,
+                                         int64_t(g.n_ref) * p, p, L.kd, p, 1.0f, g.n_ref);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 gs((g.n_ref + 127) / 128, (g.ntv_max + 127) / 128, Z);
+  sgemm_kernel<true><<<gs, 256, 0, s>>>(g, hq, int64_t(g.ntv_max) * p, p, hr, int64_t(g.n_ref) * p, 0, p, scores_ref,
+                                        int64_t(g.ntv_max) * g.n_ref, g.n_ref, p, g.n_ref, 1.0f / sqrtf(float(p)));
+  return cudaGetLastError();
 }
 
 }  // namespace vsa

@@ -44,8 +44,11 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total
   return before + x - v;
 }
 
+// ref = false: video key tiles (columns ntv[h], k[h]); ref = true: the
+// reference tiles of the R2VA budget variant (columns n_ref, k_ref[h]).
 __global__ void __launch_bounds__(kThreads) topk_kernel(Geometry g, const float* __restrict__ scores,
-                                                        int32_t* __restrict__ idx, uint32_t* __restrict__ err) {
+                                                        int32_t* __restrict__ idx, uint32_t* __restrict__ err,
+                                                        bool ref) {
   extern __shared__ uint32_t keys[];
   __shared__ int hist[256];
   __shared__ int warp_sums[kThreads / 32];
@@ -56,11 +59,11 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(Geometry g, const float*
   const int i = int(row % g.ntv_max);
   const int bh = int(row / g.ntv_max);
   const int h = bh % g.Hh;
-  const int n = g.ntv[h];
-  if (i >= n) return;
-  const int k = g.k[h];
-  const float* srow = scores + row * g.ntv_max;
-  int32_t* out = idx + row * g.k_max;
+  if (i >= g.ntv[h]) return;                   // no such query tile in this head
+  const int n = ref ? g.n_ref : g.ntv[h];       // columns
+  const int k = ref ? g.k_ref[h] : g.k[h];
+  const float* srow = scores + row * (ref ? g.n_ref : g.ntv_max);
+  int32_t* out = idx + row * (ref ? g.k_ref_max : g.k_max);
   const int tid = threadIdx.x;
 
   if (tid == 0) nan_flag = 0;
@@ -131,7 +134,19 @@ cudaError_t launch_topk(const vsa_plan* p, const float* scores, int32_t* idx, cu
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
   }
-  topk_kernel<<<unsigned(rows), kThreads, smem, s>>>(g, scores, idx, p->d_state);
+  topk_kernel<<<unsigned(rows), kThreads, smem, s>>>(g, scores, idx, p->d_state, false);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_ref(const vsa_plan* p, const float* scores_ref, int32_t* idx_ref, cudaStream_t s) {
+  const Geometry& g = p->geo;
+  const int64_t rows = int64_t(g.B) * g.Hh * g.ntv_max;
+  const size_t smem = size_t(g.n_ref) * sizeof(uint32_t);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+  }
+  topk_kernel<<<unsigned(rows), kThreads, smem, s>>>(g, scores_ref, idx_ref, p->d_state, true);
   return cudaGetLastError();
 }
 

@@ -52,6 +52,16 @@ vsa_status validate(const vsa_desc& d) {
     return VSA_ERR_INVALID_ARG;
   }
   if (!(d.softmax_scale >= 0.0f) || isinf(d.softmax_scale)) return VSA_ERR_INVALID_ARG;
+  // reference segments (R2VA budgets): flags 0/1 on existing segments, a budget per head
+  int64_t n_ref = 0;
+  for (int i = 0; i < VSA_MAX_SEGMENTS; ++i) {
+    if (d.seg_ref[i] != 0 && d.seg_ref[i] != 1) return VSA_ERR_INVALID_ARG;
+    if (d.seg_ref[i] && i >= d.n_segments) return VSA_ERR_INVALID_ARG;
+    if (d.seg_ref[i]) n_ref += cdiv(d.seg_len[i], VSA_TILE);
+  }
+  for (int h = 0; h < d.heads; ++h)
+    if (n_ref ? (d.k_ref_per_head[h] < 1 || d.k_ref_per_head[h] > n_ref) : d.k_ref_per_head[h] != 0)
+      return VSA_ERR_INVALID_ARG;
   return VSA_OK;
 }
 
@@ -152,6 +162,19 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
     g.k_max = std::max(g.k_max, g.k[h]);
   }
   g.nt_max = g.n_pre_tiles + g.ntv_max;
+  std::vector<int32_t> ref_tiles, prefix_ref(size_t(g.n_pre_tiles), -1);
+  for (int i = 0; i < d.n_segments; ++i)
+    if (d.seg_ref[i])
+      for (int t = g.seg_tile0[i]; t < g.seg_tile0[i + 1]; ++t) {
+        prefix_ref[size_t(t)] = int32_t(ref_tiles.size());
+        ref_tiles.push_back(t);
+      }
+  g.n_ref = int32_t(ref_tiles.size());
+  g.k_ref_max = 0;
+  for (int h = 0; h < d.heads; ++h) {
+    g.k_ref[h] = g.n_ref ? d.k_ref_per_head[h] : 0;
+    g.k_ref_max = std::max(g.k_ref_max, g.k_ref[h]);
+  }
 
   // the attention kernel builds each item's merged key list (at most every
   // tile of a head, 16-bit tile ids) in a per-CTA slice of global memory
@@ -175,6 +198,10 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
   info.index_elems = int64_t(g.B) * g.Hh * g.ntv_max * g.k_max;
   info.workspace_bytes = vsa::score_workspace_bytes(g, d.score_mode, d.proj_dim);
   info.lse_elems = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE;
+  info.n_ref_tiles = g.n_ref;
+  info.k_ref_max = g.k_ref_max;
+  info.ref_score_elems = int64_t(g.B) * g.Hh * g.ntv_max * g.n_ref;
+  info.ref_index_elems = int64_t(g.B) * g.Hh * g.ntv_max * g.k_ref_max;
 
   // tile valid counts
   std::vector<int32_t> counts(size_t(g.Hh) * g.nt_max, 0);
@@ -229,6 +256,14 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
   if (e == cudaSuccess)
     e = cudaMemcpy(p->d_items, items.data(), items.size() * sizeof(WorkItem), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemset(p->d_state, 0, 64);
+  if (e == cudaSuccess && g.n_pre_tiles > 0) {
+    std::vector<int32_t> ref_table(ref_tiles);
+    ref_table.insert(ref_table.end(), prefix_ref.begin(), prefix_ref.end());
+    e = cudaMalloc(&p->d_ref_tiles, ref_table.size() * sizeof(int32_t));
+    if (e == cudaSuccess)
+      e = cudaMemcpy(p->d_ref_tiles, ref_table.data(), ref_table.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+    p->d_prefix_ref = p->d_ref_tiles ? p->d_ref_tiles + g.n_ref : nullptr;
+  }
   if (e != cudaSuccess) {
     cudaGetLastError();
     vsa_status r = (e == cudaErrorMemoryAllocation) ? VSA_ERR_NO_MEMORY : VSA_ERR_CUDA;
@@ -241,8 +276,9 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
 
 vsa_status vsa_plan_destroy(vsa_plan* p) {
   if (!p) return VSA_OK;
-  if (p->d_tile_count || p->d_items || p->d_state || p->d_lists) cudaDeviceSynchronize();
+  if (p->d_tile_count || p->d_items || p->d_state || p->d_lists || p->d_ref_tiles) cudaDeviceSynchronize();
   if (p->d_tile_count) cudaFree(p->d_tile_count);
+  if (p->d_ref_tiles) cudaFree(p->d_ref_tiles);
   if (p->d_items) cudaFree(p->d_items);
   if (p->d_state) cudaFree(p->d_state);
   if (p->d_lists) cudaFree(p->d_lists);
@@ -348,7 +384,40 @@ vsa_status vsa_sparse_attn(vsa_plan* p, const void* qp, const void* kp, const vo
       (lse && !aligned16(lse)))
     return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_attn++;
-  if (vsa::launch_attn(p, qp, kp, vp, idx, op, lse, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (vsa::launch_attn(p, qp, kp, vp, idx, nullptr, op, lse, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_ref_score(vsa_plan* p, const void* kp, const float* proj_k, float* scores_ref, void* ws,
+                         void* stream) {
+  if (!p || !kp || !proj_k || !scores_ref || !ws) return fail(p, VSA_ERR_INVALID_ARG);
+  if (p->geo.n_ref == 0) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!aligned16(kp) || !aligned16(proj_k) || !aligned16(scores_ref) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_score++;
+  if (vsa::launch_ref_score(p, kp, proj_k, scores_ref, ws, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_topk_select_ref(vsa_plan* p, const float* scores_ref, int32_t* idx_ref, void* stream) {
+  if (!p || !scores_ref || !idx_ref || p->geo.n_ref == 0 || !aligned16(scores_ref) || !aligned16(idx_ref))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_select++;
+  if (vsa::launch_topk_ref(p, scores_ref, idx_ref, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_sparse_attn_ref(vsa_plan* p, const void* qp, const void* kp, const void* vp, const int32_t* idx,
+                               const int32_t* idx_ref, void* op, float* lse, void* stream) {
+  if (!p || !qp || !kp || !vp || !idx || !idx_ref || !op || p->geo.n_ref == 0) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(idx) || !aligned16(idx_ref) ||
+      !aligned16(op) || (lse && !aligned16(lse)))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_attn++;
+  if (vsa::launch_attn(p, qp, kp, vp, idx, idx_ref, op, lse, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
   return VSA_OK;
 }
@@ -357,6 +426,7 @@ vsa_status vsa_layer_forward(vsa_plan* p, const void* q, const void* k, const vo
                              const float* proj_q, const float* proj_k, void* qp, void* kp, void* vp,
                              float* scores, int32_t* idx, void* op, float* lse, void* ws, void* o,
                              void* stream) {
+  if (p && p->geo.n_ref) return fail(p, VSA_ERR_UNSUPPORTED);
   vsa_status s = vsa_tile_pack_pool(p, q, k, v, qp, kp, vp, ws, stream);
   if (s == VSA_OK) s = vsa_tile_score_pooled(p, proj_q, proj_k, scores, ws, stream);
   if (s == VSA_OK) s = vsa_topk_select(p, scores, idx, stream);

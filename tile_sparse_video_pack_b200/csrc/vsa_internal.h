@@ -28,6 +28,9 @@ struct Geometry {
   int32_t pt[VSA_MAX_HEADS], ph[VSA_MAX_HEADS], pw[VSA_MAX_HEADS];
   int32_t nY[VSA_MAX_HEADS], nX[VSA_MAX_HEADS], ntv[VSA_MAX_HEADS];
   int32_t k[VSA_MAX_HEADS];
+  // reference tiles of the R2VA budget variant (0 when no segment is marked)
+  int32_t n_ref, k_ref_max;
+  int32_t k_ref[VSA_MAX_HEADS];
 };
 
 // One 128-row block of attention work: two query tiles of one (batch, head)
@@ -53,6 +56,8 @@ struct vsa_plan {
   int64_t n_items;
   uint32_t* d_state;       // [0] error word, [1] work counter
   uint32_t* d_lists;       // attention key lists and bitmaps, one slice per CTA
+  int32_t* d_ref_tiles;    // [n_ref] prefix tile ids of the reference tiles, then
+  int32_t* d_prefix_ref;   // [n_pre_tiles] each prefix tile's position among them, or -1
   int attn_smem_bytes;
   int list_cap;            // entries of one key-list buffer in the attention kernel
 };
@@ -73,8 +78,11 @@ void score_pooled_ptrs(const vsa_plan* p, void* workspace, float** pooled_q, flo
 cudaError_t launch_project_score(const vsa_plan* p, const float* proj_q, const float* proj_k, float* scores,
                                  void* workspace, cudaStream_t s);
 cudaError_t launch_topk(const vsa_plan* p, const float* scores, int32_t* idx, cudaStream_t s);
+cudaError_t launch_topk_ref(const vsa_plan* p, const float* scores_ref, int32_t* idx_ref, cudaStream_t s);
+cudaError_t launch_ref_score(const vsa_plan* p, const void* kp, const float* proj_k, float* scores_ref,
+                             void* workspace, cudaStream_t s);
 cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp,
-                        const int32_t* idx, void* op, float* lse, cudaStream_t s);
+                        const int32_t* idx, const int32_t* idx_ref, void* op, float* lse, cudaStream_t s);
 int attn_smem_bytes(int list_cap);
 cudaError_t launch_teacher(vsa_plan* p, const void* qp, const void* kp, const float* lse, float* teacher,
                            cudaStream_t s);

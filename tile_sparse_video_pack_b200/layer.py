@@ -27,18 +27,26 @@ class TileSparseAttention:
         import torch
         if out is None:
             out = torch.empty_like(q)
+        if self.plan.info.n_ref_tiles:       # R2VA budgets: the per-call path with the reference selection
+            return self.stages(q, k, v, out, stream)
         self.plan.layer_forward(q, k, v, self.proj_q, self.proj_k, self.bufs, out, stream=stream)
         return out
 
     __call__ = forward
 
     def stages(self, q, k, v, out, stream=None):
-        """The five calls one by one (same result as :meth:`forward`)."""
+        """The calls one by one (same result as :meth:`forward`); with reference segments,
+        the reference tiles are scored and selected and the attention uses that selection."""
         b, p = self.bufs, self.plan
         p.tile_pack_pool(q, k, v, b["qp"], b["kp"], b["vp"], b["workspace"], stream)
         p.tile_score_pooled(self.proj_q, self.proj_k, b["scores"], b["workspace"], stream)
         p.topk_select(b["scores"], b["idx"], stream)
-        p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], b["lse"], stream)
+        if p.info.n_ref_tiles:
+            p.ref_score(b["kp"], self.proj_k, b["scores_ref"], b["workspace"], stream)
+            p.topk_select_ref(b["scores_ref"], b["idx_ref"], stream)
+            p.sparse_attn_ref(b["qp"], b["kp"], b["vp"], b["idx"], b["idx_ref"], b["op"], b["lse"], stream)
+        else:
+            p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], b["lse"], stream)
         p.tile_unpack(b["op"], out, stream)
         return out
 

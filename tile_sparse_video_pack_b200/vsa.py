@@ -26,7 +26,8 @@ SCORE_MODES = {"meanpool_gate": 0, "tripool": 1}
 EXPORTS = ("vsa_plan_create", "vsa_plan_destroy", "vsa_plan_query", "vsa_plan_get_stats", "vsa_k_from_sparsity",
            "vsa_tile_pack", "vsa_tile_score", "vsa_topk_select", "vsa_sparse_attn", "vsa_tile_unpack",
            "vsa_layer_forward", "vsa_plan_check", "vsa_status_string", "vsa_tile_score_static",
-           "vsa_tile_pack_pool", "vsa_tile_score_pooled", "vsa_teacher_tiles", "vsa_index_overlap")
+           "vsa_tile_pack_pool", "vsa_tile_score_pooled", "vsa_teacher_tiles", "vsa_index_overlap",
+           "vsa_ref_score", "vsa_topk_select_ref", "vsa_sparse_attn_ref")
 
 
 class VsaDesc(ctypes.Structure):
@@ -37,6 +38,7 @@ class VsaDesc(ctypes.Structure):
         ("tile_shape", (ctypes.c_int32 * 3) * MAX_HEADS),
         ("k_per_head", ctypes.c_int32 * MAX_HEADS),
         ("score_mode", ctypes.c_int32), ("proj_dim", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+        ("seg_ref", ctypes.c_int32 * MAX_SEGMENTS), ("k_ref_per_head", ctypes.c_int32 * MAX_HEADS),
     ]
 
 
@@ -46,6 +48,8 @@ class VsaPlanInfo(ctypes.Structure):
         ("ntv_max", ctypes.c_int32), ("ntv", ctypes.c_int32 * MAX_HEADS), ("k_max", ctypes.c_int32),
         ("packed_elems", ctypes.c_int64), ("score_elems", ctypes.c_int64), ("index_elems", ctypes.c_int64),
         ("workspace_bytes", ctypes.c_int64), ("lse_elems", ctypes.c_int64), ("attn_work_items", ctypes.c_int64),
+        ("n_ref_tiles", ctypes.c_int32), ("k_ref_max", ctypes.c_int32),
+        ("ref_score_elems", ctypes.c_int64), ("ref_index_elems", ctypes.c_int64),
     ]
 
 
@@ -94,6 +98,9 @@ def library() -> ctypes.CDLL:
         "vsa_tile_score_pooled": (I32, [P] * 6),
         "vsa_teacher_tiles": (I32, [P] * 6),
         "vsa_index_overlap": (I32, [P] * 5),
+        "vsa_ref_score": (I32, [P] * 6),
+        "vsa_topk_select_ref": (I32, [P] * 4),
+        "vsa_sparse_attn_ref": (I32, [P] * 9),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -112,7 +119,7 @@ def _check(status: int, where: str):
 
 
 def make_desc(batch, heads, head_dim, T, H, W, segments, tile_shapes, k_per_head, score_mode="meanpool_gate",
-              proj_dim=None, softmax_scale=0.0) -> VsaDesc:
+              proj_dim=None, softmax_scale=0.0, seg_ref=(), k_ref_per_head=()) -> VsaDesc:
     d = VsaDesc()
     d.batch, d.heads, d.head_dim = batch, heads, head_dim
     d.T, d.H, d.W = T, H, W
@@ -129,6 +136,10 @@ def make_desc(batch, heads, head_dim, T, H, W, segments, tile_shapes, k_per_head
     d.score_mode = SCORE_MODES[score_mode] if isinstance(score_mode, str) else int(score_mode)
     d.proj_dim = head_dim if proj_dim is None else proj_dim
     d.softmax_scale = softmax_scale
+    for i, f in enumerate(seg_ref):
+        d.seg_ref[i] = int(f)
+    for h, k in enumerate(k_ref_per_head):
+        d.k_ref_per_head[h] = k
     return d
 
 
@@ -176,8 +187,11 @@ class Plan:
             for (pt, ph, pw) in cfg.tile_shapes:
                 n = -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw)
                 ks.append(k_from_sparsity(sparsity, n))
+        seg_ref = tuple(getattr(cfg, "seg_ref", ()))
+        k_ref = [int(cfg.k_ref)] * cfg.heads if any(seg_ref) else []
         return cls(make_desc(cfg.batch, cfg.heads, cfg.head_dim, cfg.T, cfg.H, cfg.W, cfg.segments,
-                             cfg.tile_shapes, ks, cfg.score_mode, cfg.proj_dim))
+                             cfg.tile_shapes, ks, cfg.score_mode, cfg.proj_dim, seg_ref=seg_ref,
+                             k_ref_per_head=k_ref))
 
     def close(self):
         if getattr(self, "_h", None):
@@ -204,6 +218,8 @@ class Plan:
             "idx": (d.batch, d.heads, i.ntv_max, i.k_max),
             "lse": (d.batch, d.heads, i.nt_max, TILE),
             "workspace": (i.workspace_bytes,),
+            "scores_ref": (d.batch, d.heads, i.ntv_max, i.n_ref_tiles),
+            "idx_ref": (d.batch, d.heads, i.ntv_max, i.k_ref_max),
         }
 
     def allocate(self, device=None, with_lse=False):
@@ -221,6 +237,9 @@ class Plan:
             "workspace": torch.empty(s["workspace"], dtype=torch.uint8, device=dev),
             "lse": torch.empty(s["lse"], dtype=torch.float32, device=dev) if with_lse else None,
         }
+        if self.info.n_ref_tiles:
+            bufs["scores_ref"] = torch.empty(s["scores_ref"], dtype=torch.float32, device=dev)
+            bufs["idx_ref"] = torch.empty(s["idx_ref"], dtype=torch.int32, device=dev)
         return bufs
 
     # ---- the five calls (same names as the C ABI) ------------------------------
@@ -309,6 +328,30 @@ class Plan:
             self._h, _ptr(qp, bf, "qp", pe), _ptr(kp, bf, "kp", pe), _ptr(vp, bf, "vp", pe),
             _ptr(idx, torch.int32, "idx", self.info.index_elems), _ptr(op, bf, "op", pe),
             _ptr(lse, torch.float32, "lse", self.info.lse_elems), _stream(stream)), "vsa_sparse_attn")
+
+    def ref_score(self, kp, proj_k, scores_ref, workspace, stream=None):
+        """Scores of the reference tiles (R2VA budgets); after tile_score(_pooled) on the same workspace."""
+        import torch
+        _check(library().vsa_ref_score(
+            self._h, _ptr(kp, torch.bfloat16, "kp", self.info.packed_elems), _ptr(proj_k, torch.float32, "proj_k"),
+            _ptr(scores_ref, torch.float32, "scores_ref", self.info.ref_score_elems),
+            _ptr(workspace, torch.uint8, "workspace", self.info.workspace_bytes), _stream(stream)), "vsa_ref_score")
+
+    def topk_select_ref(self, scores_ref, idx_ref, stream=None):
+        import torch
+        _check(library().vsa_topk_select_ref(
+            self._h, _ptr(scores_ref, torch.float32, "scores_ref", self.info.ref_score_elems),
+            _ptr(idx_ref, torch.int32, "idx_ref", self.info.ref_index_elems), _stream(stream)),
+            "vsa_topk_select_ref")
+
+    def sparse_attn_ref(self, qp, kp, vp, idx, idx_ref, op, lse=None, stream=None):
+        import torch
+        pe, bf = self.info.packed_elems, torch.bfloat16
+        _check(library().vsa_sparse_attn_ref(
+            self._h, _ptr(qp, bf, "qp", pe), _ptr(kp, bf, "kp", pe), _ptr(vp, bf, "vp", pe),
+            _ptr(idx, torch.int32, "idx", self.info.index_elems),
+            _ptr(idx_ref, torch.int32, "idx_ref", self.info.ref_index_elems), _ptr(op, bf, "op", pe),
+            _ptr(lse, torch.float32, "lse", self.info.lse_elems), _stream(stream)), "vsa_sparse_attn_ref")
 
     def tile_unpack(self, op, o, stream=None):
         import torch

@@ -33,7 +33,6 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 CONFIG = "full"
-SPARSITY = 0.75
 SECONDARY_SPARSITY = 0.9
 KERNELS_PER_STEP = 7  # pack + pool 1, score 3 (2 projections, scores), select 1, attention 1, unpack 1
 
@@ -45,14 +44,19 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=CONFIG)
-    ap.add_argument("--sparsity", type=float, default=SPARSITY)
+    ap.add_argument("--sparsity", type=float, default=None,
+                    help="video-key sparsity (default: the workload's first level, 0.75 for the full clip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
     ap.add_argument("--teacher", action="store_true",
                     help="also time the teacher tile map and report the selection's tile recall")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.sparsity is None:
+        from vsa_synth import get_config
+        args.sparsity = get_config(args.config).sparsity[0]
+    return args
 
 
 def measured_peaks():
@@ -108,13 +112,20 @@ def k_list(cfg, s):
 
 
 def attention_flops(cfg, ks):
-    """4 * d * sum over query rows of their key count (full tiles: closed form)."""
+    """4 * d * sum over query rows of their key count (full tiles: closed form).
+
+    With reference segments (R2VA budgets) a video row sees the dense prefix tokens
+    plus k_ref reference tiles of 64 tokens instead of the whole prefix.
+    """
     n = cfg.n_tokens
     npre = cfg.n_prefix_tokens
     nv = cfg.n_video_tokens
+    flags = tuple(getattr(cfg, "seg_ref", ())) or (0,) * len(cfg.segments)
+    ref_tok = sum(length for length, f in zip(cfg.segments, flags) if f)
+    video_prefix = npre - ref_tok + (64 * cfg.k_ref if ref_tok else 0)
     pairs = 0
     for kh in ks:
-        pairs += npre * n + nv * (npre + kh * 64)
+        pairs += npre * n + nv * (video_prefix + kh * 64)
     return 4 * cfg.head_dim * pairs * cfg.batch
 
 
@@ -354,8 +365,14 @@ def run_ours(args, rank, world, local_rank):
             p.tile_score_pooled(pq, pk, b["scores"], b["workspace"])
             e[2].record(stream)
             p.topk_select(b["scores"], b["idx"])
+            if p.info.n_ref_tiles:          # R2VA budgets: reference tiles scored and selected too
+                p.ref_score(b["kp"], pk, b["scores_ref"], b["workspace"])
+                p.topk_select_ref(b["scores_ref"], b["idx_ref"])
             e[3].record(stream)
-            p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], None)
+            if p.info.n_ref_tiles:
+                p.sparse_attn_ref(b["qp"], b["kp"], b["vp"], b["idx"], b["idx_ref"], b["op"], None)
+            else:
+                p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], None)
             e[4].record(stream)
             p.tile_unpack(b["op"], out)
             e[5].record(stream)
@@ -448,7 +465,9 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"{cfg.name}: one layer, B={cfg.batch}, {cfg.heads} heads, d={cfg.head_dim}, "
                                f"grid {cfg.T}x{cfg.H}x{cfg.W} + prefix {list(cfg.segments)}, "
-                               f"{cfg.score_mode}, sparsity {args.sparsity} (k={ks[0]})",
+                               f"{cfg.score_mode}, sparsity {args.sparsity} (k={ks[0]})"
+                               + (f", reference segments {list(cfg.seg_ref)} with k_ref={cfg.k_ref}"
+                                  if cfg.seg_ref and any(cfg.seg_ref) else ""),
                    "tokens": cfg.n_tokens, "heads": cfg.heads, "head_dim": cfg.head_dim, "k": ks[0],
                    "layers_per_step": world, "parallelism": f"independent layers x{world}",
                    "l2": "inputs larger than L2 (Q, K, V 691 MB each)"},
@@ -458,7 +477,7 @@ def run_ours(args, rank, world, local_rank):
         "score_select_share": round((stages["score"] + stages["select"]) / sum(stages.values()), 4),
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (KERNELS_PER_STEP + (4 if cfg.seg_ref and any(cfg.seg_ref) else 0)) * args.steps,
         "clocks": clocks,
         "attention_computed_pct": round(100.0 * stats["computed_pairs"] / stats["dense_pairs"], 2),
         "secondary": secondary,

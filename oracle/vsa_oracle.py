@@ -290,7 +290,7 @@ class LayerResult:
 
 def run_layer(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, k_per_head,
               gate=None, w_q=None, w_k=None, query_tiles=None,
-              heads=None, kept=None, kept_ref=None) -> LayerResult:
+              heads=None, kept=None, kept_ref=None, qk_fp8=False) -> LayerResult:
     """The whole layer, in fp64: tile, score, select, attend.
 
     ``q``, ``k``, ``v``: ``[B, N, heads, d]`` (any float dtype; widened to fp64).
@@ -301,7 +301,9 @@ def run_layer(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, k_per_head,
     video tiles to attend with instead of the oracle's own top-k (the scores
     are still computed and returned). With reference segments (``cfg.seg_ref``),
     each video query tile also keeps its ``cfg.k_ref`` best reference tiles by the
-    same scorer; ``kept_ref`` overrides that choice like ``kept``.
+    same scorer; ``kept_ref`` overrides that choice like ``kept``. ``qk_fp8``: the
+    attention logits use Q and K quantised per packed tile to e4m3 with one fp32 scale
+    per tile (:func:`quantize_tile_e4m3`); scoring and selection still use the bf16 inputs.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -337,6 +339,9 @@ def run_layer(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, k_per_head,
             if b == 0:
                 all_scores[h], all_kept[h] = s, kept_bh
                 all_rs[h], all_rk[h] = rs, rk
+            qa, ka = q[b, :, h], k[b, :, h]
+            if qk_fp8:
+                qa, ka = dequantized_tiles(qa, til), dequantized_tiles(ka, til)
             for t in tiles_h:
                 qt = til.all[t]
                 if t < til.n_prefix:
@@ -344,8 +349,8 @@ def run_layer(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, k_per_head,
                 else:
                     kv = query_key_tokens(til, t, kept_bh[t - til.n_prefix], ref,
                                           None if rk is None else rk[t - til.n_prefix])
-                o, l, rs = softmax_attention(q[b, qt, h], k[b, kv, h], v[b, kv, h], scale)
-                out[b, qt, h], lse[b, qt, h], row_sum[b, qt, h] = o, l, rs
+                o, l, rsum = softmax_attention(qa[qt], ka[kv], v[b, kv, h], scale)
+                out[b, qt, h], lse[b, qt, h], row_sum[b, qt, h] = o, l, rsum
                 pairs += len(qt) * len(kv)
     return LayerResult(all_scores, all_kept, out, lse, row_sum, pairs, all_rs, all_rk)
 
@@ -448,3 +453,43 @@ def tile_recall(kept_row: np.ndarray, teacher_row: np.ndarray, k: int) -> float:
     keeps: the tile recall by which the BSAI VedaSparse README ("Core Technology") compares
     TripPool with mean pooling."""
     return len(np.intersect1d(kept_row, topk_row(teacher_row, k))) / k
+
+
+# ---------------------------------------------------------------------------
+# fp8 (e4m3) Q K^T with per-tile scales
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Nearest value of the e4m3 format (1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+    bits, subnormals below 2^-6, no infinities, largest finite 448), ties to the even
+    mantissa, magnitudes above 448 saturated to 448. fp64 in, fp64 out (every e4m3 value is
+    exact in fp64)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))   # exponent; subnormals share 2^-6's spacing
+    step = 2.0 ** (e - 3)                               # 8 steps per binade
+    q = np.minimum(np.round(a / step) * step, E4M3_MAX)   # np.round: half to even
+    return np.sign(x) * q
+
+
+def quantize_tile_e4m3(x: np.ndarray):
+    """Per-tile fp8 quantisation of one packed tile's rows (the tile-skipping kernels on the
+    Veda page run their QK^T in 8-bit with per-tile scales; the plainest reading): the scale
+    is the tile's largest magnitude / 448 in fp32 (1 for an all-zero tile), each value is
+    divided by it in fp32 and rounded to e4m3. Returns (codes as fp64 values, scale)."""
+    xf = np.asarray(x, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(xf))) if xf.size else np.float32(0)
+    scale = np.float32(amax / np.float32(E4M3_MAX)) if amax > 0 else np.float32(1.0)
+    return e4m3_round((xf / scale).astype(np.float64)), float(scale)
+
+
+def dequantized_tiles(x_h: np.ndarray, til: HeadTiling) -> np.ndarray:
+    """One head's token rows with every tile replaced by its e4m3 codes times its scale."""
+    out = np.array(x_h, dtype=np.float64)
+    for t in til.all:
+        codes, scale = quantize_tile_e4m3(out[t])
+        out[t] = codes * scale
+    return out

@@ -517,3 +517,60 @@ def test_mutation_r2va_drops_reference_tiles(monkeypatch):
                         lambda til, t, kept, ref=None, kept_ref=None:
                         good(til, t, kept, ref, kept_ref[:0] if kept_ref is not None else None))
     _expect_pin_failure(pin_r2va_explicit_mask, ragged_r2va_config())
+
+
+# ------------------------------------------- fp8 (e4m3) Q K^T per-tile scales ---
+
+def test_e4m3_round_matches_torch_float8():
+    """Against torch's float8_e4m3fn conversion (round to nearest even), which is a
+    library routine independent of the oracle: every finite code, every midpoint between
+    neighbouring codes, and random values within the finite range."""
+    import torch
+    codes = torch.arange(256, dtype=torch.int16).to(torch.uint8).view(torch.float8_e4m3fn).float().double().numpy()
+    finite = np.unique(codes[np.isfinite(codes)])
+    mids = (finite[1:] + finite[:-1]) / 2
+    rng = np.random.default_rng(3)
+    xs = np.concatenate([finite, mids, rng.uniform(-448, 448, 20000), rng.normal(0, 1e-2, 20000)])
+    want = torch.from_numpy(xs).to(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(O.e4m3_round(xs), want)
+    assert np.array_equal(O.e4m3_round(finite), finite)          # idempotent on the codes
+    assert O.e4m3_round(np.array([500.0, -1e6]))[0] == 448.0      # saturates (torch would give NaN)
+
+
+def test_tile_quantisation_scale_and_range():
+    rng = np.random.default_rng(4)
+    x = rng.normal(0, 3, (64, 128)).astype(np.float32)
+    codes, scale = O.quantize_tile_e4m3(x)
+    assert np.float32(scale) == np.float32(np.max(np.abs(x)) / np.float32(448.0))
+    assert np.max(np.abs(codes)) == 448.0
+    rel = np.abs(codes * scale - x) / np.maximum(np.abs(x), 1e-30)
+    assert np.max(rel[np.abs(x) > 2.0 ** -6 * scale]) <= 2.0 ** -4 + 1e-7   # half a mantissa step
+    assert O.quantize_tile_e4m3(np.zeros((3, 8)))[1] == 1.0
+
+
+def test_fp8_attention_is_exact_on_representable_inputs():
+    """Q and K entries from {0, +-0.5, +-1, +-1.75} with a 1.75 in every tile: every scale
+    is 1.75/448 = 2^-8 exactly and every entry divided by it (0, 128, 256, 448) is an e4m3
+    value, so quantisation is exact and the fp8 layer equals the bf16 one."""
+    cfg = ragged_config(batch=1)
+    inp, q, k, v = inputs_f64(cfg)
+    rng = np.random.default_rng(6)
+    vals = [-1.75, -1.0, -0.5, 0.0, 0.5, 1.0, 1.75]
+    q = rng.choice(vals, size=q.shape)
+    k = rng.choice(vals, size=k.shape)
+    q[..., 0] = k[..., 0] = 1.75       # every token, so every tile, holds the largest magnitude
+    kk = k_list(cfg, 0.5)
+    a = O.run_layer(cfg, q, k, v, kk, gate=inp.gate)
+    b = O.run_layer(cfg, q, k, v, kk, gate=inp.gate, qk_fp8=True)
+    assert np.array_equal(a.out, b.out)
+
+
+def test_fp8_attention_close_to_bf16_and_not_equal():
+    cfg = ragged_config(batch=1)
+    inp, q, k, v = inputs_f64(cfg)
+    kk = k_list(cfg, 0.5)
+    a = O.run_layer(cfg, q, k, v, kk, gate=inp.gate)
+    b = O.run_layer(cfg, q, k, v, kk, gate=inp.gate, qk_fp8=True)
+    d = np.abs(a.out - b.out)
+    assert 0 < np.max(d) < 0.3 * np.max(np.abs(a.out))      # e4m3 keeps 3 mantissa bits
+    assert all(np.array_equal(x, y) for x, y in zip(a.kept, b.kept))   # selection unchanged

@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="Q K^T from e4m3 tiles with per-tile scales (vsa_tile_pack_pool_fp8 + vsa_sparse_attn_fp8)")
     ap.add_argument("--teacher", action="store_true",
                     help="also time the teacher tile map and report the selection's tile recall")
     args = ap.parse_args()
@@ -357,10 +359,15 @@ def run_ours(args, rank, world, local_rank):
         barrier()
         torch.cuda.synchronize()
         b, p = layer.bufs, layer.plan
+        f8 = p.allocate_fp8() if args.fp8 else None
         for i in range(steps):
             e = ev[i]
             e[0].record(stream)
-            p.tile_pack_pool(q, k, v, b["qp"], b["kp"], b["vp"], b["workspace"])
+            if f8 is not None:
+                p.tile_pack_pool_fp8(q, k, v, b["qp"], b["kp"], b["vp"], f8["qp8"], f8["kp8"], f8["q_scale"],
+                                     f8["k_scale"], b["workspace"])
+            else:
+                p.tile_pack_pool(q, k, v, b["qp"], b["kp"], b["vp"], b["workspace"])
             e[1].record(stream)
             p.tile_score_pooled(pq, pk, b["scores"], b["workspace"])
             e[2].record(stream)
@@ -369,7 +376,9 @@ def run_ours(args, rank, world, local_rank):
                 p.ref_score(b["kp"], pk, b["scores_ref"], b["workspace"])
                 p.topk_select_ref(b["scores_ref"], b["idx_ref"])
             e[3].record(stream)
-            if p.info.n_ref_tiles:
+            if f8 is not None:
+                p.sparse_attn_fp8(f8["qp8"], f8["kp8"], f8["q_scale"], f8["k_scale"], b["vp"], b["idx"], b["op"])
+            elif p.info.n_ref_tiles:
                 p.sparse_attn_ref(b["qp"], b["kp"], b["vp"], b["idx"], b["idx_ref"], b["op"], None)
             else:
                 p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], None)
@@ -436,8 +445,10 @@ def run_ours(args, rank, world, local_rank):
     achieved = flops / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": measured_traffic(args.config, args.sparsity, cfg.heads),
-                "kernel": "attn_kernel (vsa_sparse_attn)",
+                "frac": round(achieved / peak, 4),
+                "traffic": None if args.fp8 else measured_traffic(args.config, args.sparsity, cfg.heads),
+                "kernel": "attn_kernel<128, fp8> (vsa_sparse_attn_fp8; e4m3 Q K^T, bf16 P V)" if args.fp8
+                          else "attn_kernel (vsa_sparse_attn)",
                 "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
                 "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),
                 "algorithmic_flops_per_launch": flops}

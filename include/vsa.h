@@ -112,6 +112,7 @@ typedef struct {
   int32_t k_ref_max;                    /* max over heads of k_ref_per_head (0: none) */
   int64_t ref_score_elems;              /* batch*heads*ntv_max*n_ref_tiles (fp32) */
   int64_t ref_index_elems;              /* batch*heads*ntv_max*k_ref_max (int32) */
+  int64_t tile_scale_elems;             /* batch*heads*nt_max: one fp32 scale per packed tile (fp8 path) */
 } vsa_plan_info;
 
 typedef struct vsa_plan vsa_plan;
@@ -268,6 +269,26 @@ VSA_API vsa_status vsa_topk_select_ref(vsa_plan* plan, const float* scores_ref, 
 VSA_API vsa_status vsa_sparse_attn_ref(vsa_plan* plan, const void* qp, const void* kp, const void* vp,
                                const int32_t* idx, const int32_t* idx_ref, void* op, float* lse,
                                void* stream);
+
+/* fp8 Q K^T (row f2; the tile-skipping kernels on the Veda page run Q K^T in
+ * 8-bit with per-tile scales). vsa_tile_pack_pool, and besides: Q and K of
+ * every packed tile as e4m3 bytes qp8, kp8 ([B, heads, nt_max, 64, head_dim]
+ * bytes, packed_elems of them) with one fp32 scale per (tile, tensor) in
+ * q_scale, k_scale ([B, heads, nt_max], tile_scale_elems): scale = the tile's
+ * largest magnitude / 448 (fp32 division; 1 for an all-zero tile), code =
+ * e4m3(x / scale) (fp32 division, round to nearest even, saturating).
+ * head_dim 128 only (VSA_ERR_UNSUPPORTED otherwise). */
+VSA_API vsa_status vsa_tile_pack_pool_fp8(vsa_plan* plan, const void* q, const void* k, const void* v,
+                                  void* qp, void* kp, void* vp, void* qp8, void* kp8, float* q_scale,
+                                  float* k_scale, void* workspace, void* stream);
+
+/* vsa_sparse_attn with the logits from the e4m3 tiles: s = (q8 . k8) *
+ * q_scale[query tile] * k_scale[key tile] * softmax_scale, accumulated in
+ * fp32 on the tensor cores; P and V stay bf16. qp8, kp8, q_scale, k_scale as
+ * written by vsa_tile_pack_pool_fp8; vp the bf16 packed V. head_dim 128. */
+VSA_API vsa_status vsa_sparse_attn_fp8(vsa_plan* plan, const void* qp8, const void* kp8, const float* q_scale,
+                               const float* k_scale, const void* vp, const int32_t* idx, void* op,
+                               float* lse, void* stream);
 
 /* Teacher tile map (row f3; the first stage of the Veda method: full attention,
  * max-pooled per tile pair, is the teacher distribution at tile level -- Veda

@@ -130,11 +130,12 @@ struct ItemInfo {
   int32_t rows_a, rows_b, end, bad;
 };
 
-template <int D>
+template <int D, bool F8 = false>
 struct Smem {
   static constexpr uint32_t kHalfBytes = 128 * 128;               // 128 rows x 128 B
-  static constexpr uint32_t kKBytes = (D / 64) * kHalfBytes;       // K tile pair (K-major)
-  static constexpr uint32_t kVBytes = kKBytes;                     // V tile pair (MN-major)
+  // K tile pair (K-major): D bf16 per row in D/64 128-byte halves, or (F8) D = 128 e4m3 bytes in one
+  static constexpr uint32_t kKBytes = F8 ? kHalfBytes : (D / 64) * kHalfBytes;
+  static constexpr uint32_t kVBytes = (D / 64) * kHalfBytes;       // V tile pair (MN-major, bf16)
   static constexpr int kKStages = VSA_K_STAGES;
   static constexpr int kVStages = VSA_V_STAGES;
   static constexpr uint32_t kQBytes = kKBytes;                     // the Q pair (K-major)
@@ -174,6 +175,8 @@ struct AttnParams {
   uint32_t* lists;         // [CTAs][2][list_cap] merged key lists (one slice per CTA)
   uint32_t* bitmaps;       // [CTAs][2][bitmap_words] scratch of the list builder
   float scale_log2;
+  const float* q_scale;    // fp8 Q K^T: [B, heads, nt_max] per-tile scales of Q and K (else null)
+  const float* k_scale;
   int32_t ntv[VSA_MAX_HEADS];
   int32_t k[VSA_MAX_HEADS];
   int32_t n_ref, k_ref_max;
@@ -191,12 +194,13 @@ __device__ __forceinline__ int warp_excl_scan(int v, int lane, int* total) {
   return x - v;
 }
 
-template <int D>
+template <int D, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv,
                 const __grid_constant__ AttnParams prm) {
-  using L = Smem<D>;
+  using L = Smem<D, F8>;
+  static_assert(!F8 || D == 128, "fp8 Q K^T: one 128-byte swizzle row per token");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -420,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row_base = inf.bh * prm.nt_max;
         if (is_k) {   // rows 0-63: tile qa, rows 64-127: tile qb (qa again when there is none)
           if (!wait_bar(bar(B_QEMPTY), (it & 1) ^ 1, abort_flag, gerr)) break;
-          mbar_expect_tx(bar(B_QFULL), 2 * (D / 64) * kTileBytes);
+          mbar_expect_tx(bar(B_QFULL), 2 * (F8 ? 1 : D / 64) * kTileBytes);
           const int qb = inf.qb >= 0 ? inf.qb : inf.qa;
-          for (int c = 0; c < D / 64; ++c) {
+          for (int c = 0; c < (F8 ? 1 : D / 64); ++c) {   // 64-row boxes of 128 bytes per row
             tma_load_2d(sbase + L::oQ + c * L::kHalfBytes, &tq, 64 * c, (row_base + inf.qa) * 64, bar(B_QFULL));
             tma_load_2d(sbase + L::oQ + c * L::kHalfBytes + 8192, &tq, 64 * c, (row_base + qb) * 64, bar(B_QFULL));
           }
@@ -434,10 +438,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int ta = int(list[2 * j] & 0xFFFFu);
           const int tb = 2 * j + 1 < inf.n_entries ? int(list[2 * j + 1] & 0xFFFFu) : ta;
           if (!(ok = wait_bar(bar(empty0 + st), ph ^ 1, abort_flag, gerr))) break;
-          mbar_expect_tx(bar(full0 + st), 2 * (D / 64) * kTileBytes);
-          if (is_k) {   // K-major: tile a rows 0-63, tile b rows 64-127 of each 64-column half
+          mbar_expect_tx(bar(full0 + st), 2 * (is_k && F8 ? 1 : D / 64) * kTileBytes);
+          if (is_k) {   // K-major: tile a rows 0-63, tile b rows 64-127 of each 128-byte half
             const uint32_t sk = sbase + L::oK + st * L::kKBytes;
-            for (int c = 0; c < D / 64; ++c) {
+            for (int c = 0; c < (F8 ? 1 : D / 64); ++c) {
               tma_load_2d(sk + c * L::kHalfBytes, map, 64 * c, (row_base + ta) * 64, bar(full0 + st));
               tma_load_2d(sk + c * L::kHalfBytes + 8192, map, 64 * c, (row_base + tb) * 64, bar(full0 + st));
             }
@@ -467,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------- S MMA ---
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idS = F8 ? idesc_e4m3(128, 128) : idesc_bf16(128, 128, 0, 0);
       // descriptors of the stage bases; a stage or k-step adds (byte offset >> 4)
       const uint64_t dq = sw128_desc(sbase + L::oQ, 16, 1024);
       const uint64_t dk0 = sw128_desc(sbase + L::oK, 16, 1024);
@@ -491,10 +495,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (su > 0 && !(ok = wait_bar(bar(B_PDONE0 + kSBuf + sb), (su - 1) & 1, abort_flag, gerr))) break;
           tc_fence_after();
           const uint64_t dk = dk0 + ((kst * L::kKBytes) >> 4);
+          if constexpr (F8) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {   // 16 channels per step
-            const uint32_t off = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
-            tc_mma(tS + sb * 128, dq + off, dk + off, idS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 32; ++kk) {   // 32 e4m3 channels (32 bytes) per step
+              const uint32_t off = (kk * 32) >> 4;
+              tc_mma_f8(tS + sb * 128, dq + off, dk + off, idS, kk > 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {   // 16 channels per step
+              const uint32_t off = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
+              tc_mma(tS + sb * 128, dq + off, dk + off, idS, kk > 0 ? 1u : 0u);
+            }
           }
           tc_commit(bar(B_SFULL0 + sb));
           tc_commit(bar(B_KEMPTY0 + kst));
@@ -579,7 +591,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tOw = tO0 + sg * 128 + lane_off;          // my warpgroup's O, my row
     float* xm = reinterpret_cast<float*>(smem + L::oXchg);   // [2 groups][128] row max
     float* xl = xm + 2 * 128;                               // [2 groups][128] row sums
-    const uint64_t c2 = f2pack(prm.scale_log2, prm.scale_log2);
+    // logit scale in log2 units; fp8 Q K^T also carries the tiles' dequantisation scales
+    float csc = prm.scale_log2;
+    uint64_t c2 = f2pack(csc, csc);
     uint32_t g = 0;
     bool ok = true;
     for (uint32_t it = 0; ok; ++it) {
@@ -625,7 +639,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mq[q] = fmaxf(t, sv[16 * q + 15]);
           }
           // raw scores; the scale is positive
-          const float bmx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * prm.scale_log2;
+          if constexpr (F8) {
+            // scale of my query tile (row-half) times the key tile's: fixed for this block
+            const int qtile = r < 64 ? inf.qa : inf.qb;
+            csc = prm.scale_log2 * prm.q_scale[size_t(inf.bh) * prm.nt_max + (qtile >= 0 ? qtile : inf.qa)] *
+                  prm.k_scale[size_t(inf.bh) * prm.nt_max + (e & 0xFFFFu)];
+            c2 = f2pack(csc, csc);
+          }
+          const float bmx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * csc;
           if (bmx > m + kLazy) {                   // also taken when m is still -inf
             alpha = m == -INFINITY ? 1.f : ex2(m - bmx);
             m = bmx;
@@ -760,18 +781,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 int attn_smem_bytes(int list_cap) {
   (void)list_cap;   // key lists live in global memory
-  static_assert(Smem<64>::oEnd <= Smem<128>::oEnd, "the d=64 layout fits the d=128 allocation");
+  static_assert(Smem<64>::oEnd <= Smem<128>::oEnd && Smem<128, true>::oEnd <= Smem<128>::oEnd,
+                "the d=64 and fp8 layouts fit the d=128 allocation");
   return 1024 + int(Smem<128>::oEnd);
 }
 
 cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp, const int32_t* idx,
-                        const int32_t* idx_ref, void* op, float* lse, cudaStream_t s) {
+                        const int32_t* idx_ref, void* op, float* lse, cudaStream_t s, const float* q_scale,
+                        const float* k_scale) {
   const Geometry& g = p->geo;
   const int64_t rows = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE;
+  const bool f8 = q_scale != nullptr;      // qp, kp are e4m3 tiles with per-tile scales
+  if (f8 && g.d != 128) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, qp, rows, g.d) || !make_map(&tk, kp, rows, g.d) || !make_map(&tv, vp, rows, g.d))
-    return cudaErrorInvalidValue;
+  const bool maps = f8 ? make_map_u8(&tq, qp, rows, g.d) && make_map_u8(&tk, kp, rows, g.d)
+                       : make_map(&tq, qp, rows, g.d) && make_map(&tk, kp, rows, g.d);
+  if (!maps || !make_map(&tv, vp, rows, g.d)) return cudaErrorInvalidValue;
   AttnParams prm;
+  prm.q_scale = q_scale;
+  prm.k_scale = k_scale;
   prm.idx = idx;
   prm.idx_ref = idx_ref;
   prm.ref_tiles = p->d_ref_tiles;
@@ -804,7 +832,11 @@ cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void*
   if (e != cudaSuccess) return e;
   const int smem = p->attn_smem_bytes;
   const int grid = int(p->n_items < p->num_sms ? p->n_items : p->num_sms);
-  if (g.d == 128) {
+  if (f8) {
+    e = cudaFuncSetAttribute(attn_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attn_kernel<128, true><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm);
+  } else if (g.d == 128) {
     e = cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attn_kernel<128><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm);

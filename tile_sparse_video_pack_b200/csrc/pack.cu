@@ -4,6 +4,7 @@
 // Tiling: Ref2VA VSA README ("two-tier attention layout": 4x4x4 video tiles,
 // segment-pure prefix tiles) and BSAI VedaSparse README ("Core Technology:
 // Head-Aware Tiling", per-head (pt, ph, pw) with product 64).
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -119,19 +120,28 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float (&x)[8]) {
 // tokens), then max and min for TripPool. The pooling itself is that of the
 // score stage (Ref2VA VSA README: mean-pooled Q, K for the gate score; BSAI
 // VedaSparse README "Core Technology: TripPool", eq. 5).
-template <int CPR, bool TRIP>
+//
+// QUANT: the same pass also writes Q and K of every packed tile as e4m3 (fp8)
+// with one fp32 scale per (tile, tensor): scale = the tile's largest
+// magnitude / 448 (1 for an all-zero tile), code = e4m3(x / scale), rounded
+// to nearest even and saturated (per-tile 8-bit Q K^T, as the tile-skipping
+// kernels on the Veda page run it).
+template <int CPR, bool TRIP, bool QUANT>
 __global__ void __launch_bounds__(256) pack_pool_kernel(Geometry g, const uint4* __restrict__ q,
                                                         const uint4* __restrict__ k,
                                                         const uint4* __restrict__ v, uint4* __restrict__ qp,
                                                         uint4* __restrict__ kp, uint4* __restrict__ vp,
                                                         const int32_t* __restrict__ counts,
-                                                        float* __restrict__ pq, float* __restrict__ pk) {
+                                                        float* __restrict__ pq, float* __restrict__ pk,
+                                                        uint2* __restrict__ qp8, uint2* __restrict__ kp8,
+                                                        float* __restrict__ q_scale, float* __restrict__ k_scale) {
   constexpr int D = CPR * 8;
   constexpr int KD = TRIP ? 3 * D : D;
   constexpr int RG = 256 / CPR;       // row groups: 16 (d = 128) or 32 (d = 64)
   constexpr int RPT = 64 / RG;        // rows per thread: 4 or 2
   constexpr int NS = TRIP ? 3 : 1;    // statistics: sum (, max, min)
   __shared__ float part[NS][2][8][D];
+  __shared__ float amax_part[2][8];
   const int64_t tile = blockIdx.x;    // bh * nt_max + n
   const int n = int(tile % g.nt_max);
   const int bh = int(tile / g.nt_max);
@@ -153,6 +163,7 @@ __global__ void __launch_bounds__(256) pack_pool_kernel(Geometry g, const uint4*
     }
   }
   const uint4 zero = make_uint4(0, 0, 0, 0);
+  uint4 keep_q[QUANT ? RPT : 1], keep_k[QUANT ? RPT : 1];   // this thread's Q, K chunks for the fp8 pass
 #pragma unroll
   for (int i = 0; i < RPT; ++i) {
     const int s = rg + RG * i;
@@ -168,6 +179,10 @@ __global__ void __launch_bounds__(256) pack_pool_kernel(Geometry g, const uint4*
     qp[dst] = a;
     kp[dst] = bb;
     vp[dst] = cc;
+    if constexpr (QUANT) {
+      keep_q[i] = a;
+      keep_k[i] = bb;
+    }
     if (pool && tok >= 0) {
       float xq[8], xk[8];
       bf16x8_to_f32(a, xq);
@@ -182,6 +197,64 @@ __global__ void __launch_bounds__(256) pack_pool_kernel(Geometry g, const uint4*
           st[NS - 1][0][e] = fminf(st[NS - 1][0][e], xq[e]);
           st[NS - 1][1][e] = fminf(st[NS - 1][1][e], xk[e]);
         }
+      }
+    }
+  }
+  if constexpr (QUANT) {
+    // the tile's largest magnitude of Q and of K, over every thread's rows
+    const int lane0 = threadIdx.x & 31, warp0 = threadIdx.x >> 5;
+    float am[2] = {0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+      float xq[8], xk[8];
+      bf16x8_to_f32(keep_q[i], xq);
+      bf16x8_to_f32(keep_k[i], xk);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        am[0] = fmaxf(am[0], fabsf(xq[e]));
+        am[1] = fmaxf(am[1], fabsf(xk[e]));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      am[0] = fmaxf(am[0], __shfl_xor_sync(0xffffffffu, am[0], o));
+      am[1] = fmaxf(am[1], __shfl_xor_sync(0xffffffffu, am[1], o));
+    }
+    if (lane0 == 0) {
+      amax_part[0][warp0] = am[0];
+      amax_part[1][warp0] = am[1];
+    }
+    __syncthreads();
+    float sc[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      float m = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) m = fmaxf(m, amax_part[t][w]);
+      sc[t] = m > 0.f ? __fdiv_rn(m, 448.0f) : 1.0f;
+    }
+    if (threadIdx.x == 0) {
+      q_scale[tile] = sc[0];
+      k_scale[tile] = sc[1];
+    }
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+      const int s = rg + RG * i;
+      const int64_t dst8 = (tile * VSA_TILE + s) * CPR + c;   // 8 bytes per 8 channels
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        float x[8];
+        bf16x8_to_f32(t ? keep_k[i] : keep_q[i], x);
+        uint32_t w[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+              make_float2(__fdiv_rn(x[4 * e], sc[t]), __fdiv_rn(x[4 * e + 1], sc[t])), __NV_SATFINITE, __NV_E4M3);
+          const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+              make_float2(__fdiv_rn(x[4 * e + 2], sc[t]), __fdiv_rn(x[4 * e + 3], sc[t])), __NV_SATFINITE, __NV_E4M3);
+          w[e] = uint32_t(lo) | (uint32_t(hi) << 16);
+        }
+        (t ? kp8 : qp8)[dst8] = make_uint2(w[0], w[1]);
       }
     }
   }
@@ -261,7 +334,8 @@ cudaError_t launch_pack(const vsa_plan* p, const void* q, const void* k, const v
 }
 
 cudaError_t launch_pack_pool(const vsa_plan* p, const void* q, const void* k, const void* v, void* qp,
-                             void* kp, void* vp, float* pooled_q, float* pooled_k, cudaStream_t s) {
+                             void* kp, void* vp, float* pooled_q, float* pooled_k, cudaStream_t s,
+                             void* qp8, void* kp8, float* q_scale, float* k_scale) {
   const Geometry& g = p->geo;
   const int64_t tiles = int64_t(g.B) * g.Hh * g.nt_max;
   const bool trip = p->desc.score_mode == VSA_SCORE_TRIPPOOL;
@@ -272,12 +346,30 @@ cudaError_t launch_pack_pool(const vsa_plan* p, const void* q, const void* k, co
   auto* kp4 = static_cast<uint4*>(kp);
   auto* vp4 = static_cast<uint4*>(vp);
   const int32_t* cnt = p->d_tile_count;
-  if (g.d == 128) {
-    if (trip) pack_pool_kernel<16, true><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k);
-    else pack_pool_kernel<16, false><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k);
+  auto* q8 = static_cast<uint2*>(qp8);
+  auto* k8 = static_cast<uint2*>(kp8);
+  if (qp8) {   // with the fp8 copies of Q and K (head_dim 128 only)
+    if (g.d != 128) return cudaErrorInvalidValue;
+    if (trip)
+      pack_pool_kernel<16, true, true><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k,
+                                                             q8, k8, q_scale, k_scale);
+    else
+      pack_pool_kernel<16, false, true><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k,
+                                                              q8, k8, q_scale, k_scale);
+  } else if (g.d == 128) {
+    if (trip)
+      pack_pool_kernel<16, true, false><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k,
+                                                              nullptr, nullptr, nullptr, nullptr);
+    else
+      pack_pool_kernel<16, false, false><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k,
+                                                               nullptr, nullptr, nullptr, nullptr);
   } else {
-    if (trip) pack_pool_kernel<8, true><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k);
-    else pack_pool_kernel<8, false><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k);
+    if (trip)
+      pack_pool_kernel<8, true, false><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k,
+                                                             nullptr, nullptr, nullptr, nullptr);
+    else
+      pack_pool_kernel<8, false, false><<<tiles, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4, cnt, pooled_q, pooled_k,
+                                                              nullptr, nullptr, nullptr, nullptr);
   }
   return cudaGetLastError();
 }

@@ -146,6 +146,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, 
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) |
          (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
+// Instruction descriptor, kind::f8f6f4: e4m3 A and B (format code 0), both K-major, fp32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+// A and B (8-bit) from shared memory; K = 32 per instruction.
+__device__ __forceinline__ void tc_mma_f8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
 
 
 // Bounded wait on an mbarrier phase. Returns false on timeout or when another
@@ -192,6 +203,19 @@ inline EncodeTiledFn get_encode() {
 }
 
 // Packed [rows, d] bf16 viewed as a 2D tensor; 64 x 64 boxes, 128-byte swizzle.
+// Packed [rows, d] e4m3 bytes (d = 128: one 128-byte row per token); 64-row boxes, 128-byte swizzle.
+inline bool make_map_u8(CUtensorMap* m, const void* base, int64_t rows, int d) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(d)};
+  cuuint32_t box[2] = {cuuint32_t(d), 64};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int d) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;

@@ -202,6 +202,7 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
   info.k_ref_max = g.k_ref_max;
   info.ref_score_elems = int64_t(g.B) * g.Hh * g.ntv_max * g.n_ref;
   info.ref_index_elems = int64_t(g.B) * g.Hh * g.ntv_max * g.k_ref_max;
+  info.tile_scale_elems = int64_t(g.B) * g.Hh * g.nt_max;
 
   // tile valid counts
   std::vector<int32_t> counts(size_t(g.Hh) * g.nt_max, 0);
@@ -333,6 +334,40 @@ vsa_status vsa_tile_pack_pool(vsa_plan* p, const void* q, const void* k, const v
   float *pq, *pk;
   vsa::score_pooled_ptrs(p, ws, &pq, &pk);
   if (vsa::launch_pack_pool(p, q, k, v, qp, kp, vp, pq, pk, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_tile_pack_pool_fp8(vsa_plan* p, const void* q, const void* k, const void* v, void* qp, void* kp,
+                                  void* vp, void* qp8, void* kp8, float* q_scale, float* k_scale, void* ws,
+                                  void* stream) {
+  if (!p || !q || !k || !v || !qp || !kp || !vp || !qp8 || !kp8 || !q_scale || !k_scale || !ws)
+    return fail(p, VSA_ERR_INVALID_ARG);
+  if (p->geo.d != 128) return fail(p, VSA_ERR_UNSUPPORTED);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qp) || !aligned16(kp) || !aligned16(vp) ||
+      !aligned16(qp8) || !aligned16(kp8) || !aligned16(q_scale) || !aligned16(k_scale) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_pack++;
+  float *pq, *pk;
+  vsa::score_pooled_ptrs(p, ws, &pq, &pk);
+  if (vsa::launch_pack_pool(p, q, k, v, qp, kp, vp, pq, pk, static_cast<cudaStream_t>(stream), qp8, kp8, q_scale,
+                            k_scale) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_sparse_attn_fp8(vsa_plan* p, const void* qp8, const void* kp8, const float* q_scale,
+                               const float* k_scale, const void* vp, const int32_t* idx, void* op, float* lse,
+                               void* stream) {
+  if (!p || !qp8 || !kp8 || !q_scale || !k_scale || !vp || !idx || !op) return fail(p, VSA_ERR_INVALID_ARG);
+  if (p->geo.d != 128) return fail(p, VSA_ERR_UNSUPPORTED);
+  if (!aligned16(qp8) || !aligned16(kp8) || !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(vp) ||
+      !aligned16(idx) || !aligned16(op) || (lse && !aligned16(lse)))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_attn++;
+  if (vsa::launch_attn(p, qp8, kp8, vp, idx, nullptr, op, lse, static_cast<cudaStream_t>(stream), q_scale,
+                       k_scale) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
   return VSA_OK;
 }

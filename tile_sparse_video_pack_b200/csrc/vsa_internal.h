@@ -67,8 +67,11 @@ namespace vsa {
 // Launchers (return cudaGetLastError()).
 cudaError_t launch_pack(const vsa_plan* p, const void* q, const void* k, const void* v, void* qp,
                         void* kp, void* vp, cudaStream_t s);
+// qp8 != null: also the e4m3 copies of Q and K and their per-tile scales (head_dim 128)
 cudaError_t launch_pack_pool(const vsa_plan* p, const void* q, const void* k, const void* v, void* qp,
-                             void* kp, void* vp, float* pooled_q, float* pooled_k, cudaStream_t s);
+                             void* kp, void* vp, float* pooled_q, float* pooled_k, cudaStream_t s,
+                             void* qp8 = nullptr, void* kp8 = nullptr, float* q_scale = nullptr,
+                             float* k_scale = nullptr);
 cudaError_t launch_unpack(const vsa_plan* p, const void* op, void* o, cudaStream_t s);
 cudaError_t launch_score(const vsa_plan* p, const void* qp, const void* kp, const float* proj_q,
                          const float* proj_k, float* scores, void* workspace, cudaStream_t s);
@@ -81,8 +84,10 @@ cudaError_t launch_topk(const vsa_plan* p, const float* scores, int32_t* idx, cu
 cudaError_t launch_topk_ref(const vsa_plan* p, const float* scores_ref, int32_t* idx_ref, cudaStream_t s);
 cudaError_t launch_ref_score(const vsa_plan* p, const void* kp, const float* proj_k, float* scores_ref,
                              void* workspace, cudaStream_t s);
+// q_scale != null: qp, kp are e4m3 tiles (head_dim 128) with per-tile scales q_scale, k_scale
 cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp,
-                        const int32_t* idx, const int32_t* idx_ref, void* op, float* lse, cudaStream_t s);
+                        const int32_t* idx, const int32_t* idx_ref, void* op, float* lse, cudaStream_t s,
+                        const float* q_scale = nullptr, const float* k_scale = nullptr);
 int attn_smem_bytes(int list_cap);
 cudaError_t launch_teacher(vsa_plan* p, const void* qp, const void* kp, const float* lse, float* teacher,
                            cudaStream_t s);

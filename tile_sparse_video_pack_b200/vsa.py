@@ -27,7 +27,8 @@ EXPORTS = ("vsa_plan_create", "vsa_plan_destroy", "vsa_plan_query", "vsa_plan_ge
            "vsa_tile_pack", "vsa_tile_score", "vsa_topk_select", "vsa_sparse_attn", "vsa_tile_unpack",
            "vsa_layer_forward", "vsa_plan_check", "vsa_status_string", "vsa_tile_score_static",
            "vsa_tile_pack_pool", "vsa_tile_score_pooled", "vsa_teacher_tiles", "vsa_index_overlap",
-           "vsa_ref_score", "vsa_topk_select_ref", "vsa_sparse_attn_ref")
+           "vsa_ref_score", "vsa_topk_select_ref", "vsa_sparse_attn_ref", "vsa_tile_pack_pool_fp8",
+           "vsa_sparse_attn_fp8")
 
 
 class VsaDesc(ctypes.Structure):
@@ -50,6 +51,7 @@ class VsaPlanInfo(ctypes.Structure):
         ("workspace_bytes", ctypes.c_int64), ("lse_elems", ctypes.c_int64), ("attn_work_items", ctypes.c_int64),
         ("n_ref_tiles", ctypes.c_int32), ("k_ref_max", ctypes.c_int32),
         ("ref_score_elems", ctypes.c_int64), ("ref_index_elems", ctypes.c_int64),
+        ("tile_scale_elems", ctypes.c_int64),
     ]
 
 
@@ -101,6 +103,8 @@ def library() -> ctypes.CDLL:
         "vsa_ref_score": (I32, [P] * 6),
         "vsa_topk_select_ref": (I32, [P] * 4),
         "vsa_sparse_attn_ref": (I32, [P] * 9),
+        "vsa_tile_pack_pool_fp8": (I32, [P] * 13),
+        "vsa_sparse_attn_fp8": (I32, [P] * 10),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -272,6 +276,40 @@ class Plan:
             _ptr(qp, bf, "qp", pe), _ptr(kp, bf, "kp", pe), _ptr(vp, bf, "vp", pe),
             _ptr(workspace, torch.uint8, "workspace", self.info.workspace_bytes), _stream(stream)),
             "vsa_tile_pack_pool")
+
+    def tile_pack_pool_fp8(self, q, k, v, qp, kp, vp, qp8, kp8, q_scale, k_scale, workspace, stream=None):
+        """tile_pack_pool plus e4m3 copies of Q and K with one fp32 scale per tile (head_dim 128)."""
+        import torch
+        n_tok = self.desc.batch * self.info.n_tokens * self.desc.heads * self.desc.head_dim
+        pe, bf, u8, f32 = self.info.packed_elems, torch.bfloat16, torch.uint8, torch.float32
+        ns = self.info.tile_scale_elems
+        _check(library().vsa_tile_pack_pool_fp8(
+            self._h, _ptr(q, bf, "q", n_tok), _ptr(k, bf, "k", n_tok), _ptr(v, bf, "v", n_tok),
+            _ptr(qp, bf, "qp", pe), _ptr(kp, bf, "kp", pe), _ptr(vp, bf, "vp", pe),
+            _ptr(qp8, u8, "qp8", pe), _ptr(kp8, u8, "kp8", pe), _ptr(q_scale, f32, "q_scale", ns),
+            _ptr(k_scale, f32, "k_scale", ns),
+            _ptr(workspace, u8, "workspace", self.info.workspace_bytes), _stream(stream)), "vsa_tile_pack_pool_fp8")
+
+    def sparse_attn_fp8(self, qp8, kp8, q_scale, k_scale, vp, idx, op, lse=None, stream=None):
+        """sparse_attn with Q K^T from the e4m3 tiles and their per-tile scales."""
+        import torch
+        pe, u8, f32, bf = self.info.packed_elems, torch.uint8, torch.float32, torch.bfloat16
+        ns = self.info.tile_scale_elems
+        _check(library().vsa_sparse_attn_fp8(
+            self._h, _ptr(qp8, u8, "qp8", pe), _ptr(kp8, u8, "kp8", pe), _ptr(q_scale, f32, "q_scale", ns),
+            _ptr(k_scale, f32, "k_scale", ns), _ptr(vp, bf, "vp", pe),
+            _ptr(idx, torch.int32, "idx", self.info.index_elems), _ptr(op, bf, "op", pe),
+            _ptr(lse, f32, "lse", self.info.lse_elems), _stream(stream)), "vsa_sparse_attn_fp8")
+
+    def allocate_fp8(self, device=None):
+        """The e4m3 Q, K tiles and their per-tile scales."""
+        import torch
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        pe, ns = self.info.packed_elems, self.info.tile_scale_elems
+        return {"qp8": torch.empty(pe, dtype=torch.uint8, device=dev),
+                "kp8": torch.empty(pe, dtype=torch.uint8, device=dev),
+                "q_scale": torch.empty(ns, dtype=torch.float32, device=dev),
+                "k_scale": torch.empty(ns, dtype=torch.float32, device=dev)}
 
     def tile_score_pooled(self, proj_q, proj_k, scores, workspace, stream=None):
         """Projection and scores from the descriptors tile_pack_pool left in the workspace."""

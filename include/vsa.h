@@ -274,9 +274,10 @@ VSA_API vsa_status vsa_sparse_attn_ref(vsa_plan* plan, const void* qp, const voi
  * 8-bit with per-tile scales). vsa_tile_pack_pool, and besides: Q and K of
  * every packed tile as e4m3 bytes qp8, kp8 ([B, heads, nt_max, 64, head_dim]
  * bytes, packed_elems of them) with one fp32 scale per (tile, tensor) in
- * q_scale, k_scale ([B, heads, nt_max], tile_scale_elems): scale = the tile's
- * largest magnitude / 448 (fp32 division; 1 for an all-zero tile), code =
- * e4m3(x / scale) (fp32 division, round to nearest even, saturating).
+ * q_scale, k_scale ([B, heads, nt_max], tile_scale_elems): with amax the
+ * tile's largest magnitude, code = e4m3(x * (448 / amax)) (fp32 product,
+ * round to nearest even, saturating) and scale = amax / 448 (fp32; 1 for an
+ * all-zero tile).
  * head_dim 128 only (VSA_ERR_UNSUPPORTED otherwise). */
 VSA_API vsa_status vsa_tile_pack_pool_fp8(vsa_plan* plan, const void* q, const void* k, const void* v,
                                   void* qp, void* kp, void* vp, void* qp8, void* kp8, float* q_scale,

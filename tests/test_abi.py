@@ -144,3 +144,17 @@ def test_null_arguments(lib):
     assert lib.vsa_sparse_attn(None, None, None, None, None, None, None, None) == 1
     assert lib.vsa_plan_check(None) == 1
     assert lib.vsa_plan_query(None, None) == 1
+
+
+def test_every_compute_call_rejects_a_null_plan(lib):
+    """A NULL plan (with every other pointer NULL) is an argument error, returned before any
+    CUDA call, for every entry point that takes a plan."""
+    ar = header_arity()
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    for name, n in ar.items():
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)", text)
+        first = m.group(1).split(",")[0]
+        if "vsa_plan*" not in first.replace(" ", "") or name in ("vsa_plan_destroy",):
+            continue
+        args = [None] * n
+        assert getattr(lib, name)(*args) == 1, name   # VSA_ERR_INVALID_ARG

@@ -34,10 +34,13 @@ def all_rows_valid(r):
     assert bool(torch.isfinite(r.out.float()).all())
 
 
-def sampled_parity(r, heads, n_video_samples=6, seed=0):
+def sampled_parity(r, heads, n_video_samples=6, seed=0, out=None, qk_fp8=False):
+    """Complete score rows and top-k sets of the sampled heads, and attention rows of sampled
+    query tiles against the oracle (``out``: another output of the same run to check instead,
+    ``qk_fp8``: against the oracle's fp8 model)."""
     rng = np.random.default_rng(seed)
     cfg = r.cfg
-    got_all = None
+    got_all = None if out is None else bf16_to_f64(out)
     for h in heads:
         sub, q, k, v, wq, wk = head_slice(cfg, r.inp, h)
         til = O.head_tiling(sub, 0)
@@ -47,8 +50,9 @@ def sampled_parity(r, heads, n_video_samples=6, seed=0):
         npre, nv = til.n_prefix, til.n_video
         qt = sorted({0, npre // 2, npre - 1} if npre else set())
         qt += sorted({npre, npre + 1, npre + nv - 1, *(npre + rng.integers(0, nv, n_video_samples))})
+        kept_ref = {0: r.ref_kept(0, h)} if r.plan.info.n_ref_tiles else None
         res = O.run_layer(sub, q, k, v, [r.k[h]], gate=r.inp.gate, w_q=wq, w_k=wk,
-                          query_tiles={0: qt}, kept={0: kept})
+                          query_tiles={0: qt}, kept={0: kept}, kept_ref=kept_ref, qk_fp8=qk_fp8)
         if got_all is None:
             got_all = bf16_to_f64(r.out)
         rows = np.concatenate([til.all[t] for t in qt])
@@ -58,7 +62,7 @@ def sampled_parity(r, heads, n_video_samples=6, seed=0):
 @pytest.mark.parametrize("sparsity", [0.75, 0.9])
 def test_full_clip(sparsity):
     cfg = get_config("full")
-    r = GpuRun(cfg, sparsity).run()
+    r = GpuRun(cfg, sparsity).run(fused=True)          # the bench's path: pack fused with pooling
     all_rows_valid(r)
     sampled_parity(r, heads=[0, 13])
     want_pairs = O.attention_flops(cfg, r.k) // (4 * cfg.head_dim)
@@ -68,7 +72,7 @@ def test_full_clip(sparsity):
 @pytest.mark.parametrize("sparsity", [0.9, 0.95])
 def test_veda_head_aware(sparsity):
     cfg = get_config("veda")
-    r = GpuRun(cfg, sparsity).run()
+    r = GpuRun(cfg, sparsity).run(fused=True)
     all_rows_valid(r)
     sampled_parity(r, heads=[0, 1, 2, 3])     # one head of each tile shape
 
@@ -77,7 +81,7 @@ def test_long_clip_dense_and_sparse():
     import torch
     import torch.nn.functional as F
     cfg = get_config("long")
-    r = GpuRun(cfg, 0.0).run()               # k = all tiles: dense attention
+    r = GpuRun(cfg, 0.0).run(fused=True)     # k = all tiles: dense attention
     all_rows_valid(r)
     sampled_parity(r, heads=[5], n_video_samples=3)
     # cross-check (not the oracle): torch dense attention on two heads
@@ -88,6 +92,38 @@ def test_long_clip_dense_and_sparse():
         got = r.out[:, :, h].unsqueeze(1).float()
         err = (got - ref).abs().max().item()
         assert err <= 2e-2, err
-    r2 = GpuRun(cfg, 0.9, inputs=r.inp).run()
+    r2 = GpuRun(cfg, 0.9, inputs=r.inp).run(fused=True)
     all_rows_valid(r2)
     sampled_parity(r2, heads=[3], n_video_samples=3)
+
+
+def test_full_clip_fp8():
+    """The fp8 Q K^T path at full size, against the oracle's fp8 model on sampled rows."""
+    import torch
+    cfg = get_config("full")
+    r = GpuRun(cfg, 0.75).run(fused=True)
+    f8 = r.plan.allocate_fp8()
+    b = r.bufs
+    r.plan.tile_pack_pool_fp8(r.q, r.k_t, r.v, b["qp"], b["kp"], b["vp"], f8["qp8"], f8["kp8"], f8["q_scale"],
+                              f8["k_scale"], b["workspace"])
+    op8 = torch.zeros_like(b["op"])
+    r.plan.sparse_attn_fp8(f8["qp8"], f8["kp8"], f8["q_scale"], f8["k_scale"], b["vp"], b["idx"], op8)
+    out8 = torch.empty_like(r.out)
+    r.plan.tile_unpack(op8, out8)
+    r.plan.check()
+    assert bool(torch.isfinite(out8.float()).all())
+    sampled_parity(r, heads=[7], out=out8, qk_fp8=True)
+
+
+def test_r2va_full_clip():
+    """R2VA budgets at full size: 32 of 60 reference tiles and 32 of 1680 video tiles."""
+    cfg = get_config("r2va").with_(heads=4, tile_shapes=get_config("r2va").tile_shapes[:4])
+    r = GpuRun(cfg, cfg.sparsity[0]).run(fused=True)
+    all_rows_valid(r)
+    for h in (0, 3):
+        sub, q, k, v, wq, wk = head_slice(cfg, r.inp, h)
+        til = O.head_tiling(sub, 0)
+        ref = O.ref_tiles(sub)
+        want = O.tile_scores(q[0, :, 0], k[0, :, 0], til, sub, 0, r.inp.gate, key_tiles=[til.prefix[t] for t in ref])
+        check_topk_rows(r.ref_kept(0, h), want, cfg.k_ref)
+    sampled_parity(r, heads=[0, 3], n_video_samples=4)

@@ -28,7 +28,7 @@ What it computes, in the order the pages give it:
 4. Exact softmax attention over the kept tiles only (BSAI VedaSparse README,
    "Core Technology: Tile-Skipping"; "Implementation": ``_veda_sparse``).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 * VSA score: S[i, j] = (qbar_i G) . (kbar_j G) / sqrt(d), one d x d gate G per
   layer shared by all heads; qbar/kbar are means over the tile's tokens.
 * TripPool score: S = (desc_q W_q[h]) . (desc_k W_k[h]) / sqrt(p), desc = [avg;

@@ -59,7 +59,7 @@ def bf16_to_f64(t) -> np.ndarray:
     return bf16_bits_to_f32(t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)).astype(np.float64)
 
 
-class GpuRun:
+class LayerRun:
     """Inputs of one config on the device plus every intermediate of one GPU layer run."""
 
     def __init__(self, cfg, sparsity, k_per_head=None, inputs=None):

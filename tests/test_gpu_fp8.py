@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 
 import oracle.vsa_oracle as O
-from gpu_util import GpuRun, bf16_to_f64, check_close, oracle_inputs_f64, ragged_gpu_config
+from gpu_util import LayerRun, bf16_to_f64, check_close, oracle_inputs_f64, ragged_gpu_config
 from vsa_synth import get_config
 
 pytestmark = pytest.mark.gpu
@@ -22,7 +22,7 @@ def run(name):
     import torch
     if name not in _runs:
         make, s = CASES[name]
-        r = GpuRun(make(), s).run(fused=True)
+        r = LayerRun(make(), s).run(fused=True)
         f8 = r.plan.allocate_fp8()
         b = r.bufs
         r.plan.tile_pack_pool_fp8(r.q, r.k_t, r.v, b["qp"], b["kp"], b["vp"], f8["qp8"], f8["kp8"],
@@ -70,7 +70,7 @@ def test_fp8_attention_matches_oracle_model(name):
 
 def test_fp8_needs_head_dim_128():
     import tile_sparse_video_pack_b200 as T
-    r = GpuRun(get_config("tiny"), 0.5).run(fused=True)
+    r = LayerRun(get_config("tiny"), 0.5).run(fused=True)
     f8 = r.plan.allocate_fp8()
     with pytest.raises(T.vsa.VsaError, match="UNSUPPORTED"):
         r.plan.sparse_attn_fp8(f8["qp8"], f8["kp8"], f8["q_scale"], f8["k_scale"], r.bufs["vp"], r.bufs["idx"],

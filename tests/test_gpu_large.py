@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 import oracle.vsa_oracle as O
-from gpu_util import (GpuRun, bf16_to_f64, check_close, check_topk_rows, n_video_tiles)
+from gpu_util import (LayerRun, bf16_to_f64, check_close, check_topk_rows, n_video_tiles)
 from vsa_synth import bf16_bits_to_f32, get_config
 
 pytestmark = pytest.mark.gpu
@@ -62,7 +62,7 @@ def sampled_parity(r, heads, n_video_samples=6, seed=0, out=None, qk_fp8=False):
 @pytest.mark.parametrize("sparsity", [0.75, 0.9])
 def test_full_clip(sparsity):
     cfg = get_config("full")
-    r = GpuRun(cfg, sparsity).run(fused=True)          # the bench's path: pack fused with pooling
+    r = LayerRun(cfg, sparsity).run(fused=True)          # the bench's path: pack fused with pooling
     all_rows_valid(r)
     sampled_parity(r, heads=[0, 13])
     want_pairs = O.attention_flops(cfg, r.k) // (4 * cfg.head_dim)
@@ -72,7 +72,7 @@ def test_full_clip(sparsity):
 @pytest.mark.parametrize("sparsity", [0.9, 0.95])
 def test_veda_head_aware(sparsity):
     cfg = get_config("veda")
-    r = GpuRun(cfg, sparsity).run(fused=True)
+    r = LayerRun(cfg, sparsity).run(fused=True)
     all_rows_valid(r)
     sampled_parity(r, heads=[0, 1, 2, 3])     # one head of each tile shape
 
@@ -81,7 +81,7 @@ def test_long_clip_dense_and_sparse():
     import torch
     import torch.nn.functional as F
     cfg = get_config("long")
-    r = GpuRun(cfg, 0.0).run(fused=True)     # k = all tiles: dense attention
+    r = LayerRun(cfg, 0.0).run(fused=True)     # k = all tiles: dense attention
     all_rows_valid(r)
     sampled_parity(r, heads=[5], n_video_samples=3)
     # cross-check (not the oracle): torch dense attention on two heads
@@ -92,7 +92,7 @@ def test_long_clip_dense_and_sparse():
         got = r.out[:, :, h].unsqueeze(1).float()
         err = (got - ref).abs().max().item()
         assert err <= 2e-2, err
-    r2 = GpuRun(cfg, 0.9, inputs=r.inp).run(fused=True)
+    r2 = LayerRun(cfg, 0.9, inputs=r.inp).run(fused=True)
     all_rows_valid(r2)
     sampled_parity(r2, heads=[3], n_video_samples=3)
 
@@ -101,7 +101,7 @@ def test_full_clip_fp8():
     """The fp8 Q K^T path at full size, against the oracle's fp8 model on sampled rows."""
     import torch
     cfg = get_config("full")
-    r = GpuRun(cfg, 0.75).run(fused=True)
+    r = LayerRun(cfg, 0.75).run(fused=True)
     f8 = r.plan.allocate_fp8()
     b = r.bufs
     r.plan.tile_pack_pool_fp8(r.q, r.k_t, r.v, b["qp"], b["kp"], b["vp"], f8["qp8"], f8["kp8"], f8["q_scale"],
@@ -118,7 +118,7 @@ def test_full_clip_fp8():
 def test_r2va_full_clip():
     """R2VA budgets at full size: 32 of 60 reference tiles and 32 of 1680 video tiles."""
     cfg = get_config("r2va").with_(heads=4, tile_shapes=get_config("r2va").tile_shapes[:4])
-    r = GpuRun(cfg, cfg.sparsity[0]).run(fused=True)
+    r = LayerRun(cfg, cfg.sparsity[0]).run(fused=True)
     all_rows_valid(r)
     for h in (0, 3):
         sub, q, k, v, wq, wk = head_slice(cfg, r.inp, h)

@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 
 import oracle.vsa_oracle as O
-from gpu_util import (GpuRun, bf16_to_f64, check_close, check_topk_rows, k_list, n_video_tiles,
+from gpu_util import (LayerRun, bf16_to_f64, check_close, check_topk_rows, k_list, n_video_tiles,
                       no_prefix_config, oracle_inputs_f64, ragged_gpu_config, scale_of, SCORE_REL, to_device)
 from vsa_synth import get_config
 
@@ -28,7 +28,7 @@ _runs = {}
 def gpu_run(name, fused=False):
     if (name, fused) not in _runs:
         make, s = CASES[name]
-        _runs[name, fused] = GpuRun(make(), s).run(fused=fused)
+        _runs[name, fused] = LayerRun(make(), s).run(fused=fused)
     return _runs[name, fused]
 
 
@@ -99,7 +99,7 @@ def test_attention_matches_oracle(name, fused):
 def test_dense_when_k_is_all(name):
     make, _ = CASES[name]
     cfg = make()
-    r = GpuRun(cfg, 0.0, k_per_head=[n_video_tiles(cfg, h) for h in range(cfg.heads)]).run()
+    r = LayerRun(cfg, 0.0, k_per_head=[n_video_tiles(cfg, h) for h in range(cfg.heads)]).run()
     q, k, v = oracle_inputs_f64(r.inp)
     want = O.dense_attention(q, k, v, scale_of(cfg))
     check_close(bf16_to_f64(r.out), want)
@@ -136,7 +136,7 @@ def test_pack_pool_descriptors_match_pool_stage(name):
 
 def test_k_one_and_edges():
     cfg = ragged_gpu_config(128, seed=23)
-    r = GpuRun(cfg, 1.0).run()          # k = 1 for every head
+    r = LayerRun(cfg, 1.0).run()          # k = 1 for every head
     assert r.k == [1] * cfg.heads
     q, k, v = oracle_inputs_f64(r.inp)
     kept = {h: r.kept(0, h) for h in range(cfg.heads)}
@@ -151,7 +151,7 @@ def test_k_one_and_edges():
 def test_bad_index_is_latched_not_read():
     import tile_sparse_video_pack_b200 as T
     import torch
-    r = GpuRun(get_config("tiny"), 0.5).run()
+    r = LayerRun(get_config("tiny"), 0.5).run()
     idx = r.bufs["idx"].clone()
     idx[0, 0, 1, 0] = 99                 # out of range
     op = torch.zeros_like(r.bufs["op"])
@@ -193,7 +193,7 @@ def test_running_max_jumps_late_in_the_row():
     n_last = cfg.H * cfg.W * 2                       # tokens of the last two frames
     k[:, -n_last:] *= 6.0
     inp = dataclasses.replace(inp, k=f32_to_bf16_bits(k).reshape(inp.k.shape))
-    r = GpuRun(cfg, 0.5, inputs=inp).run()
+    r = LayerRun(cfg, 0.5, inputs=inp).run()
     q, kk, v = oracle_inputs_f64(r.inp)
     kept = {(b, h): r.kept(b, h) for b in range(cfg.batch) for h in range(cfg.heads)}
     res = O.run_layer(cfg, q, kk, v, r.k, gate=r.inp.gate, w_q=r.inp.w_q, w_k=r.inp.w_k, kept=kept)

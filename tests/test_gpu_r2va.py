@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 
 import oracle.vsa_oracle as O
-from gpu_util import (GpuRun, SCORE_REL, bf16_to_f64, check_close, check_topk_rows, oracle_inputs_f64,
+from gpu_util import (LayerRun, SCORE_REL, bf16_to_f64, check_close, check_topk_rows, oracle_inputs_f64,
                       r2va_gpu_config)
 from vsa_synth import get_config
 
@@ -24,7 +24,7 @@ _runs = {}
 def run(name):
     if name not in _runs:
         make, s = CASES[name]
-        _runs[name] = GpuRun(make(), s).run(fused=True)
+        _runs[name] = LayerRun(make(), s).run(fused=True)
     return _runs[name]
 
 
@@ -70,7 +70,7 @@ def test_layer_forward_refuses_reference_plans():
 def test_bad_reference_index_is_latched():
     import torch
     import tile_sparse_video_pack_b200 as T
-    r = GpuRun(r2va_gpu_config(128), 0.5).run(fused=True)
+    r = LayerRun(r2va_gpu_config(128), 0.5).run(fused=True)
     b = r.bufs
     b["idx_ref"][0, 0, 0, :] = torch.tensor([1, 0], dtype=torch.int32)   # not ascending
     r.plan.sparse_attn_ref(b["qp"], b["kp"], b["vp"], b["idx"], b["idx_ref"], b["op"], b["lse"])

@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 import oracle.vsa_oracle as O
-from gpu_util import GpuRun, n_video_tiles, oracle_inputs_f64, ragged_gpu_config, scale_of
+from gpu_util import LayerRun, n_video_tiles, oracle_inputs_f64, ragged_gpu_config, scale_of
 from vsa_synth import get_config
 
 pytestmark = pytest.mark.gpu
@@ -27,8 +27,8 @@ def teacher_run(name):
     import torch
     make, s = CASES[name]
     cfg = make()
-    dense = GpuRun(cfg, 0.0, k_per_head=[n_video_tiles(cfg, h) for h in range(cfg.heads)]).run()
-    sparse = GpuRun(cfg, s, inputs=dense.inp).run()
+    dense = LayerRun(cfg, 0.0, k_per_head=[n_video_tiles(cfg, h) for h in range(cfg.heads)]).run()
+    sparse = LayerRun(cfg, s, inputs=dense.inp).run()
     teacher = torch.zeros_like(sparse.bufs["scores"])
     sparse.plan.teacher_tiles(dense.bufs["qp"], dense.bufs["kp"], dense.bufs["lse"], teacher)
     t_idx = torch.zeros_like(sparse.bufs["idx"])

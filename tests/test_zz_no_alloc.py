@@ -26,10 +26,10 @@ def _check_same(got, want, rel):
 
 def test_static_scratch_scores_match_workspace_scores_twice():
     import torch
-    from gpu_util import SCORE_REL, GpuRun
+    from gpu_util import SCORE_REL, LayerRun
     from vsa_synth import get_config
 
-    r = GpuRun(get_config("medium"), 0.75)
+    r = LayerRun(get_config("medium"), 0.75)
     b, p = r.bufs, r.plan
     p.tile_pack(r.q, r.k_t, r.v, b["qp"], b["kp"], b["vp"])
     p.check()

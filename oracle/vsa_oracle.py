@@ -408,19 +408,22 @@ def attention_flops(cfg, k_per_head) -> int:
     Mirrors the "Attention computed: X% of full attention" accounting of the
     Veda node (Veda news page, "Узел ComfyUI").
     """
+    ref = ref_tiles(cfg)
     total_pairs = 0
     for h in range(cfg.heads):
         til = head_tiling(cfg, h)
         n_pre_tok = sum(len(t) for t in til.prefix)
         n_all = cfg.n_tokens
         total_pairs += n_pre_tok * n_all
-        # every video tile keeps k tiles; their sizes depend on which tiles are
-        # kept only when tiles are partial, so this closed form needs full tiles
+        # every video tile keeps k tiles (and k_ref reference tiles); their sizes
+        # depend on which tiles are kept only when tiles are partial, so this
+        # closed form needs full tiles
         sizes = [len(t) for t in til.video]
-        if min(sizes) != TILE:
-            raise ValueError("closed-form count needs full video tiles")
+        if min(sizes) != TILE or any(len(til.prefix[r]) != TILE for r in ref):
+            raise ValueError("closed-form count needs full video and reference tiles")
+        seen_prefix = n_pre_tok - TILE * len(ref) + (TILE * int(cfg.k_ref) if len(ref) else 0)
         kh = int(k_per_head[h])
-        total_pairs += sum(sizes) * (n_pre_tok + kh * TILE)
+        total_pairs += sum(sizes) * (seen_prefix + kh * TILE)
     return 4 * cfg.head_dim * total_pairs * cfg.batch
 
 

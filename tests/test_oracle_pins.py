@@ -574,3 +574,22 @@ def test_fp8_attention_close_to_bf16_and_not_equal():
     d = np.abs(a.out - b.out)
     assert 0 < np.max(d) < 0.3 * np.max(np.abs(a.out))      # e4m3 keeps 3 mantissa bits
     assert all(np.array_equal(x, y) for x, y in zip(a.kept, b.kept))   # selection unchanged
+
+
+def test_flop_count_with_reference_budgets_matches_run():
+    """The closed-form count with reference budgets equals the pairs the tile loop computes
+    (full reference tiles: a 128-token reference segment)."""
+    cfg = ragged_config(batch=1).with_(name="r2va_full_tiles", segments=(100, 128, 30), seg_ref=(0, 1, 0),
+                                       k_ref=1, tile_shapes=((2, 4, 8),) * 4, seed=15)
+    inp, q, k, v = inputs_f64(cfg)
+    kk = k_list(cfg, 0.5)
+    res = O.run_layer(cfg, q, k, v, kk, gate=inp.gate)
+    assert O.attention_flops(cfg, kk) == 4 * cfg.head_dim * res.computed_pairs
+
+
+@pytest.mark.parametrize("name", ["full", "r2va", "long"])
+def test_bench_flop_count_is_the_oracle_count(name):
+    import bench
+    cfg = get_config(name)
+    ks = [O.k_from_sparsity(cfg.sparsity[-1], n_video_tiles(cfg, h)) for h in range(cfg.heads)]
+    assert bench.attention_flops(cfg, ks) == O.attention_flops(cfg, ks)

@@ -8,7 +8,9 @@
 * Closed forms: Q = 0 gives uniform weights; V = c gives c; a zero gate makes
   all scores tie so the k lowest tiles win; constant tiles pool to their
   constant; one-hot tiles fix which key tile wins and so the orientation of the
-  score matrix.
+  score matrix; tiles with known avg, max and min pools fix the exact TripPool
+  score matrices, and with them the descriptor's block order, which projection
+  goes with queries and which with keys, and each head's own weights.
 * The tile permutation matches a closed-form (tile, slot) formula.
 * Mutation tests plant plausible mistakes in the oracle and check that a pin
   catches each of them.
@@ -121,6 +123,11 @@ def pin_one_hot_orientation():
     res = O.run_layer(cfg, q, k, q.copy(), kk, gate=np.eye(16), query_tiles={})
     got = res.kept[0][:, 0]
     assert np.array_equal(got, (np.arange(8) - 3) % 8), got
+    # pooled features are exactly e_i and e_{(j+3) mod 8}: the scaled dot product over the
+    # 16 gate outputs is 1/sqrt(16) on the matching pair and 0 elsewhere
+    i = np.arange(8)[:, None]
+    j = np.arange(8)[None, :]
+    assert np.array_equal(res.scores[0], np.where(i == (j + 3) % 8, 0.25, 0.0))
 
 
 def pin_constant_tiles_pool(cfg):
@@ -135,6 +142,54 @@ def pin_constant_tiles_pool(cfg):
             assert np.allclose(O.mean_pool(x[tok]), (n + 1) / 2, rtol=0, atol=1e-14)
             tp = O.tripool(x[tok])
             assert np.allclose(tp, np.r_[[(n + 1) / 2] * 3, [n] * 3, [1] * 3], rtol=0, atol=1e-14)
+
+
+def pin_tripool_projection_orientation():
+    """TripPool scores on an 8-tile grid whose avg, max and min pools are all known.
+
+    Video query tile i: every token e_i, one token also 100 at coordinate
+    (i+1) mod 8, so avg = e_i + (100/64) e_{i+1}, max = e_i + 100 e_{i+1}, min = e_i.
+    Video key tile j: every token e_{(j+3) mod 8}, one token also 100 at (j+6) mod 8.
+    Head 0 projects the query's max block and the key's min block; head 1 the query's
+    min block and the key's max block (identity on the chosen block, zero elsewhere).
+    So S_0[i, j] = (1[j = i-3] + 100 * 1[j = i-2]) / 4 and
+    S_1[i, j] = (1[j = i-3] + 100 * 1[j = i-6]) / 4 (indices mod 8), exactly in fp64.
+    The block order of the descriptor, which projection goes with which side, and
+    which head's weights are used all change these matrices.
+    """
+    d = 16
+    cfg = LayerConfig(name="tp_onehot", batch=1, heads=2, head_dim=d, T=4, H=8, W=16,
+                      segments=(64,), tile_shapes=((4, 4, 4), (4, 4, 4)), score_mode="tripool",
+                      proj_dim=d, sparsity=(0.75,), seed=0)
+    q = np.zeros((1, cfg.n_tokens, 2, d))
+    k = np.zeros((1, cfg.n_tokens, 2, d))
+    for h in range(2):
+        for t, tok in enumerate(O.head_tiling(cfg, h).video):
+            q[0, tok, h, t] = 1.0
+            k[0, tok, h, (t + 3) % 8] = 1.0
+            first = min(tok)                               # one token of the tile
+            q[0, first, h, (t + 1) % 8] = 100.0
+            k[0, first, h, (t + 6) % 8] = 100.0
+
+    def block(b):                                          # identity on block b of [avg; max; min]
+        w = np.zeros((3 * d, d))
+        w[b * d:(b + 1) * d] = np.eye(d)
+        return w
+
+    AVG, MAX, MIN = 0, 1, 2
+    w_q = np.stack([block(MAX), block(MIN)])
+    w_k = np.stack([block(MIN), block(MAX)])
+    kk = [2, 2]
+    res = O.run_layer(cfg, q, k, q.copy(), kk, w_q=w_q, w_k=w_k, query_tiles={})
+    i = np.arange(8)[:, None]
+    j = np.arange(8)[None, :]
+    want0 = (np.where(j == (i - 3) % 8, 1.0, 0.0) + np.where(j == (i - 2) % 8, 100.0, 0.0)) / 4
+    want1 = (np.where(j == (i - 3) % 8, 1.0, 0.0) + np.where(j == (i - 6) % 8, 100.0, 0.0)) / 4
+    assert np.array_equal(res.scores[0], want0), res.scores[0]
+    assert np.array_equal(res.scores[1], want1), res.scores[1]
+    r = np.arange(8)
+    assert np.array_equal(res.kept[0], np.sort(np.stack([(r - 3) % 8, (r - 2) % 8], 1), 1))
+    assert np.array_equal(res.kept[1], np.sort(np.stack([(r - 3) % 8, (r - 6) % 8], 1), 1))
 
 
 # ---------------------------------------------------------------- tests -----
@@ -234,6 +289,10 @@ def test_one_hot_orientation():
 
 def test_constant_tiles_pool():
     pin_constant_tiles_pool(ragged_config(batch=1))
+
+
+def test_tripool_projection_orientation():
+    pin_tripool_projection_orientation()
 
 
 def test_permutation_closed_form():
@@ -346,6 +405,47 @@ def test_mutation_video_rows_lose_prefix(monkeypatch):
 def test_mutation_pool_over_64(monkeypatch):
     monkeypatch.setattr(O, "mean_pool", lambda x: x.sum(axis=0) / 64.0)
     _expect_pin_failure(pin_constant_tiles_pool, ragged_config(batch=1))
+
+
+def test_mutation_sum_pool_in_scores(monkeypatch):
+    monkeypatch.setattr(O, "mean_pool", lambda x: x.sum(axis=0))
+    _expect_pin_failure(pin_one_hot_orientation)
+
+
+@pytest.mark.parametrize("order", [(0, 2, 1), (1, 0, 2), (1, 2, 0), (2, 0, 1), (2, 1, 0)])
+def test_mutation_tripool_block_order(monkeypatch, order):
+    good = O.tripool
+
+    def bad(x):
+        d = x.shape[1]
+        parts = [good(x)[b * d:(b + 1) * d] for b in range(3)]
+        return np.concatenate([parts[b] for b in order])
+    monkeypatch.setattr(O, "tripool", bad)
+    _expect_pin_failure(pin_tripool_projection_orientation)
+
+
+def test_mutation_tripool_projections_swapped(monkeypatch):
+    good = O.tile_scores
+
+    def bad(q_h, k_h, til, cfg, h, gate=None, w_q=None, w_k=None, key_tiles=None):
+        return good(q_h, k_h, til, cfg, h, gate, w_k, w_q, key_tiles)
+    monkeypatch.setattr(O, "tile_scores", bad)
+    _expect_pin_failure(pin_tripool_projection_orientation)
+
+
+def test_mutation_tripool_first_head_weights(monkeypatch):
+    good = O.tile_scores
+
+    def bad(q_h, k_h, til, cfg, h, *a, **kw):
+        return good(q_h, k_h, til, cfg, 0, *a, **kw)
+    monkeypatch.setattr(O, "tile_scores", bad)
+    _expect_pin_failure(pin_tripool_projection_orientation)
+
+
+def test_mutation_unscaled_scores(monkeypatch):
+    good = O.tile_scores
+    monkeypatch.setattr(O, "tile_scores", lambda *a, **kw: 4.0 * good(*a, **kw))
+    _expect_pin_failure(pin_one_hot_orientation)
 
 
 # ------------------------------------------------ teacher map and recall ---
@@ -563,6 +663,66 @@ def test_fp8_attention_is_exact_on_representable_inputs():
     a = O.run_layer(cfg, q, k, v, kk, gate=inp.gate)
     b = O.run_layer(cfg, q, k, v, kk, gate=inp.gate, qk_fp8=True)
     assert np.array_equal(a.out, b.out)
+
+
+def pin_fp8_scales_are_per_tile():
+    """Tiles of different magnitudes: tile t holds c_t * v with c_t in {1, 3, 9}, v from
+    {0, +-0.5, +-1, +-1.25}, and its first token also +-1.75 c_t at channel 0 (the sign
+    alternates between tiles). Per tile the scale is c_t / 256 exactly and every entry maps
+    to 0, 128, 256, 320 or 448, all e4m3 values, so the fp8 layer equals the bf16 one bit for
+    bit. One scale for the whole tensor (a tile of c = 1 against 9/256: 0.5 maps to 14.2),
+    one per token (a row whose largest entry is 1.25: 1 maps to 358.4) or a signed maximum
+    (1.25 c_t in place of 1.75 c_t) leaves the e4m3 grid and changes the output."""
+    cfg = ragged_config(batch=1)
+    inp, q, k, v = inputs_f64(cfg)
+    rng = np.random.default_rng(8)
+    vals = [-1.25, -1.0, -0.5, 0.0, 0.5, 1.0, 1.25]
+    q = rng.choice(vals, size=q.shape)
+    k = rng.choice(vals, size=k.shape)
+    for h in range(cfg.heads):
+        for t, tok in enumerate(O.head_tiling(cfg, h).all):
+            c = 3.0 ** (t % 3)
+            sign = 1.0 if t % 2 == 0 else -1.0
+            for x in (q, k):
+                x[0, tok, h] *= c
+                x[0, tok[0], h, 0] = sign * 1.75 * c
+    kk = k_list(cfg, 0.5)
+    a = O.run_layer(cfg, q, k, v, kk, gate=inp.gate)
+    b = O.run_layer(cfg, q, k, v, kk, gate=inp.gate, qk_fp8=True)
+    assert np.array_equal(a.out, b.out), np.max(np.abs(a.out - b.out))
+
+
+def test_fp8_scales_are_per_tile():
+    pin_fp8_scales_are_per_tile()
+
+
+def test_mutation_fp8_one_scale_per_tensor(monkeypatch):
+    def bad(x_h, til):
+        codes, scale = O.quantize_tile_e4m3(np.asarray(x_h, dtype=np.float64))
+        return codes * scale
+    monkeypatch.setattr(O, "dequantized_tiles", bad)
+    _expect_pin_failure(pin_fp8_scales_are_per_tile)
+
+
+def test_mutation_fp8_one_scale_per_token(monkeypatch):
+    def bad(x_h, til):
+        out = np.array(x_h, dtype=np.float64)
+        for r in range(out.shape[0]):
+            codes, scale = O.quantize_tile_e4m3(out[r:r + 1])
+            out[r:r + 1] = codes * scale
+        return out
+    monkeypatch.setattr(O, "dequantized_tiles", bad)
+    _expect_pin_failure(pin_fp8_scales_are_per_tile)
+
+
+def test_mutation_fp8_signed_max(monkeypatch):
+    def bad(x):
+        xf = np.asarray(x, dtype=np.float32)
+        amax = np.float32(np.max(xf))
+        inv = np.float32(np.float32(O.E4M3_MAX) / amax)
+        return O.e4m3_round((xf * inv).astype(np.float64)), float(np.float32(amax / np.float32(O.E4M3_MAX)))
+    monkeypatch.setattr(O, "quantize_tile_e4m3", bad)
+    _expect_pin_failure(pin_fp8_scales_are_per_tile)
 
 
 def test_fp8_attention_close_to_bf16_and_not_equal():

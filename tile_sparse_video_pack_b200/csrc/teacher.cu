@@ -1,5 +1,5 @@
 // Teacher tile map and selection overlap (the Veda method's first stage and
-// the tile-recall figure it is judged by).
+// the tile-recall figure that measures a selection against it).
 //
 // What it computes (Veda news page, "Что делает Veda": full attention,
 // max-pooled per tile pair, is the teacher distribution at tile level; BSAI

@@ -124,6 +124,12 @@ BAD = {
     "score_mode": dict(score_mode=7),
     "tripool_proj": dict(score_mode="tripool", proj_dim=12),
     "scale": dict(softmax_scale=-1.0),
+    # R2VA budgets: segment 1 (64 tokens, one tile) may be marked as a reference stream
+    "seg_ref_value": dict(seg_ref=(0, 2), k_ref_per_head=(1, 1)),
+    "seg_ref_past_segments": dict(seg_ref=(0, 0, 1), k_ref_per_head=(1, 1)),
+    "k_ref_zero": dict(seg_ref=(0, 1), k_ref_per_head=(0, 1)),
+    "k_ref_too_big": dict(seg_ref=(0, 1), k_ref_per_head=(1, 2)),
+    "k_ref_without_reference": dict(k_ref_per_head=(1, 1)),
 }
 
 
@@ -133,6 +139,21 @@ def test_plan_rejects_bad_descriptor(lib, case):
     st = lib.vsa_plan_create(ctypes.byref(_desc(**BAD[case])), ctypes.byref(h))
     assert st == 1, (case, V.STATUS_NAMES.get(st))
     assert not h.value
+
+
+@pytest.mark.parametrize("over", [{}, dict(seg_ref=(0, 1), k_ref_per_head=(1, 1)),
+                                  dict(score_mode="tripool", proj_dim=16)])
+def test_plan_accepts_good_descriptor(lib, over):
+    """A valid descriptor passes host validation: with no GPU the create fails only at its
+    first CUDA call; with one it succeeds."""
+    h = ctypes.c_void_p()
+    st = lib.vsa_plan_create(ctypes.byref(_desc(**over)), ctypes.byref(h))
+    assert st in (0, 3, 6), V.STATUS_NAMES.get(st)      # OK, CUDA or NO_MEMORY, never INVALID_ARG
+    if st == 0:
+        assert h.value
+        assert lib.vsa_plan_destroy(h) == 0
+    else:
+        assert not h.value
 
 
 def test_null_arguments(lib):

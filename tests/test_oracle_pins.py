@@ -12,6 +12,8 @@
   score matrices, and with them the descriptor's block order, which projection
   goes with queries and which with keys, and each head's own weights.
 * The tile permutation matches a closed-form (tile, slot) formula.
+* A printed figure: the share of full attention the Veda node reports for its
+  1344x768 render at 90 % sparsity (tests/golden/veda_node_attention_share.txt).
 * Mutation tests plant plausible mistakes in the oracle and check that a pin
   catches each of them.
 """
@@ -361,6 +363,26 @@ def test_flop_count_matches_run():
     assert abs(f / dense - 0.3151) < 5e-4
 
 
+def pin_veda_node_attention_share():
+    """The share of full attention the Veda node reports for its 1344x768, 90 % render
+    (tests/golden/veda_node_attention_share.txt), from the oracle's count of computed
+    pairs (4 d per pair) over the dense count, rounded to one decimal as printed."""
+    with open(os.path.join(GOLDEN, "veda_node_attention_share.txt")) as f:
+        rows = [x.split() for x in f.read().splitlines() if x and not x.startswith("#")]
+    for T, H, W, text, s, computed, skipped in rows:
+        cfg = LayerConfig(name="veda_node", batch=1, heads=1, head_dim=128, T=int(T), H=int(H), W=int(W),
+                          segments=(int(text),), tile_shapes=((4, 4, 4),), score_mode="meanpool_gate",
+                          proj_dim=128, sparsity=(float(s),), seed=0)
+        kk = k_list(cfg, float(s))
+        share = 100.0 * O.attention_flops(cfg, kk) / (4 * cfg.head_dim * cfg.n_tokens ** 2)
+        assert f"{share:.1f}" == computed, share
+        assert f"{100.0 - share:.1f}" == skipped, share
+
+
+def test_veda_node_attention_share():
+    pin_veda_node_attention_share()
+
+
 # ------------------------------------------------------- planted mistakes ---
 
 def _expect_pin_failure(pin, *args):
@@ -446,6 +468,24 @@ def test_mutation_unscaled_scores(monkeypatch):
     good = O.tile_scores
     monkeypatch.setattr(O, "tile_scores", lambda *a, **kw: 4.0 * good(*a, **kw))
     _expect_pin_failure(pin_one_hot_orientation)
+
+
+def test_mutation_prefix_rows_sparse_in_count(monkeypatch):
+    """Counting prefix query rows like video rows (prefix keys plus k video tiles)
+    moves the share off the printed figure."""
+    def bad(cfg, k_per_head):
+        n_pre, n = cfg.n_prefix_tokens, cfg.n_tokens
+        return sum(4 * cfg.head_dim * n * (n_pre + 64 * kh) for kh in k_per_head)
+    monkeypatch.setattr(O, "attention_flops", bad)
+    _expect_pin_failure(pin_veda_node_attention_share)
+
+
+def test_mutation_video_rows_without_prefix_keys_in_count(monkeypatch):
+    def bad(cfg, k_per_head):
+        n_pre, nv, n = cfg.n_prefix_tokens, cfg.n_video_tokens, cfg.n_tokens
+        return sum(4 * cfg.head_dim * (n_pre * n + nv * 64 * kh) for kh in k_per_head)
+    monkeypatch.setattr(O, "attention_flops", bad)
+    _expect_pin_failure(pin_veda_node_attention_share)
 
 
 # ------------------------------------------------ teacher map and recall ---

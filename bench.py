@@ -34,6 +34,7 @@ if ROOT not in sys.path:
 
 CONFIG = "full"
 SECONDARY_SPARSITY = 0.9
+METRIC = "ms per attention layer at 107k video tokens, 75% video sparsity (90% in secondary); effective TFLOP/s"
 KERNELS_PER_STEP = 7  # pack + pool 1, score 3 (2 projections, scores), select 1, attention 1, unpack 1
 
 
@@ -135,6 +136,18 @@ def layer_bytes(cfg, ks):
     """Algorithmic HBM bytes of the element-wise stages (pack, pool, select, unpack)."""
     tok = cfg.batch * cfg.n_tokens * cfg.heads * cfg.head_dim * 2
     return {"pack": 2 * 3 * tok, "unpack": 2 * tok}
+
+
+def workload_config(cfg, sparsity, k0, world):
+    """The `config` object of the bench line, shared by both arms."""
+    ref = cfg.seg_ref and any(cfg.seg_ref)
+    return {"workload": f"{cfg.name}: one layer, B={cfg.batch}, {cfg.heads} heads, d={cfg.head_dim}, "
+                        f"grid {cfg.T}x{cfg.H}x{cfg.W} + prefix {list(cfg.segments)}, "
+                        f"{cfg.score_mode}, sparsity {sparsity} (k={k0})"
+                        + (f", reference segments {list(cfg.seg_ref)} with k_ref={cfg.k_ref}" if ref else ""),
+            "tokens": cfg.n_tokens, "heads": cfg.heads, "head_dim": cfg.head_dim, "k": k0,
+            "layers_per_step": world, "parallelism": f"independent layers x{world}",
+            "l2": "inputs larger than L2 (Q, K, V 691 MB each)"}
 
 
 # ------------------------------------------------------------------ clocks ----
@@ -505,18 +518,11 @@ def run_ours(args, rank, world, local_rank):
 
     value = job_ms_per_layer(ms_step, 1, world)
     line = {
-        "metric": "ms per attention layer at 107k video tokens, 75% video sparsity (90% in secondary); effective TFLOP/s",
+        "metric": METRIC,
         "value": round(value, 3), "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_step, 3), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{cfg.name}: one layer, B={cfg.batch}, {cfg.heads} heads, d={cfg.head_dim}, "
-                               f"grid {cfg.T}x{cfg.H}x{cfg.W} + prefix {list(cfg.segments)}, "
-                               f"{cfg.score_mode}, sparsity {args.sparsity} (k={ks[0]})"
-                               + (f", reference segments {list(cfg.seg_ref)} with k_ref={cfg.k_ref}"
-                                  if cfg.seg_ref and any(cfg.seg_ref) else ""),
-                   "tokens": cfg.n_tokens, "heads": cfg.heads, "head_dim": cfg.head_dim, "k": ks[0],
-                   "layers_per_step": world, "parallelism": f"independent layers x{world}",
-                   "l2": "inputs larger than L2 (Q, K, V 691 MB each)"},
+        "config": workload_config(cfg, args.sparsity, ks[0], world),
         "stages_ms": {a: round(b, 3) for a, b in stages.items()},
         "effective_tflops": {"attn_kernel": round(achieved, 1),
                              "layer": round(flops / (ms_step * 1e-3) / 1e12, 1)},
@@ -541,8 +547,13 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
+        import oracle.vsa_oracle as O
         from vsa_synth import get_config
         cfg = get_config(args.config)
+        if args.heads:
+            cfg = cfg.with_(heads=args.heads, tile_shapes=cfg.tile_shapes[:args.heads])
+        pt, ph, pw = cfg.tile_shapes[0]
+        k0 = O.k_from_sparsity(args.sparsity, -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw))
         sampler = OracleSample(cfg, args.sparsity)
         per_step = max(2.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
         vals = []
@@ -554,11 +565,11 @@ def main():
             last = sampler.run(per_step)
             vals.append(last["value"])
         v = statistics.median(vals)
-        line = {"impl": "reference", "metric": "ms per attention layer at 107k video tokens, 75% video sparsity",
-                "value": v, "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        line = {"impl": "reference", "metric": METRIC,
+                "value": v, "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": v, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f64", "data": "synthetic",
-                "config": {"workload": f"{cfg.name}: one layer, sparsity {args.sparsity}", "tokens": cfg.n_tokens},
+                "config": workload_config(cfg, args.sparsity, k0, world),
                 "cpu_baseline": {**last, "value": v},
                 "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
                 "wall_s": round(time.time() - t0, 1)}

@@ -81,7 +81,7 @@ typedef struct {
   int32_t k_per_head[VSA_MAX_HEADS];    /* kept video key tiles per video query tile,
                                            1 .. number of video tiles of that head */
   int32_t score_mode;                   /* vsa_score_mode */
-  int32_t proj_dim;                     /* mean-pool gate: == head_dim; TripPool: 16..128, %16 == 0 */
+  int32_t proj_dim;                     /* mean-pool gate: == head_dim; TripPool: 8..256, a multiple of 8 */
   float softmax_scale;                  /* 0 -> 1/sqrt(head_dim) */
   /* R2VA budget variant (BSAI VedaSparse README, v3.4.2 notes on the R2VA
    * predictor: per query, 32 reference tiles and 32 video tiles; text / VLM /

@@ -123,6 +123,8 @@ BAD = {
     "proj": dict(proj_dim=32),
     "score_mode": dict(score_mode=7),
     "tripool_proj": dict(score_mode="tripool", proj_dim=12),
+    "tripool_proj_small": dict(score_mode="tripool", proj_dim=4),
+    "tripool_proj_big": dict(score_mode="tripool", proj_dim=264),
     "scale": dict(softmax_scale=-1.0),
     # R2VA budgets: segment 1 (64 tokens, one tile) may be marked as a reference stream
     "seg_ref_value": dict(seg_ref=(0, 2), k_ref_per_head=(1, 1)),
@@ -142,7 +144,8 @@ def test_plan_rejects_bad_descriptor(lib, case):
 
 
 @pytest.mark.parametrize("over", [{}, dict(seg_ref=(0, 1), k_ref_per_head=(1, 1)),
-                                  dict(score_mode="tripool", proj_dim=16)])
+                                  dict(score_mode="tripool", proj_dim=8),
+                                  dict(score_mode="tripool", proj_dim=256)])
 def test_plan_accepts_good_descriptor(lib, over):
     """A valid descriptor passes host validation: with no GPU the create fails only at its
     first CUDA call; with one it succeeds."""

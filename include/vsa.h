@@ -30,6 +30,10 @@
  *    There is no CPU path and no fallback kernel.
  *  - A plan may be used by one stream at a time; calls on the same plan that
  *    overlap on the GPU share the attention kernel's work counter and race.
+ *  - A plan belongs to the device that was current when it was created. Every
+ *    call that launches work, and vsa_plan_check(), must be made with that
+ *    device current; otherwise it returns VSA_ERR_INVALID_ARG and launches
+ *    nothing.
  */
 #ifndef VSA_H_
 #define VSA_H_
@@ -136,7 +140,8 @@ typedef struct {
  * VSA_ERR_CUDA / VSA_ERR_NO_MEMORY for device failures. */
 VSA_API vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out);
 
-/* Frees the plan's device tables. Synchronises the device first. NULL is OK. */
+/* Frees the plan's device tables. Synchronises the plan's device first (making
+ * it current for the call and restoring the caller's device after). NULL is OK. */
 VSA_API vsa_status vsa_plan_destroy(vsa_plan* plan);
 
 VSA_API vsa_status vsa_plan_query(const vsa_plan* plan, vsa_plan_info* out);

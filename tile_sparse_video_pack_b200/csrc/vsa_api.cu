@@ -24,6 +24,17 @@ vsa_status fail(vsa_plan* p, vsa_status s) {
   return s;
 }
 
+// Work is launched on the current device; a plan's tables live on the device
+// that was current when it was created, so the two must agree.
+bool on_plan_device(const vsa_plan* p) {
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return cur == p->device;
+}
+
 // Host-side validation of a descriptor; no CUDA call is made here.
 vsa_status validate(const vsa_desc& d) {
   if (d.batch < 1 || d.heads < 1 || d.heads > VSA_MAX_HEADS) return VSA_ERR_INVALID_ARG;
@@ -277,12 +288,20 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
 
 vsa_status vsa_plan_destroy(vsa_plan* p) {
   if (!p) return VSA_OK;
-  if (p->d_tile_count || p->d_items || p->d_state || p->d_lists || p->d_ref_tiles) cudaDeviceSynchronize();
-  if (p->d_tile_count) cudaFree(p->d_tile_count);
-  if (p->d_ref_tiles) cudaFree(p->d_ref_tiles);
-  if (p->d_items) cudaFree(p->d_items);
-  if (p->d_state) cudaFree(p->d_state);
-  if (p->d_lists) cudaFree(p->d_lists);
+  if (p->d_tile_count || p->d_items || p->d_state || p->d_lists || p->d_ref_tiles) {
+    // wait for the plan's own device, then put the caller's current device back
+    int cur = -1;
+    const bool switch_dev = cudaGetDevice(&cur) == cudaSuccess && cur != p->device;
+    if (switch_dev) cudaSetDevice(p->device);
+    cudaDeviceSynchronize();
+    if (p->d_tile_count) cudaFree(p->d_tile_count);
+    if (p->d_ref_tiles) cudaFree(p->d_ref_tiles);
+    if (p->d_items) cudaFree(p->d_items);
+    if (p->d_state) cudaFree(p->d_state);
+    if (p->d_lists) cudaFree(p->d_lists);
+    if (switch_dev) cudaSetDevice(cur);
+    cudaGetLastError();
+  }
   delete p;
   return VSA_OK;
 }
@@ -318,6 +337,7 @@ vsa_status vsa_tile_pack(vsa_plan* p, const void* q, const void* k, const void* 
     ++n;
   }
   if (n == 0) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_pack++;
   if (vsa::launch_pack(p, q, k, v, qp, kp, vp, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
@@ -330,6 +350,7 @@ vsa_status vsa_tile_pack_pool(vsa_plan* p, const void* q, const void* k, const v
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qp) || !aligned16(kp) || !aligned16(vp) ||
       (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_pack++;
   float *pq, *pk;
   vsa::score_pooled_ptrs(p, ws, &pq, &pk);
@@ -348,6 +369,7 @@ vsa_status vsa_tile_pack_pool_fp8(vsa_plan* p, const void* q, const void* k, con
       !aligned16(qp8) || !aligned16(kp8) || !aligned16(q_scale) || !aligned16(k_scale) ||
       (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_pack++;
   float *pq, *pk;
   vsa::score_pooled_ptrs(p, ws, &pq, &pk);
@@ -365,6 +387,7 @@ vsa_status vsa_sparse_attn_fp8(vsa_plan* p, const void* qp8, const void* kp8, co
   if (!aligned16(qp8) || !aligned16(kp8) || !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(vp) ||
       !aligned16(idx) || !aligned16(op) || (lse && !aligned16(lse)))
     return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_attn++;
   if (vsa::launch_attn(p, qp8, kp8, vp, idx, nullptr, op, lse, static_cast<cudaStream_t>(stream), q_scale,
                        k_scale) != cudaSuccess)
@@ -377,6 +400,7 @@ vsa_status vsa_tile_score_pooled(vsa_plan* p, const float* proj_q, const float* 
   if (!p || !proj_q || !proj_k || !scores || !ws) return fail(p, VSA_ERR_INVALID_ARG);
   if (!aligned16(proj_q) || !aligned16(proj_k) || !aligned16(scores) || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_score++;
   if (vsa::launch_project_score(p, proj_q, proj_k, scores, ws, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
@@ -385,6 +409,7 @@ vsa_status vsa_tile_score_pooled(vsa_plan* p, const float* proj_q, const float* 
 
 vsa_status vsa_tile_unpack(vsa_plan* p, const void* op, void* o, void* stream) {
   if (!p || !op || !o || !aligned16(op) || !aligned16(o)) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_unpack++;
   if (vsa::launch_unpack(p, op, o, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
@@ -397,6 +422,7 @@ vsa_status vsa_tile_score(vsa_plan* p, const void* qp, const void* kp, const flo
   if (!aligned16(qp) || !aligned16(kp) || !aligned16(proj_q) || !aligned16(proj_k) ||
       !aligned16(scores) || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_score++;
   if (vsa::launch_score(p, qp, kp, proj_q, proj_k, scores, ws, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
@@ -406,6 +432,7 @@ vsa_status vsa_tile_score(vsa_plan* p, const void* qp, const void* kp, const flo
 
 vsa_status vsa_topk_select(vsa_plan* p, const float* scores, int32_t* idx, void* stream) {
   if (!p || !scores || !idx || !aligned16(scores) || !aligned16(idx)) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_select++;
   if (vsa::launch_topk(p, scores, idx, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
@@ -418,6 +445,7 @@ vsa_status vsa_sparse_attn(vsa_plan* p, const void* qp, const void* kp, const vo
   if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(idx) || !aligned16(op) ||
       (lse && !aligned16(lse)))
     return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_attn++;
   if (vsa::launch_attn(p, qp, kp, vp, idx, nullptr, op, lse, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
@@ -430,6 +458,7 @@ vsa_status vsa_ref_score(vsa_plan* p, const void* kp, const float* proj_k, float
   if (p->geo.n_ref == 0) return fail(p, VSA_ERR_INVALID_ARG);
   if (!aligned16(kp) || !aligned16(proj_k) || !aligned16(scores_ref) || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_score++;
   if (vsa::launch_ref_score(p, kp, proj_k, scores_ref, ws, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
@@ -439,6 +468,7 @@ vsa_status vsa_ref_score(vsa_plan* p, const void* kp, const float* proj_k, float
 vsa_status vsa_topk_select_ref(vsa_plan* p, const float* scores_ref, int32_t* idx_ref, void* stream) {
   if (!p || !scores_ref || !idx_ref || p->geo.n_ref == 0 || !aligned16(scores_ref) || !aligned16(idx_ref))
     return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_select++;
   if (vsa::launch_topk_ref(p, scores_ref, idx_ref, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
@@ -451,6 +481,7 @@ vsa_status vsa_sparse_attn_ref(vsa_plan* p, const void* qp, const void* kp, cons
   if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(idx) || !aligned16(idx_ref) ||
       !aligned16(op) || (lse && !aligned16(lse)))
     return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_attn++;
   if (vsa::launch_attn(p, qp, kp, vp, idx, idx_ref, op, lse, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
@@ -475,6 +506,7 @@ vsa_status vsa_teacher_tiles(vsa_plan* p, const void* qp, const void* kp, const 
   if (!p || !qp || !kp || !lse || !teacher || !aligned16(qp) || !aligned16(kp) || !aligned16(lse) ||
       !aligned16(teacher))
     return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   if (vsa::launch_teacher(p, qp, kp, lse, teacher, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
   return VSA_OK;
@@ -484,6 +516,7 @@ vsa_status vsa_index_overlap(vsa_plan* p, const int32_t* idx_a, const int32_t* i
                              void* stream) {
   if (!p || !idx_a || !idx_b || !counts || !aligned16(idx_a) || !aligned16(idx_b) || !aligned16(counts))
     return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   if (vsa::launch_overlap(p, idx_a, idx_b, counts, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
   return VSA_OK;
@@ -491,6 +524,7 @@ vsa_status vsa_index_overlap(vsa_plan* p, const int32_t* idx_a, const int32_t* i
 
 vsa_status vsa_plan_check(vsa_plan* p) {
   if (!p) return VSA_ERR_INVALID_ARG;
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return fail(p, VSA_ERR_CUDA);
   uint32_t err = 0;

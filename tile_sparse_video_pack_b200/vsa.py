@@ -154,6 +154,9 @@ def _ptr(t, dtype, name, min_numel=0):
     import torch
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        # the library launches on the current device, which must also be the plan's
+        raise ValueError(f"{name} is on {t.device}, but cuda:{torch.cuda.current_device()} is the current device")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():

@@ -651,6 +651,47 @@ def test_r2va_zero_gate_keeps_lowest_reference_tiles():
         assert np.all(res.ref_kept[h] == np.array([0, 1]))
 
 
+def pin_r2va_reference_orientation():
+    """Reference tiles are described by their K rows, like video key tiles. Video query
+    tile i pools (Q) to e_i; reference tile r holds K = e_{2r} and, as a decoy, Q = e_{2r+1}.
+    With the identity gate and k_ref = 1, even query tiles keep reference tile i/2 (score
+    1/sqrt(16)) and odd ones see only zeros and keep tile 0 by the tie rule; pooling the
+    reference tiles' Q would swap the two cases."""
+    d = 16
+    cfg = LayerConfig(name="r2va_onehot", batch=1, heads=1, head_dim=d, T=4, H=8, W=16,
+                      segments=(64, 256, 64), tile_shapes=((4, 4, 4),), score_mode="meanpool_gate",
+                      proj_dim=d, sparsity=(0.5,), seed=0, seg_ref=(0, 1, 0), k_ref=1)
+    til = O.head_tiling(cfg, 0)
+    ref = O.ref_tiles(cfg)
+    assert list(ref) == [1, 2, 3, 4]
+    q = np.zeros((1, cfg.n_tokens, 1, d))
+    k = np.zeros((1, cfg.n_tokens, 1, d))
+    for i, tok in enumerate(til.video):
+        q[0, tok, 0, i] = 1.0
+    for r, t in enumerate(ref):
+        k[0, til.prefix[t], 0, 2 * r] = 1.0
+        q[0, til.prefix[t], 0, 2 * r + 1] = 1.0
+    res = O.run_layer(cfg, q, k, q.copy(), [4], gate=np.eye(d), query_tiles={})
+    want = np.array([[i // 2] if i % 2 == 0 else [0] for i in range(8)])
+    assert np.array_equal(res.ref_kept[0], want), res.ref_kept[0]
+    i = np.arange(8)[:, None]
+    r = np.arange(4)[None, :]
+    assert np.array_equal(res.ref_scores[0], np.where(i == 2 * r, 0.25, 0.0))
+
+
+def test_r2va_reference_orientation():
+    pin_r2va_reference_orientation()
+
+
+def test_mutation_r2va_reference_tiles_pooled_from_q(monkeypatch):
+    good = O.tile_scores
+
+    def bad(q_h, k_h, til, cfg, h, gate=None, w_q=None, w_k=None, key_tiles=None):
+        return good(q_h, q_h if key_tiles is not None else k_h, til, cfg, h, gate, w_q, w_k, key_tiles)
+    monkeypatch.setattr(O, "tile_scores", bad)
+    _expect_pin_failure(pin_r2va_reference_orientation)
+
+
 def test_mutation_r2va_drops_reference_tiles(monkeypatch):
     good = O.query_key_tokens
     monkeypatch.setattr(O, "query_key_tokens",

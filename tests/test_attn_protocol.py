@@ -17,7 +17,7 @@ def test_valid_items_never_deadlock_or_race():
 
 
 def test_items_without_key_blocks_can_alias_the_list_slot():
-    """Known issue in the kernel as built: with an item that has no key blocks (only a rejected
+    """Known issue in the current kernel: with an item that has no key blocks (only a rejected
     item on a layer without prefix tiles), the list slot can be refilled twice before the S
     issuer has seen it; its parity wait then never passes (the kernel's bounded wait times out).
     Starving the S issuer and the V producer shows it deterministically."""

@@ -150,6 +150,51 @@ def workload_config(cfg, sparsity, k0, world):
             "l2": "inputs larger than L2 (Q, K, V 691 MB each)"}
 
 
+def attn_roofline(args, cfg, peaks, flops, attn_ms):
+    """The `roofline` object for the attention kernel from its event-timed mean duration."""
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    # fp8: Q K^T (half the FLOPs) at the e4m3 rate, twice bf16's (nominal ratio), P V at bf16, so the
+    # mixed peak is 1 / (0.5 / 2 + 0.5 / 1) = 4/3 of the measured bf16 peak
+    mix = 4.0 / 3.0 if args.fp8 else 1.0
+    peak = round(peaks["bf16_tflops_sustained"] * mix, 1)
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": None if args.fp8 else measured_traffic(args.config, args.sparsity, cfg.heads),
+            "kernel": "attn_kernel<128, fp8> (vsa_sparse_attn_fp8; e4m3 Q K^T, bf16 P V)" if args.fp8
+                      else "attn_kernel (vsa_sparse_attn)",
+            "peak_kind": (f"half e4m3 (2x bf16, nominal ratio), half bf16: 4/3 x bf16 dense, sustained, "
+                          f"{peaks['source']}") if args.fp8 else f"bf16 dense, sustained, {peaks['source']}",
+            "frac_of_burst_peak": round(achieved / (peaks["bf16_tflops"] * mix), 4),
+            "algorithmic_flops_per_launch": flops}
+
+
+def bench_line(args, cfg, world, ks, flops, ms_step, stages, roofline, e2e, clocks, stats, secondary,
+               teacher=None):
+    """The JSON line of the CUDA arm (rank 0 prints it)."""
+    ref = cfg.seg_ref and any(cfg.seg_ref)
+    line = {
+        "metric": METRIC,
+        "value": round(job_ms_per_layer(ms_step, 1, world), 3), "unit": "ms", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(cfg, args.sparsity, ks[0], world),
+        "stages_ms": {a: round(b, 3) for a, b in stages.items()},
+        "effective_tflops": {"attn_kernel": roofline["achieved"],
+                             "layer": round(flops / (ms_step * 1e-3) / 1e12, 1)},
+        "score_select_share": round((stages["score"] + stages["select"]) / sum(stages.values()), 4),
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": (KERNELS_PER_STEP + (4 if ref else 0)) * args.steps,
+        "clocks": clocks,
+        "attention_computed_pct": round(100.0 * stats["computed_pairs"] / stats["dense_pairs"], 2),
+        "secondary": secondary,
+    }
+    if teacher is not None:
+        line["teacher"] = teacher
+    return line
+
+
 # ------------------------------------------------------------------ clocks ----
 
 class ClockSampler:
@@ -489,21 +534,7 @@ def run_ours(args, rank, world, local_rank):
     ks = k_list(cfg, args.sparsity)
     layer, out, ms_step, stages, clocks, stats = timed_layer(args.sparsity, args.steps, args.warmup, True)
     flops = attention_flops(cfg, ks)
-    attn_ms = max_over_ranks(stages["attn"])
-    achieved = flops / (attn_ms * 1e-3) / 1e12
-    # fp8: Q K^T (half the FLOPs) at the e4m3 rate, twice bf16's (nominal ratio), P V at bf16, so the
-    # mixed peak is 1 / (0.5 / 2 + 0.5 / 1) = 4/3 of the measured bf16 peak
-    mix = 4.0 / 3.0 if args.fp8 else 1.0
-    peak = round(peaks["bf16_tflops_sustained"] * mix, 1)
-    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4),
-                "traffic": None if args.fp8 else measured_traffic(args.config, args.sparsity, cfg.heads),
-                "kernel": "attn_kernel<128, fp8> (vsa_sparse_attn_fp8; e4m3 Q K^T, bf16 P V)" if args.fp8
-                          else "attn_kernel (vsa_sparse_attn)",
-                "peak_kind": (f"half e4m3 (2x bf16, nominal ratio), half bf16: 4/3 x bf16 dense, sustained, "
-                              f"{peaks['source']}") if args.fp8 else f"bf16 dense, sustained, {peaks['source']}",
-                "frac_of_burst_peak": round(achieved / (peaks["bf16_tflops"] * mix), 4),
-                "algorithmic_flops_per_launch": flops}
+    roofline = attn_roofline(args, cfg, peaks, flops, max_over_ranks(stages["attn"]))
 
     # end to end through host buffers: pinned H2D of q, k, v, the layer, D2H of o
     e2e = None if args.no_e2e else e2e_measure(args, layer, q, k, v, out, stream, world, barrier, max_over_ranks)
@@ -519,28 +550,8 @@ def run_ours(args, rank, world, local_rank):
                      "layer_tflops": round(f2 / (ms2 * 1e-3) / 1e12, 1)}
 
     teacher = teacher_measure(layer, ks) if args.teacher else None
-
-    value = job_ms_per_layer(ms_step, 1, world)
-    line = {
-        "metric": METRIC,
-        "value": round(value, 3), "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms_step, 3), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(cfg, args.sparsity, ks[0], world),
-        "stages_ms": {a: round(b, 3) for a, b in stages.items()},
-        "effective_tflops": {"attn_kernel": round(achieved, 1),
-                             "layer": round(flops / (ms_step * 1e-3) / 1e12, 1)},
-        "score_select_share": round((stages["score"] + stages["select"]) / sum(stages.values()), 4),
-        "roofline": roofline,
-        "e2e": e2e,
-        "gpu_launches": (KERNELS_PER_STEP + (4 if cfg.seg_ref and any(cfg.seg_ref) else 0)) * args.steps,
-        "clocks": clocks,
-        "attention_computed_pct": round(100.0 * stats["computed_pairs"] / stats["dense_pairs"], 2),
-        "secondary": secondary,
-    }
-    if teacher is not None:
-        line["teacher"] = teacher
-    return line
+    return bench_line(args, cfg, world, ks, flops, ms_step, stages, roofline, e2e, clocks, stats, secondary,
+                      teacher)
 
 
 def main():

@@ -1,0 +1,76 @@
+"""The CUDA arm's JSON line and roofline object, assembled on CPU from fixed stage times.
+
+The stage times are those of the committed full-clip bench line
+(profiles/bench_full_clip.md); the line built from them must carry every key
+the bench contract asks for and reproduce that run's derived figures.
+"""
+import json
+import types
+
+import pytest
+
+import bench
+import oracle.vsa_oracle as O
+from vsa_synth import get_config
+
+STAGES = {"pack_pool": 0.68, "score": 0.717, "select": 0.775, "attn": 59.311, "unpack": 0.515}
+
+
+def _args(**over):
+    a = dict(steps=20, warmup=3, sparsity=0.75, fp8=False, config="full", teacher=False)
+    a.update(over)
+    return types.SimpleNamespace(**a)
+
+
+def _ks(cfg, s):
+    return [O.k_from_sparsity(s, -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw))
+            for (pt, ph, pw) in cfg.tile_shapes]
+
+
+def _line(args, cfg):
+    ks = _ks(cfg, args.sparsity)
+    flops = bench.attention_flops(cfg, ks)
+    peaks = bench.measured_peaks()
+    roof = bench.attn_roofline(args, cfg, peaks, flops, STAGES["attn"])
+    ms_step = sum(STAGES.values())
+    e2e = {"value": 66.965, "unit": "ms", "h2d_bytes_per_step": 3 * 691273728, "d2h_bytes_per_step": 691273728}
+    clocks = {"sm_mhz": 1650.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    stats = {"computed_pairs": 3151, "dense_pairs": 10000}
+    return bench.bench_line(args, cfg, 1, ks, flops, ms_step, STAGES, roof, e2e, clocks, stats, None), peaks
+
+
+def test_line_has_the_contract_keys_and_reproduces_the_recorded_run():
+    cfg = get_config("full")
+    line, peaks = _line(_args(), cfg)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in line, key
+    json.dumps(line)
+    assert line["metric"] == bench.METRIC and line["unit"] == "ms" and line["higher_is_better"] is False
+    assert line["value"] == pytest.approx(sum(STAGES.values()), abs=1e-3)
+    assert line["gpu_launches"] == 7 * 20
+    r = line["roofline"]
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["algorithmic_flops_per_launch"] == O.attention_flops(cfg, _ks(cfg, 0.75))
+    if peaks["source"] == "measured" and peaks["bf16_tflops_sustained"] == 1387.5:
+        assert r["achieved"] == 826.3 and r["frac"] == 0.5956      # the committed bench line's figures
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"], abs=1e-3)
+    traffic = bench.measured_traffic("full", 0.75, 24)
+    assert r["traffic"] == traffic
+    if traffic is not None:                                        # the capture is of this kernel source
+        assert traffic == int((559744000 + 122771456) / 4 * 24)
+
+
+def test_fp8_line_uses_the_mixed_peak_and_no_traffic():
+    cfg = get_config("full")
+    line, peaks = _line(_args(fp8=True), cfg)
+    r = line["roofline"]
+    assert r["peak"] == round(peaks["bf16_tflops_sustained"] * 4 / 3, 1)
+    assert r["traffic"] is None and "e4m3" in r["peak_kind"]
+
+
+def test_r2va_line_counts_the_reference_launches():
+    cfg = get_config("r2va")
+    line, _ = _line(_args(sparsity=cfg.sparsity[0], config="r2va"), cfg)
+    assert line["gpu_launches"] == (7 + 4) * 20
+    assert "reference segments" in line["config"]["workload"]

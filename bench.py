@@ -226,24 +226,31 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        rows = []
         with open(self.path) as f:
-            for ln in f:
-                parts = [p.strip() for p in ln.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:9]))
-                except ValueError:
-                    continue
+            lines = f.readlines()
         os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        load = [r for r in rows if r[2] > 300.0] or rows
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in load for i in range(4) if r[3][i + 1].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
-                "samples": len(load), "power_w_max": max(r[2] for r in rows), "reasons": reasons}
+        return summarize_clocks(lines)
+
+
+def summarize_clocks(lines):
+    """Median SM clock under load, the maximum clock and the throttle reasons seen, from
+    `nvidia-smi --query-gpu=<ClockSampler.FIELDS> --format=csv,noheader,nounits` rows."""
+    rows = []
+    for ln in lines:
+        parts = [p.strip() for p in ln.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:9]))
+        except ValueError:
+            continue
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+    load = [r for r in rows if r[2] > 300.0] or rows     # samples drawing over 300 W: the timed kernels
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in load for i in range(4) if r[3][i + 1].lower().startswith("active")})
+    return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+            "samples": len(load), "power_w_max": max(r[2] for r in rows), "reasons": reasons}
 
 
 # ------------------------------------------------------------- CPU oracle ----

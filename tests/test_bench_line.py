@@ -74,3 +74,19 @@ def test_r2va_line_counts_the_reference_launches():
     line, _ = _line(_args(sparsity=cfg.sparsity[0], config="r2va"), cfg)
     assert line["gpu_launches"] == (7 + 4) * 20
     assert "reference segments" in line["config"]["workload"]
+
+
+def test_clock_summary_reads_nvidia_smi_rows():
+    rows = [
+        "0, 1980, 1965, 120.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",   # idle
+        "0, 1650, 1965, 1005.2, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1665, 1965, 998.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1635, 1965, 1010.9, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "[N/A], garbage",
+    ]
+    c = bench.summarize_clocks(rows)
+    assert c["sm_mhz"] == 1650.0 and c["sm_max_mhz"] == 1965.0 and c["samples"] == 3
+    assert c["reasons"] == ["sw_power_cap"] and c["power_w_max"] == 1010.9
+    hot = rows[1].replace("Not Active, Not Active, Not Active, Active", "Active, Not Active, Active, Not Active")
+    assert bench.summarize_clocks([hot])["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert bench.summarize_clocks([])["reasons"] == ["no samples"]

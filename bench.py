@@ -132,12 +132,6 @@ def attention_flops(cfg, ks):
     return 4 * cfg.head_dim * pairs * cfg.batch
 
 
-def layer_bytes(cfg, ks):
-    """Algorithmic HBM bytes of the element-wise stages (pack, pool, select, unpack)."""
-    tok = cfg.batch * cfg.n_tokens * cfg.heads * cfg.head_dim * 2
-    return {"pack": 2 * 3 * tok, "unpack": 2 * tok}
-
-
 def workload_config(cfg, sparsity, k0, world):
     """The `config` object of the bench line, shared by both arms."""
     ref = cfg.seg_ref and any(cfg.seg_ref)

@@ -1,8 +1,8 @@
 """The CUDA arm's JSON line and roofline object, assembled on CPU from fixed stage times.
 
 The stage times are those of the committed full-clip bench line
-(profiles/bench_full_clip.md); the line built from them must carry every key
-the bench contract asks for and reproduce that run's derived figures.
+(profiles/bench_full_clip.md); the line built from them must carry every field
+of a bench line and reproduce that run's derived figures.
 """
 import json
 import types
@@ -39,7 +39,7 @@ def _line(args, cfg):
     return bench.bench_line(args, cfg, 1, ks, flops, ms_step, STAGES, roof, e2e, clocks, stats, None), peaks
 
 
-def test_line_has_the_contract_keys_and_reproduces_the_recorded_run():
+def test_line_has_every_key_and_reproduces_the_recorded_run():
     cfg = get_config("full")
     line, peaks = _line(_args(), cfg)
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",

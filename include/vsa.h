@@ -58,7 +58,7 @@ extern "C" {
 typedef enum {
   VSA_OK = 0,
   VSA_ERR_INVALID_ARG = 1,     /* bad pointer, size, shape or alignment */
-  VSA_ERR_UNSUPPORTED = 2,     /* valid request this build does not run */
+  VSA_ERR_UNSUPPORTED = 2,     /* valid request these kernels do not handle */
   VSA_ERR_CUDA = 3,            /* a CUDA runtime or driver call failed */
   VSA_ERR_DEVICE_TIMEOUT = 4,  /* a device-side wait ran past its limit */
   VSA_ERR_BAD_INDEX = 5,       /* a kept-tile list holds an out-of-range or repeated tile */

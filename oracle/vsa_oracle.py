@@ -480,18 +480,14 @@ def e4m3_round(x) -> np.ndarray:
 
 def quantize_tile_e4m3(x: np.ndarray):
     """Per-tile fp8 quantisation of one packed tile's rows (the tile-skipping kernels on the
-    Veda page run their QK^T in 8-bit with per-tile scales; the plainest reading): with the
-    tile's largest magnitude amax, each value is multiplied in fp32 by 448 / amax (one fp32
-    division per tile) and rounded to e4m3; the dequantisation scale is amax / 448 in fp32.
-    An all-zero tile uses 1 for both. Returns (codes as fp64 values, scale)."""
+    Veda page run their QK^T in 8-bit with per-tile scales; the plainest reading): the scale
+    s is the tile's largest magnitude / 448 in fp32 (1 for an all-zero tile), and each value
+    is divided by s in fp32 (one correctly rounded division per element) and rounded to
+    e4m3. Returns (codes as fp64 values, scale)."""
     xf = np.asarray(x, dtype=np.float32)
     amax = np.float32(np.max(np.abs(xf))) if xf.size else np.float32(0)
-    if amax > 0:
-        inv = np.float32(np.float32(E4M3_MAX) / amax)
-        scale = np.float32(amax / np.float32(E4M3_MAX))
-    else:
-        inv = scale = np.float32(1.0)
-    return e4m3_round((xf * inv).astype(np.float64)), float(scale)
+    scale = np.float32(amax / np.float32(E4M3_MAX)) if amax > 0 else np.float32(1.0)
+    return e4m3_round((xf / scale).astype(np.float64)), float(scale)
 
 
 def dequantized_tiles(x_h: np.ndarray, til: HeadTiling) -> np.ndarray:

@@ -729,6 +729,37 @@ def test_tile_quantisation_scale_and_range():
     assert O.quantize_tile_e4m3(np.zeros((3, 8)))[1] == 1.0
 
 
+def pin_fp8_codes_divide_by_the_scale():
+    """A tile whose largest magnitude is 1.53125 = 49/32 has the scale 49/32 / 448 = 7/2048,
+    exact in fp32. Its entry 0.341796875 = 175/512 divided by that scale is exactly 100, the
+    midpoint between the e4m3 codes 96 and 104, so rounding to nearest even gives 96.
+    Multiplying by the rounded reciprocal fl(448 / amax) instead lands just above 100 and
+    gives 104, so this tile tells the two rules apart."""
+    x = np.full((64, 128), 0.341796875, dtype=np.float32)
+    x[0, 0] = 1.53125
+    codes, scale = O.quantize_tile_e4m3(x)
+    assert scale == 7 / 2048
+    assert codes[0, 0] == 448.0
+    assert np.all(codes.ravel()[1:] == 96.0), np.unique(codes)
+
+
+def test_fp8_codes_divide_by_the_scale():
+    pin_fp8_codes_divide_by_the_scale()
+    # the other rule really does differ on this tile
+    inv = np.float32(np.float32(448.0) / np.float32(1.53125))
+    assert O.e4m3_round(np.float64(np.float32(0.341796875) * inv)) == 104.0
+
+
+def test_mutation_fp8_reciprocal_multiply(monkeypatch):
+    def bad(x):
+        xf = np.asarray(x, dtype=np.float32)
+        amax = np.float32(np.max(np.abs(xf)))
+        inv = np.float32(np.float32(O.E4M3_MAX) / amax)
+        return O.e4m3_round((xf * inv).astype(np.float64)), float(np.float32(amax / np.float32(O.E4M3_MAX)))
+    monkeypatch.setattr(O, "quantize_tile_e4m3", bad)
+    _expect_pin_failure(pin_fp8_codes_divide_by_the_scale)
+
+
 def test_fp8_attention_is_exact_on_representable_inputs():
     """Q and K entries from {0, +-0.5, +-1, +-1.75} with a 1.75 in every tile: every scale
     is 1.75/448 = 2^-8 exactly and every entry divided by it (0, 128, 256, 448) is an e4m3

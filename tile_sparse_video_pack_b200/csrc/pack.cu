@@ -123,9 +123,10 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float (&x)[8]) {
 //
 // QUANT: the same pass also writes Q and K of every packed tile as e4m3 (fp8)
 // with one fp32 scale per (tile, tensor): with amax the tile's largest
-// magnitude, code = e4m3(x * (448 / amax)) (fp32 product, rounded to nearest
-// even, saturated) and scale = amax / 448 (1 for an all-zero tile) -- per-tile
-// 8-bit Q K^T, as the tile-skipping kernels on the Veda page run it.
+// magnitude, scale = amax / 448 (1 for an all-zero tile) and code = e4m3(x /
+// scale) (correctly rounded fp32 division, then rounded to nearest even and
+// saturated) -- per-tile 8-bit Q K^T, as the tile-skipping kernels on the Veda
+// page run it.
 template <int CPR, bool TRIP, bool QUANT>
 __global__ void __launch_bounds__(256) pack_pool_kernel(Geometry g, const uint4* __restrict__ q,
                                                         const uint4* __restrict__ k,
@@ -225,14 +226,13 @@ __global__ void __launch_bounds__(256) pack_pool_kernel(Geometry g, const uint4*
       amax_part[1][warp0] = am[1];
     }
     __syncthreads();
-    float sc[2], inv[2];   // dequantisation scale amax / 448 and quantisation factor 448 / amax
+    float sc[2];   // dequantisation scale amax / 448; codes are x / scale
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       float m = 0.f;
 #pragma unroll
       for (int w = 0; w < 8; ++w) m = fmaxf(m, amax_part[t][w]);
       sc[t] = m > 0.f ? __fdiv_rn(m, 448.0f) : 1.0f;
-      inv[t] = m > 0.f ? __fdiv_rn(448.0f, m) : 1.0f;
     }
     if (threadIdx.x == 0) {
       q_scale[tile] = sc[0];
@@ -250,9 +250,9 @@ __global__ void __launch_bounds__(256) pack_pool_kernel(Geometry g, const uint4*
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
-              make_float2(__fmul_rn(x[4 * e], inv[t]), __fmul_rn(x[4 * e + 1], inv[t])), __NV_SATFINITE, __NV_E4M3);
+              make_float2(__fdiv_rn(x[4 * e], sc[t]), __fdiv_rn(x[4 * e + 1], sc[t])), __NV_SATFINITE, __NV_E4M3);
           const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
-              make_float2(__fmul_rn(x[4 * e + 2], inv[t]), __fmul_rn(x[4 * e + 3], inv[t])), __NV_SATFINITE,
+              make_float2(__fdiv_rn(x[4 * e + 2], sc[t]), __fdiv_rn(x[4 * e + 3], sc[t])), __NV_SATFINITE,
               __NV_E4M3);
           w[e] = uint32_t(lo) | (uint32_t(hi) << 16);
         }

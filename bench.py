@@ -10,11 +10,17 @@ reference-image, 640 reference-audio tokens), mean-pool gate scoring, 75% video
 sparsity (420 kept tiles); the 90% line is measured in the same run. Inputs are
 seeded synthetic tensors (3 x 691 MB, larger than L2).
 
-Multi-GPU (torchrun): every rank runs its own layer (independent problems, no
-collective on the data path); the time is the max over ranks.
+Other workloads (--config): veda (head-aware tiles, TripPool, 90% and 95%), long
+(230k video tokens, sparsity 0 ... 0.95), r2va, medium, tiny. Every sparsity level
+of the workload other than the first is measured in the same run ("sweep").
+
+Multi-GPU (torchrun): by default every rank runs its own layer (independent
+problems, weak scaling); with --split heads the ranks share one layer, each
+running its block of heads (strong scaling). Neither has a collective on the data
+path; the time is the max over ranks.
 
 --impl reference times the fp64 CPU oracle (the only reference there is) on a
-bounded sample of the same workload and extrapolates to one layer.
+fixed bounded sample of the same workload and extrapolates to one layer.
 """
 from __future__ import annotations
 
@@ -33,8 +39,15 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 CONFIG = "full"
-SECONDARY_SPARSITY = 0.9
-METRIC = "ms per attention layer at 107k video tokens, 75% video sparsity (90% in secondary); effective TFLOP/s"
+METRIC = "ms per attention layer at 107k video tokens, 75% video sparsity (90% in sweep); effective TFLOP/s"
+
+
+def metric_for(cfg):
+    """The metric string: the headline one for the full clip, a workload-specific one otherwise."""
+    if cfg.name == CONFIG:
+        return METRIC
+    return (f"ms per attention layer, {cfg.name} workload ({cfg.n_video_tokens} video tokens), "
+            f"sparsity {cfg.sparsity[0]} (other levels in sweep); effective TFLOP/s")
 KERNELS_PER_STEP = 7  # pack + pool 1, score 3 (2 projections, scores), select 1, attention 1, unpack 1
 
 
@@ -48,7 +61,10 @@ def parse():
     ap.add_argument("--sparsity", type=float, default=None,
                     help="video-key sparsity (default: the workload's first level, 0.75 for the full clip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-secondary", "--no-sweep", dest="no_secondary", action="store_true",
+                    help="measure only the first sparsity level of the workload")
+    ap.add_argument("--split", default="layers", choices=["layers", "heads"],
+                    help="multi-GPU: each rank its own layer (weak scaling) or its block of one layer's heads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
     ap.add_argument("--fp8", action="store_true",
@@ -132,16 +148,21 @@ def attention_flops(cfg, ks):
     return 4 * cfg.head_dim * pairs * cfg.batch
 
 
-def workload_config(cfg, sparsity, k0, world):
+def workload_config(cfg, sparsity, k0, world, split="layers"):
     """The `config` object of the bench line, shared by both arms."""
     ref = cfg.seg_ref and any(cfg.seg_ref)
+    mb = cfg.batch * cfg.n_tokens * cfg.heads * cfg.head_dim * 2 / 1e6
+    heads_split = split == "heads" and world > 1
     return {"workload": f"{cfg.name}: one layer, B={cfg.batch}, {cfg.heads} heads, d={cfg.head_dim}, "
                         f"grid {cfg.T}x{cfg.H}x{cfg.W} + prefix {list(cfg.segments)}, "
                         f"{cfg.score_mode}, sparsity {sparsity} (k={k0})"
                         + (f", reference segments {list(cfg.seg_ref)} with k_ref={cfg.k_ref}" if ref else ""),
             "tokens": cfg.n_tokens, "heads": cfg.heads, "head_dim": cfg.head_dim, "k": k0,
-            "layers_per_step": world, "parallelism": f"independent layers x{world}",
-            "l2": "inputs larger than L2 (Q, K, V 691 MB each)"}
+            "layers_per_step": 1 if heads_split else world,
+            "parallelism": (f"heads of one layer split over {world} ranks" if heads_split
+                            else f"independent layers x{world}"),
+            "l2": (f"inputs larger than L2 (Q, K, V {mb:.0f} MB each)" if mb > 126 else
+                   f"inputs {mb:.0f} MB each: L2-resident between steps")}
 
 
 def attn_roofline(args, cfg, peaks, flops, attn_ms):
@@ -150,29 +171,34 @@ def attn_roofline(args, cfg, peaks, flops, attn_ms):
     # fp8: Q K^T (half the FLOPs) at the e4m3 rate, twice bf16's (nominal ratio), P V at bf16, so the
     # mixed peak is 1 / (0.5 / 2 + 0.5 / 1) = 4/3 of the measured bf16 peak
     mix = 4.0 / 3.0 if args.fp8 else 1.0
-    peak = round(peaks["bf16_tflops_sustained"] * mix, 1)
+    # each launch is timed on its own (tens of ms), not a seconds-long loop: the burst peak
+    peak = round(peaks["bf16_tflops"] * mix, 1)
     return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
             "traffic": None if args.fp8 else measured_traffic(args.config, args.sparsity, cfg.heads),
             "kernel": "attn_kernel<128, fp8> (vsa_sparse_attn_fp8; e4m3 Q K^T, bf16 P V)" if args.fp8
                       else "attn_kernel (vsa_sparse_attn)",
-            "peak_kind": (f"half e4m3 (2x bf16, nominal ratio), half bf16: 4/3 x bf16 dense, sustained, "
-                          f"{peaks['source']}") if args.fp8 else f"bf16 dense, sustained, {peaks['source']}",
-            "frac_of_burst_peak": round(achieved / (peaks["bf16_tflops"] * mix), 4),
+            "peak_kind": (f"half e4m3 (2x bf16, nominal ratio), half bf16: 4/3 x bf16 dense, burst, "
+                          f"{peaks['source']}") if args.fp8 else f"bf16 dense, burst, {peaks['source']}",
+            "frac_of_sustained_peak": round(achieved / (peaks["bf16_tflops_sustained"] * mix), 4),
             "algorithmic_flops_per_launch": flops}
 
 
-def bench_line(args, cfg, world, ks, flops, ms_step, stages, roofline, e2e, clocks, stats, secondary,
+def bench_line(args, cfg, world, ks, flops, ms_step, stages, roofline, e2e, clocks, stats, sweep,
                teacher=None):
-    """The JSON line of the CUDA arm (rank 0 prints it)."""
+    """The JSON line of the CUDA arm (rank 0 prints it). With the heads of one layer split over
+    the ranks, `cfg`, `ks` and `flops` are the whole layer's and a step is that one layer."""
     ref = cfg.seg_ref and any(cfg.seg_ref)
+    split = getattr(args, "split", "layers")
+    heads_split = split == "heads" and world > 1
     line = {
-        "metric": METRIC,
-        "value": round(job_ms_per_layer(ms_step, 1, world), 3), "unit": "ms", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms_step, 3), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "metric": metric_for(cfg),
+        "value": round(ms_step if heads_split else job_ms_per_layer(ms_step, 1, world), 3), "unit": "ms",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3), "higher_is_better": False,
+        "scaling": "strong" if heads_split else "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(cfg, args.sparsity, ks[0], world),
+        "config": workload_config(cfg, args.sparsity, ks[0], world, split),
         "stages_ms": {a: round(b, 3) for a, b in stages.items()},
         "effective_tflops": {"attn_kernel": roofline["achieved"],
                              "layer": round(flops / (ms_step * 1e-3) / 1e12, 1)},
@@ -182,7 +208,7 @@ def bench_line(args, cfg, world, ks, flops, ms_step, stages, roofline, e2e, cloc
         "gpu_launches": (KERNELS_PER_STEP + (4 if ref else 0)) * args.steps,
         "clocks": clocks,
         "attention_computed_pct": round(100.0 * stats["computed_pairs"] / stats["dense_pairs"], 2),
-        "secondary": secondary,
+        "sweep": sweep,
     }
     if teacher is not None:
         line["teacher"] = teacher
@@ -250,13 +276,16 @@ def summarize_clocks(lines):
 # ------------------------------------------------------------- CPU oracle ----
 
 class OracleSample:
-    """The fp64 oracle, as it stands, timed on a bounded sample of one layer (head 0).
+    """The fp64 oracle, as it stands, timed on a fixed bounded sample of one layer.
 
-    Scores and top-k of the head are timed in full; attention is timed on
-    randomly drawn query tiles (three video tiles per prefix tile) until a time
-    budget is spent; the per-tile means are extrapolated to every query tile of
-    every head of the layer.
+    One sample: scores and top-k of head 0 in full, then attention (the same two
+    oracle calls run_layer makes per query tile) of a fixed, evenly spaced set of
+    head 0's query tiles -- n_video video tiles and n_prefix prefix tiles. Each
+    kind's mean time per tile is extrapolated to every query tile of every head.
+    Both bench arms use this class with the same sample, so their estimates agree.
     """
+
+    N_VIDEO, N_PREFIX = 48, 16
 
     def __init__(self, cfg, sparsity):
         import numpy as np
@@ -271,10 +300,13 @@ class OracleSample:
         self.ks = [O.k_from_sparsity(sparsity, -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw))
                    for (pt, ph, pw) in self.sub.tile_shapes]
         self.til = O.head_tiling(self.sub, 0)
-        self.rng = np.random.default_rng(0)
+        til = self.til
+        pick = lambda n, m: sorted({int(x) for x in np.linspace(0, n - 1, min(n, m))}) if n else []
+        self.video_tiles = [til.n_prefix + i for i in pick(til.n_video, self.N_VIDEO)]
+        self.prefix_tiles = pick(til.n_prefix, self.N_PREFIX)
 
-    def run(self, budget_s):
-        """Times the oracle's own steps: scores + top-k of the head, then its per-tile attention."""
+    def run(self):
+        """One sample; returns the extrapolated ms per layer and what was timed."""
         np, O, sub, til, inp = self.np, self.O, self.sub, self.til, self.inp
         t0 = time.perf_counter()
         s = O.tile_scores(self.q[0, :, 0], self.k[0, :, 0], til, sub, 0, inp.gate, inp.w_q, inp.w_k)
@@ -282,43 +314,51 @@ class OracleSample:
         t_select = time.perf_counter() - t0
         scale = 1.0 / math.sqrt(sub.head_dim)
         q, k, v = self.q[0, :, 0], self.k[0, :, 0], self.v[0, :, 0]
-        t_pre = t_vid = 0.0
-        n_pre = n_vid = 0
-        t_start = time.perf_counter()
-        while time.perf_counter() - t_start < budget_s or n_vid == 0:
-            for kind in ("video", "video", "video", "prefix"):
-                if kind == "prefix" and til.n_prefix == 0:
-                    continue
-                t = (int(self.rng.integers(0, til.n_prefix)) if kind == "prefix"
-                     else til.n_prefix + int(self.rng.integers(0, til.n_video)))
-                t1 = time.perf_counter()
-                # the same two calls run_layer makes for one query tile
+        spent = {}
+        for kind, tiles in (("video", self.video_tiles), ("prefix", self.prefix_tiles)):
+            t1 = time.perf_counter()
+            for t in tiles:
                 kv = O.query_key_tokens(til, t, None if t < til.n_prefix else kept[t - til.n_prefix])
-                qt = til.all[t]
-                O.softmax_attention(q[qt], k[kv], v[kv], scale)
-                dt = time.perf_counter() - t1
-                if kind == "prefix":
-                    t_pre, n_pre = t_pre + dt, n_pre + 1
-                else:
-                    t_vid, n_vid = t_vid + dt, n_vid + 1
-        t_vid_row = t_vid / n_vid
-        t_pre_row = t_pre / n_pre if n_pre else 0.0
-        per_head = t_select + t_vid_row * til.n_video + t_pre_row * til.n_prefix
+                O.softmax_attention(q[til.all[t]], k[kv], v[kv], scale)
+            spent[kind] = time.perf_counter() - t1
+        per_head = t_select
+        per_head += spent["video"] / max(1, len(self.video_tiles)) * til.n_video
+        per_head += spent["prefix"] / max(1, len(self.prefix_tiles)) * til.n_prefix
         ms = per_head * self.cfg.heads * self.cfg.batch * 1e3
         try:
             cores = len(os.sched_getaffinity(0))
         except AttributeError:
             cores = os.cpu_count()
         sample = (f"head 0 of {self.cfg.heads}: scores + top-k of all {til.n_video} video query tiles, attention "
-                  f"of {n_vid} video and {n_pre} prefix query tiles drawn at random (fp64 numpy; BLAS on all "
-                  f"cores); extrapolated to {self.cfg.heads} heads x ({til.n_video} video + {til.n_prefix} "
-                  f"prefix) query tiles")
+                  f"of a fixed set of {len(self.video_tiles)} video and {len(self.prefix_tiles)} prefix query "
+                  f"tiles (fp64 numpy; BLAS on all cores); extrapolated to {self.cfg.heads} heads x "
+                  f"({til.n_video} video + {til.n_prefix} prefix) query tiles")
         return {"value": round(ms, 1), "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample,
-                "extrapolated": True, "cpu_seconds": round(time.perf_counter() - t0, 1)}
+                "extrapolated": True, "sample_s": round(time.perf_counter() - t0, 5)}
 
 
-def cpu_baseline(cfg, sparsity, budget_s=20.0):
-    return OracleSample(cfg, sparsity).run(budget_s)
+def oracle_full_layer_ms(cfg, sparsity):
+    """The fp64 oracle's whole layer (every head and query tile), timed once: for workloads small
+    enough to run in full (the medium one takes seconds to tens of seconds)."""
+    import numpy as np
+    import oracle.vsa_oracle as O
+    from vsa_synth import bf16_bits_to_f32, make_layer_inputs
+    inp = make_layer_inputs(cfg)
+    f = lambda b: bf16_bits_to_f32(b).astype(np.float64)
+    q, k, v = f(inp.q), f(inp.k), f(inp.v)
+    ks = [O.k_from_sparsity(sparsity, -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw))
+          for (pt, ph, pw) in cfg.tile_shapes]
+    t0 = time.perf_counter()
+    O.run_layer(cfg, q, k, v, ks, gate=inp.gate, w_q=inp.w_q, w_k=inp.w_k)
+    return (time.perf_counter() - t0) * 1e3
+
+
+def cpu_baseline(cfg, sparsity):
+    """The oracle on the host: one warm-up sample and one timed sample of this workload."""
+    s = OracleSample(cfg, sparsity)
+    s.run()
+    return s.run()
+
 
 
 # ---------------------------------------------------------------- ranks ------
@@ -334,6 +374,17 @@ def max_over_ranks_on(x: float, device, world: int) -> float:
     return float(t.item())
 
 
+def all_ranks_sum(x: float, device, world: int) -> float:
+    """The sum of every rank's x (the head blocks of one layer add up to the layer)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def job_ms_per_layer(ms_step_max: float, layers_per_rank: int, world: int) -> float:
     """Whole-job time per layer: the slowest rank's step time over all layers processed in a step."""
     return ms_step_max / (layers_per_rank * world)
@@ -341,7 +392,7 @@ def job_ms_per_layer(ms_step_max: float, layers_per_rank: int, world: int) -> fl
 
 # ---------------------------------------------------------------- GPU arm ----
 
-def e2e_measure(args, layer, q, k, v, out, stream, world, barrier, max_over_ranks):
+def e2e_measure(args, layer, q, k, v, out, stream, world, barrier, max_over_ranks, layers=None):
     """The same layer through the public API from pinned host buffers, copies inside the timing.
 
     Every step copies its q, k, v in from pinned host memory, runs the layer and copies o
@@ -400,10 +451,37 @@ def e2e_measure(args, layer, q, k, v, out, stream, world, barrier, max_over_rank
     # the layer is deterministic: what came back equals the device-timed run's output
     if not torch.equal(ho[(steps - 1) & 1].view(torch.int16), out.cpu().view(torch.int16)):
         raise RuntimeError("end-to-end output differs from the device-timed run")
-    ms = max_over_ranks(e0.elapsed_time(e1) / steps) / world
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps) / (world if layers is None else layers)
     return {"value": round(ms, 3), "unit": "ms", "h2d_bytes_per_step": 3 * q.numel() * q.element_size() * world,
             "d2h_bytes_per_step": out.numel() * out.element_size() * world, "steps": steps,
             "overlap": "h2d of step i+1 and d2h of step i-1 run on copy streams during step i"}
+
+
+def gpu_layer_ms(cfg, sparsity, steps=10, warmup=3):
+    """Mean device time of one whole layer (vsa_layer_forward) of `cfg` on the current GPU."""
+    import numpy as np
+    import torch
+    import tile_sparse_video_pack_b200 as T
+    from vsa_synth import make_layer_inputs
+    inp = make_layer_inputs(cfg)
+    to_dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    if cfg.score_mode == "meanpool_gate":
+        pq = pk = torch.from_numpy(inp.gate).cuda()
+    else:
+        pq, pk = torch.from_numpy(inp.w_q).cuda(), torch.from_numpy(inp.w_k).cuda()
+    layer = T.TileSparseAttention.from_config(cfg, sparsity, pq, pk)
+    out = torch.empty_like(q)
+    for _ in range(warmup):
+        layer(q, k, v, out)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        layer(q, k, v, out)
+    e1.record()
+    torch.cuda.synchronize()
+    layer.plan.check()
+    return e0.elapsed_time(e1) / steps
 
 
 def run_ours(args, rank, world, local_rank):
@@ -415,6 +493,8 @@ def run_ours(args, rank, world, local_rank):
     from tile_sparse_video_pack_b200.build import build
     from vsa_synth import get_config, make_layer_inputs
 
+    from tile_sparse_video_pack_b200.shard import partition_heads, shard_config, shard_heads_of
+
     build()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -422,12 +502,19 @@ def run_ours(args, rank, world, local_rank):
     if args.heads:
         cfg = cfg.with_(heads=args.heads, tile_shapes=cfg.tile_shapes[:args.heads])
     inp = make_layer_inputs(cfg)
-    to_dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
-    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
-    if cfg.score_mode == "meanpool_gate":
+    layer_cfg = cfg                              # the whole layer (for the FLOP count and the line)
+    heads_split = args.split == "heads" and world > 1
+    h0, h1 = partition_heads(cfg.heads, world, rank) if heads_split else (0, cfg.heads)
+    if heads_split:                              # this rank's block of the layer's heads
+        cfg = shard_config(cfg, h0, h1)
+    pick = lambda x: shard_heads_of(x, h0, h1, 2) if heads_split else x
+    to_dev = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v = to_dev(pick(inp.q)), to_dev(pick(inp.k)), to_dev(pick(inp.v))
+    if cfg.score_mode == "meanpool_gate":        # the gate is shared by all heads: replicated
         pq = pk = torch.from_numpy(inp.gate).to(dev)
-    else:
-        pq, pk = torch.from_numpy(inp.w_q).to(dev), torch.from_numpy(inp.w_k).to(dev)
+    else:                                        # per-head projections: this rank's heads
+        w = lambda x: shard_heads_of(x, h0, h1, 0) if heads_split else x
+        pq, pk = torch.from_numpy(w(inp.w_q)).to(dev), torch.from_numpy(w(inp.w_k)).to(dev)
     peaks = measured_peaks()
     stream = torch.cuda.current_stream()
 
@@ -534,25 +621,35 @@ def run_ours(args, rank, world, local_rank):
 
     ks = k_list(cfg, args.sparsity)
     layer, out, ms_step, stages, clocks, stats = timed_layer(args.sparsity, args.steps, args.warmup, True)
-    flops = attention_flops(cfg, ks)
-    roofline = attn_roofline(args, cfg, peaks, flops, max_over_ranks(stages["attn"]))
+    if heads_split:                  # the whole layer's pairs: the sum over the ranks' head blocks
+        stats = {key: int(all_ranks_sum(float(val), dev, world)) for key, val in stats.items()}
+    flops = attention_flops(layer_cfg, k_list(layer_cfg, args.sparsity))
+    roofline = attn_roofline(args, layer_cfg, peaks, flops, max_over_ranks(stages["attn"]))
+    # every rank's stage times are its own; the line reports the slowest rank's
+    stages = {name: max_over_ranks(val) for name, val in stages.items()}
 
     # end to end through host buffers: pinned H2D of q, k, v, the layer, D2H of o
-    e2e = None if args.no_e2e else e2e_measure(args, layer, q, k, v, out, stream, world, barrier, max_over_ranks)
+    e2e = None if args.no_e2e else e2e_measure(args, layer, q, k, v, out, stream, world, barrier, max_over_ranks,
+                                               layers=1 if heads_split else world)
 
-    secondary = None
+    # the workload's other sparsity levels, measured in the same run
+    sweep = []
     if not args.no_secondary:
-        ks2 = k_list(cfg, SECONDARY_SPARSITY)
-        _, _, ms2, st2, _, _ = timed_layer(SECONDARY_SPARSITY, max(3, args.steps // 2), 2, False)
-        f2 = attention_flops(cfg, ks2)
-        secondary = {"sparsity": SECONDARY_SPARSITY, "k": ks2[0], "ms_per_layer": round(ms2 / world, 3),
-                     "stages_ms": {a: round(b, 3) for a, b in st2.items()},
-                     "attn_tflops": round(f2 / (st2["attn"] * 1e-3) / 1e12, 1),
-                     "layer_tflops": round(f2 / (ms2 * 1e-3) / 1e12, 1)}
+        for s2 in [x for x in layer_cfg.sparsity if x != args.sparsity]:
+            f2 = attention_flops(layer_cfg, k_list(layer_cfg, s2))
+            _, _, ms2, st2, _, _ = timed_layer(s2, max(3, args.steps // 2), 2, False)
+            st2 = {name: max_over_ranks(val) for name, val in st2.items()}
+            sweep.append({"sparsity": s2, "k": k_list(layer_cfg, s2)[0],
+                          "ms_per_layer": round(ms2 if heads_split else ms2 / world, 3),
+                          "stages_ms": {a: round(b, 3) for a, b in st2.items()},
+                          "attn_tflops": round(f2 / (st2["attn"] * 1e-3) / 1e12, 1),
+                          "attn_frac_of_burst_peak": round(f2 / (st2["attn"] * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                          "layer_tflops": round(f2 / (ms2 * 1e-3) / 1e12, 1),
+                          "algorithmic_flops": f2})
 
     teacher = teacher_measure(layer, ks) if args.teacher else None
-    return bench_line(args, cfg, world, ks, flops, ms_step, stages, roofline, e2e, clocks, stats, secondary,
-                      teacher)
+    return bench_line(args, layer_cfg, world, k_list(layer_cfg, args.sparsity), flops, ms_step, stages, roofline,
+                      e2e, clocks, stats, sweep, teacher)
 
 
 def main():
@@ -571,22 +668,26 @@ def main():
         pt, ph, pw = cfg.tile_shapes[0]
         k0 = O.k_from_sparsity(args.sparsity, -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw))
         sampler = OracleSample(cfg, args.sparsity)
-        per_step = max(2.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
-        vals = []
         for _ in range(args.warmup):
-            sampler.run(per_step / 2)
+            sampler.run()
         t0 = time.time()
-        last = None
-        for _ in range(args.steps):
-            last = sampler.run(per_step)
+        vals, walls, last = [], [], None
+        for _ in range(args.steps):          # a step: one fixed sample of the layer, run in full
+            last = sampler.run()
             vals.append(last["value"])
+            walls.append(last["sample_s"])
         v = statistics.median(vals)
-        line = {"impl": "reference", "metric": METRIC,
+        line = {"impl": "reference", "metric": metric_for(cfg),
                 "value": v, "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": v, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+                # what one step (sample) actually took; `value` is the layer time extrapolated from it
+                "ms_per_step": round(1e3 * statistics.mean(walls), 3) if walls else 0.0,
+                "extrapolated": True,
+                "step": "one fixed sample of the layer (see cpu_baseline.sample), timed in full; value = the "
+                        "median over steps of the whole-layer time extrapolated from each sample",
+                "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f64", "data": "synthetic",
                 "config": workload_config(cfg, args.sparsity, k0, world),
-                "cpu_baseline": {**last, "value": v},
+                "cpu_baseline": {**last, "value": v} if last else None,
                 "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
                 "wall_s": round(time.time() - t0, 1)}
         print(json.dumps(line), flush=True)
@@ -602,7 +703,16 @@ def main():
         line = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             from vsa_synth import get_config
-            line["cpu_baseline"] = cpu_baseline(get_config(args.config), args.sparsity)
+            cfg = get_config(args.config)
+            if args.heads:
+                cfg = cfg.with_(heads=args.heads, tile_shapes=cfg.tile_shapes[:args.heads])
+            line["cpu_baseline"] = cpu_baseline(cfg, args.sparsity)
+            # the medium workload, small enough for the oracle to run whole, beside the GPU's time for it
+            med = get_config("medium")
+            line["cpu_baseline"]["medium_full_layer"] = {
+                "workload": "medium (24 heads, 7,680 video tokens, 75%)", "extrapolated": False,
+                "oracle_ms": round(oracle_full_layer_ms(med, med.sparsity[0]), 1),
+                "gpu_ms": round(gpu_layer_ms(med, med.sparsity[0]), 3)}
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -207,9 +207,16 @@ VSA_API vsa_status vsa_tile_score_pooled(vsa_plan* plan, const float* proj_q, co
  *  - The scratch is a 32 MiB array in device memory, held by every GPU that
  *    loads this library until the process exits. Plans whose workspace_bytes
  *    exceed 32 MiB are rejected with VSA_ERR_UNSUPPORTED.
- *  - The call allocates nothing. Its first call on a device looks up the
- *    array's device address (cudaGetSymbolAddress) with that device current;
- *    make that first call before any stream capture.
+ *  - The call allocates nothing. The array's device address is looked up
+ *    (cudaGetSymbolAddress, with the device current) by every
+ *    vsa_plan_create and kept per device; if no plan had been created on
+ *    the device, the first call of this function looks it up instead, so
+ *    make that first call before any stream capture. After a
+ *    cudaDeviceReset, create new plans (old ones are invalid anyway): that
+ *    refreshes the address.
+ *  - Plans with reference segments (seg_ref) are rejected with
+ *    VSA_ERR_UNSUPPORTED: vsa_ref_score needs the projected pooled Q in the
+ *    caller's workspace, which this call does not write.
  *  - The current device must be the plan's device (else VSA_ERR_INVALID_ARG).
  *  - Every call on a device shares the one array, which keeps the last
  *    call's contents (each call writes every scratch element before reading
@@ -221,18 +228,33 @@ VSA_API vsa_status vsa_tile_score_static(vsa_plan* plan, const void* qp, const v
                                          const float* proj_q, const float* proj_k, float* scores,
                                          void* stream);
 
-/* a5. For every (b, h, video query tile i) keep the k_per_head[h] video key
- * tiles with the largest scores; equal scores keep the lower tile index. The
- * kept tile indices (0-based video tile ids) are written sorted ascending to
- * idx[b][h][i][0 .. k-1] (int32, [B, heads, ntv_max, k_max]). -0.0 and +0.0
- * compare equal; NaN scores are rejected on the device (VSA_ERR_BAD_INDEX via
- * vsa_plan_check). Veda page "Что делает Veda" (head-aware top-k forms the
- * tile mask); Ref2VA VSA README item 2 (top-k only over video key tiles). */
-VSA_API vsa_status vsa_topk_select(vsa_plan* plan, const float* scores, int32_t* idx, void* stream);
+/* Per-call k. k_per_head, where the calls below take it, is a HOST array of
+ * `heads` int32 values read during the call (the caller keeps ownership; it
+ * may be reused as soon as the call returns): the kept video key tiles per
+ * video query tile of each head for this call, each in 1 .. min(video tiles of
+ * the head, k_max of the plan) -- k_max, the largest k_per_head of the plan's
+ * descriptor, is the row width of the index tables. NULL means the plan's own
+ * k_per_head. Any other value is rejected with VSA_ERR_INVALID_ARG before
+ * anything is launched. One plan created at the largest k thus serves every
+ * smaller sparsity (Ref2VA VSA README: "75% video sparsity top-k"; BSAI
+ * VedaSparse README, "Nodes": keep_percent per run). The top-k and attention
+ * calls of one layer must be given the same k. */
+
+/* a5. For every (b, h, video query tile i) keep the k[h] video key tiles with
+ * the largest scores (k from k_per_head, above); equal scores keep the lower
+ * tile index. The kept tile indices (0-based video tile ids) are written
+ * sorted ascending to idx[b][h][i][0 .. k[h]-1] (int32, [B, heads, ntv_max,
+ * k_max]; entries past k[h] untouched). -0.0 and +0.0 compare equal; NaN
+ * scores are rejected on the device (VSA_ERR_BAD_INDEX via vsa_plan_check).
+ * Veda page "Что делает Veda" (head-aware top-k forms the tile mask); Ref2VA
+ * VSA README item 2 (top-k only over video key tiles). */
+VSA_API vsa_status vsa_topk_select(vsa_plan* plan, const float* scores, const int32_t* k_per_head, int32_t* idx,
+                                   void* stream);
 
 /* a6. Block-sparse exact attention on packed tiles. A prefix query tile
  * attends to every valid key of its head; a video query tile attends to every
- * prefix tile plus the video tiles listed in idx[b][h][i][0 .. k-1] (ascending,
+ * prefix tile plus the video tiles listed in idx[b][h][i][0 .. k[h]-1] (k from
+ * k_per_head, as for vsa_topk_select; ascending,
  * distinct, in range -- otherwise the rows are skipped and VSA_ERR_BAD_INDEX is
  * latched). o = softmax(scale * q k^T over the valid keys) v, fp32 accumulation,
  * written as bf16 to op ([B, heads, nt_max, 64, d]); rows of unused slots of
@@ -243,7 +265,7 @@ VSA_API vsa_status vsa_topk_select(vsa_plan* plan, const float* scores, int32_t*
  * BSAI VedaSparse README "Core Technology: Tile-Skipping", "v3.4 Highlights"
  * (sink = exact_kv_and_rows: conditioning rows and keys stay exact). */
 VSA_API vsa_status vsa_sparse_attn(vsa_plan* plan, const void* qp, const void* kp, const void* vp,
-                           const int32_t* idx, void* op, float* lse, void* stream);
+                           const int32_t* idx, const int32_t* k_per_head, void* op, float* lse, void* stream);
 
 /* a7. Inverse of the pack permutation: [B, heads, nt_max, 64, d] -> [B, N, heads, d]. */
 VSA_API vsa_status vsa_tile_unpack(vsa_plan* plan, const void* op, void* o, void* stream);
@@ -272,17 +294,17 @@ VSA_API vsa_status vsa_topk_select_ref(vsa_plan* plan, const float* scores_ref, 
  * prefix tiles stay dense and prefix query rows still see every key. Indices
  * out of range or not ascending are rejected as in vsa_sparse_attn. */
 VSA_API vsa_status vsa_sparse_attn_ref(vsa_plan* plan, const void* qp, const void* kp, const void* vp,
-                               const int32_t* idx, const int32_t* idx_ref, void* op, float* lse,
-                               void* stream);
+                               const int32_t* idx, const int32_t* idx_ref, const int32_t* k_per_head, void* op,
+                               float* lse, void* stream);
 
 /* fp8 Q K^T (row f2; the tile-skipping kernels on the Veda page run Q K^T in
  * 8-bit with per-tile scales). vsa_tile_pack_pool, and besides: Q and K of
  * every packed tile as e4m3 bytes qp8, kp8 ([B, heads, nt_max, 64, head_dim]
  * bytes, packed_elems of them) with one fp32 scale per (tile, tensor) in
  * q_scale, k_scale ([B, heads, nt_max], tile_scale_elems): with amax the
- * tile's largest magnitude, code = e4m3(x * (448 / amax)) (fp32 product,
- * round to nearest even, saturating) and scale = amax / 448 (fp32; 1 for an
- * all-zero tile).
+ * tile's largest magnitude, scale = amax / 448 (fp32; 1 for an all-zero tile)
+ * and code = e4m3(x / scale) (correctly rounded fp32 division, then round to
+ * nearest even, saturating).
  * head_dim 128 only (VSA_ERR_UNSUPPORTED otherwise). */
 VSA_API vsa_status vsa_tile_pack_pool_fp8(vsa_plan* plan, const void* q, const void* k, const void* v,
                                   void* qp, void* kp, void* vp, void* qp8, void* kp8, float* q_scale,
@@ -293,8 +315,8 @@ VSA_API vsa_status vsa_tile_pack_pool_fp8(vsa_plan* plan, const void* q, const v
  * fp32 on the tensor cores; P and V stay bf16. qp8, kp8, q_scale, k_scale as
  * written by vsa_tile_pack_pool_fp8; vp the bf16 packed V. head_dim 128. */
 VSA_API vsa_status vsa_sparse_attn_fp8(vsa_plan* plan, const void* qp8, const void* kp8, const float* q_scale,
-                               const float* k_scale, const void* vp, const int32_t* idx, void* op,
-                               float* lse, void* stream);
+                               const float* k_scale, const void* vp, const int32_t* idx, const int32_t* k_per_head,
+                               void* op, float* lse, void* stream);
 
 /* Teacher tile map (row f3; the first stage of the Veda method: full attention,
  * max-pooled per tile pair, is the teacher distribution at tile level -- Veda
@@ -313,14 +335,14 @@ VSA_API vsa_status vsa_teacher_tiles(vsa_plan* plan, const void* qp, const void*
                              float* teacher, void* stream);
 
 /* For every (batch, head, video query tile) row of two index tables
- * ([B, heads, ntv_max, k_max] int32, ascending rows of the head's k, as
- * vsa_topk_select writes them): the number of indices the rows share, in
+ * ([B, heads, ntv_max, k_max] int32, ascending rows of k[h] entries, k from
+ * k_per_head as for vsa_topk_select): the number of indices the rows share, in
  * counts [B, heads, ntv_max] (0 for rows past a head's ntv). With a = the
  * scorer's selection and b = the teacher's top-k, counts / k is the tile
  * recall of the scorer (BSAI VedaSparse README, "Core Technology": TripPool
  * tile recall against full attention). */
 VSA_API vsa_status vsa_index_overlap(vsa_plan* plan, const int32_t* idx_a, const int32_t* idx_b,
-                             int32_t* counts, void* stream);
+                             const int32_t* k_per_head, int32_t* counts, void* stream);
 
 /* The whole layer in order on one stream, on caller-provided buffers (sizes
  * from vsa_plan_query): vsa_tile_pack_pool, vsa_tile_score_pooled,
@@ -332,6 +354,23 @@ VSA_API vsa_status vsa_layer_forward(vsa_plan* plan, const void* q, const void* 
                              const float* proj_q, const float* proj_k,
                              void* qp, void* kp, void* vp, float* scores, int32_t* idx,
                              void* op, float* lse, void* workspace, void* o, void* stream);
+
+/* Bound of every device-side wait of the plan's tcgen05 kernels (attention,
+ * teacher map), in nanoseconds: 1,000 .. 60,000,000,000; 0 restores the
+ * default of two seconds. A kernel whose wait runs past it stops: it latches
+ * VSA_ERR_DEVICE_TIMEOUT (returned by vsa_plan_check), lets its own copies and
+ * tensor-core work finish, frees its tensor memory and returns, leaving the
+ * CUDA context usable (fail loudly, never hang: "From 650 s to 72 s", "What
+ * transfers"). Host-side setting, read at each launch. */
+VSA_API vsa_status vsa_plan_set_wait_limit(vsa_plan* plan, uint64_t limit_ns);
+
+/* Test hook for the timeout path above; no counterpart on the pages. With
+ * on = 1, every later attention launch of this plan has its softmax warps,
+ * after their first block of scores, wait on a barrier that nothing arrives
+ * on, so each CTA runs into the wait limit and takes the abort path with
+ * copies and tensor-core work in flight. on = 0 (the default) turns it off.
+ * Not for production use. */
+VSA_API vsa_status vsa_plan_set_test_hold(vsa_plan* plan, int32_t on);
 
 /* Waits for the plan's device (cudaDeviceSynchronize), then returns and clears
  * the latched device error (VSA_OK if none), or VSA_ERR_CUDA if the device

@@ -16,12 +16,28 @@ that is, while the current phase's parity differs from p. A waiter that falls
 two phases behind therefore waits for good: that is the aliasing the model
 looks for.
 
-Items are given as their key-block counts. `slot_readers_release` models the
-list-slot barrier counting every role that reads the slot (13 arrivals)
-instead of the eight softmax warps alone. `faults` plants protocol mistakes
-(the tests check that the model catches them): "s_skips_pv_done" (the S issuer
-reuses an S buffer without waiting for the PVs that read its P) and
-"softmax_parity" (the softmax waits on the wrong phase parity).
+Items are given as their key-block counts. `slot_readers_release` (the
+kernel's counts) has the list-slot barrier count every role that reads the
+slot (13 arrivals); False models the earlier kernel, whose barrier counted the
+eight softmax warps alone. `faults` plants protocol mistakes (the tests check
+that the model catches them): "s_skips_pv_done" (the S issuer reuses an S
+buffer without waiting for the PVs that read its P) and "softmax_parity" (the
+softmax waits on the wrong phase parity), "mma_no_drain" and "tma_no_drain"
+(the MMA issuers or the producer lanes leave without draining).
+
+Bounded waits and the abort path: every wait of the kernel gives up after a
+time limit. When no role can move and nothing is in flight, the model lets one
+waiting role run out of time: it raises the abort flag. From then on a wait
+whose phase has not completed returns false and the role leaves its loop (a
+wait whose phase has completed still returns true, as try_wait does). On the
+way out the producer lanes wait for their own copies in flight, and each MMA
+issuer commits to the drain barrier (counted by the three issuers) and waits
+for it, so that no copy or MMA is in flight when the CTA ends and frees its
+tensor memory; the model raises Hazard otherwise. `hold` models the kernel's
+test hold: the softmax warps wait, at their first block, on a barrier nothing
+arrives on. `timeout_p` lets a wait that has not passed run out early, with
+probability timeout_p per step, while copies and MMAs are still in flight (a
+limit shorter than a copy's latency, as a caller may set one).
 """
 from __future__ import annotations
 
@@ -54,9 +70,11 @@ def _check(cond, msg):
         raise Hazard(msg)
 
 
-def run(blocks_per_item, rng, slot_readers_release=False, starve=(), faults=(), max_steps=1_000_000):
+def run(blocks_per_item, rng, slot_readers_release=True, starve=(), faults=(), hold=False, timeout_p=0.0,
+        max_steps=1_000_000):
     n_items = len(blocks_per_item)
-    bars = {"QFULL": Bar(1), "QEMPTY": Bar(1), "OFULL": Bar(2), "OFREE": Bar(8), "LX": Bar(8)}
+    bars = {"QFULL": Bar(1), "QEMPTY": Bar(1), "OFULL": Bar(2), "OFREE": Bar(8), "LX": Bar(8),
+            "HOLD": Bar(1), "DRAIN": Bar(3)}
     for i in range(K_STAGES):
         bars[f"KFULL{i}"], bars[f"KEMPTY{i}"] = Bar(1), Bar(1)
     for i in range(V_STAGES):
@@ -71,6 +89,7 @@ def run(blocks_per_item, rng, slot_readers_release=False, starve=(), faults=(), 
     st = {"info": [None, None], "Q": None, "q_free": -1, "K": [None] * K_STAGES, "V": [None] * V_STAGES,
           "S": [None] * S_BUFS, "s_done": -1, "pv_done": [-1, -1], "epilogue_done": -1, "epi": {}}
     pending = []   # (issuer, completion)
+    flags = {"abort": False}
 
     def later(issuer, fn):
         pending.append((issuer, fn))
@@ -78,10 +97,18 @@ def run(blocks_per_item, rng, slot_readers_release=False, starve=(), faults=(), 
     def wait(name, parity):
         return name, parity
 
+    def drain_copies(issuer):       # a producer lane waits for its own copies in flight
+        return "copies", issuer
+
+    def drain_mmas(issuer):         # an MMA issuer: commit to DRAIN, then wait for all three commits
+        later(issuer, lambda: bars["DRAIN"].arrive())
+        return "drain", 0
+
     def scheduler():
         for it in range(n_items + 1):
             slot = it & 1
-            yield wait(f"LEMPTY{slot}", ((it >> 1) & 1) ^ 1)
+            if not (yield wait(f"LEMPTY{slot}", ((it >> 1) & 1) ^ 1)):
+                return
             st["info"][slot] = (it, blocks_per_item[it]) if it < n_items else None
             for _ in range(32):
                 bars[f"LFULL{slot}"].arrive()
@@ -91,19 +118,23 @@ def run(blocks_per_item, rng, slot_readers_release=False, starve=(), faults=(), 
     def producer(is_k):
         g, stage, ph = 0, 0, 0
         n_st = K_STAGES if is_k else V_STAGES
+        ok = True
         for it in range(n_items + 1):
             slot = it & 1
-            yield wait(f"LFULL{slot}", (it >> 1) & 1)
+            if not (ok := (yield wait(f"LFULL{slot}", (it >> 1) & 1))):
+                break
             info = st["info"][slot]
             if info is None:
-                return
+                break
             _check(info[0] == it, f"{'K' if is_k else 'V'} producer took item {info[0]} for {it}")
             if is_k:
-                yield wait("QEMPTY", (it & 1) ^ 1)
+                if not (ok := (yield wait("QEMPTY", (it & 1) ^ 1))):
+                    break
                 _check(st["q_free"] >= it - 1, "Q reloaded while in use")
                 later("tmaK", lambda it=it: (st.__setitem__("Q", it), bars["QFULL"].arrive()))
             for _ in range(info[1]):
-                yield wait(f"{'K' if is_k else 'V'}EMPTY{stage}", ph ^ 1)
+                if not (ok := (yield wait(f"{'K' if is_k else 'V'}EMPTY{stage}", ph ^ 1))):
+                    break
                 consumed = st["s_done"] if is_k else min(st["pv_done"])
                 _check(consumed >= g - n_st, f"stage {stage} reloaded before block {g - n_st} was used")
 
@@ -114,31 +145,41 @@ def run(blocks_per_item, rng, slot_readers_release=False, starve=(), faults=(), 
                 g, stage = g + 1, stage + 1
                 if stage == n_st:
                     stage, ph = 0, ph ^ 1
+            if not ok:
+                break
             if slot_readers_release:
                 bars[f"LEMPTY{slot}"].arrive()
+        if flags["abort"] and "tma_no_drain" not in faults:
+            yield drain_copies("tmaK" if is_k else "tmaV")
 
     def s_issuer():
         kst, kph, sb, su, g = 0, 0, 0, 0, 0
+        ok = True
         for it in range(n_items + 1):
             slot = it & 1
-            yield wait(f"LFULL{slot}", (it >> 1) & 1)
+            if not (ok := (yield wait(f"LFULL{slot}", (it >> 1) & 1))):
+                break
             info = st["info"][slot]
             if info is None:
-                return
+                break
             _check(info[0] == it, f"S issuer took item {info[0]} for {it}")
             nblk = info[1]
             if slot_readers_release:
                 bars[f"LEMPTY{slot}"].arrive()
-            yield wait("QFULL", it & 1)
+            if not (ok := (yield wait("QFULL", it & 1))):
+                break
             _check(st["Q"] == it, "S reads a stale Q")
             if nblk == 0:
                 later("S", lambda it=it: (st.__setitem__("q_free", it), bars["QEMPTY"].arrive()))
             for j in range(nblk):
-                yield wait(f"KFULL{kst}", kph)
+                if not (ok := (yield wait(f"KFULL{kst}", kph))):
+                    break
                 _check(st["K"][kst] == g, f"S({g}) reads K stage {kst} holding {st['K'][kst]}")
                 if su > 0 and "s_skips_pv_done" not in faults:   # P of block g - 2 sits in this buffer
-                    yield wait(f"PDONE0_{sb}", (su - 1) & 1)
-                    yield wait(f"PDONE1_{sb}", (su - 1) & 1)
+                    if not (ok := (yield wait(f"PDONE0_{sb}", (su - 1) & 1))):
+                        break
+                    if not (ok := (yield wait(f"PDONE1_{sb}", (su - 1) & 1))):
+                        break
                 _check(min(st["pv_done"]) >= g - S_BUFS, f"S({g}) overwrites P({g - S_BUFS}) before PV read it")
 
                 def land(sb=sb, g=g, kst=kst, last=(j == nblk - 1), it=it):
@@ -154,27 +195,36 @@ def run(blocks_per_item, rng, slot_readers_release=False, starve=(), faults=(), 
                     kst, kph = 0, kph ^ 1
                 if sb == S_BUFS:
                     sb, su = 0, su + 1
+            if not ok:
+                break
+        if "mma_no_drain" not in faults:
+            yield drain_mmas("S")
 
     def pv_issuer(w):
         vst, vph, sb, su, g = 0, 0, 0, 0, 0
+        ok = True
         for it in range(n_items + 1):
             slot = it & 1
-            yield wait(f"LFULL{slot}", (it >> 1) & 1)
+            if not (ok := (yield wait(f"LFULL{slot}", (it >> 1) & 1))):
+                break
             info = st["info"][slot]
             if info is None:
-                return
+                break
             _check(info[0] == it, f"PV{w} took item {info[0]} for {it}")
             nblk = info[1]
             if slot_readers_release:
                 bars[f"LEMPTY{slot}"].arrive()
-            yield wait("OFREE", (it & 1) ^ 1)
+            if not (ok := (yield wait("OFREE", (it & 1) ^ 1))):
+                break
             _check(st["epilogue_done"] >= it - 1, f"PV{w} overwrites O before the epilogue of item {it - 1}")
             if nblk == 0:
                 later(f"PV{w}", lambda: bars["OFULL"].arrive())
             for j in range(nblk):
-                yield wait(f"VFULL{vst}", vph)
+                if not (ok := (yield wait(f"VFULL{vst}", vph))):
+                    break
                 _check(st["V"][vst] == g, f"PV{w}({g}) reads V stage {vst} holding {st['V'][vst]}")
-                yield wait(f"PFULL{w}_{sb}", su & 1)
+                if not (ok := (yield wait(f"PFULL{w}_{sb}", su & 1))):
+                    break
                 _check(st["S"][sb] == g, f"PV{w}({g}) reads P in S buffer {sb} holding block {st['S'][sb]}")
 
                 def land(w=w, g=g, vst=vst, sb=sb, last=(j == nblk - 1)):
@@ -189,29 +239,40 @@ def run(blocks_per_item, rng, slot_readers_release=False, starve=(), faults=(), 
                     vst, vph = 0, vph ^ 1
                 if sb == S_BUFS:
                     sb, su = 0, su + 1
+            if not ok:
+                break
+        if "mma_no_drain" not in faults:
+            yield drain_mmas(f"PV{w}")
 
     def softmax_warp(sg):
         g = 0
         for it in range(n_items + 1):
             slot = it & 1
-            yield wait(f"LFULL{slot}", (it >> 1) & 1)
+            if not (yield wait(f"LFULL{slot}", (it >> 1) & 1)):
+                return
             info = st["info"][slot]
             if info is None:
                 return
             _check(info[0] == it, f"softmax took item {info[0]} for {it}")
             for j in range(info[1]):
                 sbuf = g % S_BUFS
-                yield wait(f"SFULL{sbuf}", ((g // S_BUFS) + ("softmax_parity" in faults)) & 1)
+                if not (yield wait(f"SFULL{sbuf}", ((g // S_BUFS) + ("softmax_parity" in faults)) & 1)):
+                    return
                 _check(st["S"][sbuf] == g, f"softmax block {g} reads S buffer holding {st['S'][sbuf]}")
+                if hold and g == 0 and not (yield wait("HOLD", 0)):
+                    return
                 if j > 0 and rng.random() < 0.2:   # the O rescale waits for its previous PV
-                    yield wait(f"PDONE{sg}_{(g - 1) % S_BUFS}", ((g - 1) // S_BUFS) & 1)
+                    if not (yield wait(f"PDONE{sg}_{(g - 1) % S_BUFS}", ((g - 1) // S_BUFS) & 1)):
+                        return
                     _check(st["pv_done"][sg] >= g - 1, "O rescaled while the previous PV accumulates")
                 bars[f"PFULL{sg}_{sbuf}"].arrive()
                 g += 1
-            yield wait("OFULL", it & 1)
+            if not (yield wait("OFULL", it & 1)):
+                return
             _check(info[1] == 0 or min(st["pv_done"]) >= g - 1, "epilogue before the item's last PV")
             bars["LX"].arrive()
-            yield wait("LX", it & 1)
+            if not (yield wait("LX", it & 1)):
+                return
             st["epi"][it] = st["epi"].get(it, 0) + 1
             if st["epi"][it] == 8:
                 st["epilogue_done"] = it
@@ -224,29 +285,55 @@ def run(blocks_per_item, rng, slot_readers_release=False, starve=(), faults=(), 
         for wi in range(4):
             roles[f"softmax {sg}.{wi}"] = softmax_warp(sg)
     waiting = {}
+    timed_out = []
 
-    def step(name):
+    def step(name, value):
         try:
-            waiting[name] = next(roles[name])
+            waiting[name] = roles[name].send(value)
         except StopIteration:
             waiting[name] = None
 
+    def resume_value(name):
+        """True: the wait returns true; False: it gives up (abort); None: still waiting."""
+        kind, arg = waiting[name]
+        if kind == "copies":
+            return True if not any(iss == arg for iss, _ in pending) else None
+        if kind == "drain":
+            return True if bars["DRAIN"].passed(arg) else None    # drain waits ignore the abort flag
+        if bars[kind].passed(arg):
+            return True
+        return False if flags["abort"] else None
+
     for name in roles:
-        step(name)
+        step(name, None)
     for _ in range(max_steps):
         live = [k for k, v in waiting.items() if v is not None]
-        if not live and not pending:
-            return "ok"
-        ready = [("role", k) for k in live if bars[waiting[k][0]].passed(waiting[k][1])]
+        if not live:
+            # every thread has reached the end of the kernel: TMEM is freed, the CTA exits
+            _check(not pending, "the CTA ends with copies or MMAs in flight: " + ", ".join(i for i, _ in pending))
+            return "ok" if not flags["abort"] else "aborted: " + timed_out[0]
+        if not flags["abort"] and timeout_p and rng.random() < timeout_p:
+            blocked = [k for k in live if resume_value(k) is None]
+            if blocked:                     # a wait runs out with work still in flight
+                k = rng.choice(blocked)
+                timed_out.append(f"{k} waits {waiting[k][0]} parity {waiting[k][1]} (early)")
+                flags["abort"] = True
+        ready = [("role", k) for k in live if resume_value(k) is not None]
         issuers = list(dict.fromkeys(iss for iss, _ in pending))
         choices = ready + [("done", i) for i in issuers]
         preferred = [c for c in choices if c[1] not in starve]
         choices = preferred or choices
         if not choices:
-            return "deadlock: " + "; ".join(f"{k} waits {waiting[k][0]} parity {waiting[k][1]}" for k in live)
+            stuck = "; ".join(f"{k} waits {waiting[k][0]} parity {waiting[k][1]}" for k in live)
+            if flags["abort"]:
+                return "deadlock after abort: " + stuck
+            # nothing can move: one bounded wait runs out and raises the abort flag
+            timed_out.append(stuck)
+            flags["abort"] = True
+            continue
         kind, who = rng.choice(choices)
         if kind == "role":
-            step(who)
+            step(who, resume_value(who))
         else:
             idx = next(i for i, (iss, _) in enumerate(pending) if iss == who)
             pending.pop(idx)[1]()

@@ -165,7 +165,7 @@ def test_null_arguments(lib):
     assert lib.vsa_plan_create(ctypes.byref(_desc()), None) == 1
     assert lib.vsa_plan_destroy(None) == 0
     assert lib.vsa_tile_pack(None, None, None, None, None, None, None, None) == 1
-    assert lib.vsa_sparse_attn(None, None, None, None, None, None, None, None) == 1
+    assert lib.vsa_sparse_attn(None, None, None, None, None, None, None, None, None) == 1
     assert lib.vsa_plan_check(None) == 1
     assert lib.vsa_plan_query(None, None) == 1
 
@@ -180,5 +180,9 @@ def test_every_compute_call_rejects_a_null_plan(lib):
         first = m.group(1).split(",")[0]
         if "vsa_plan*" not in first.replace(" ", "") or name in ("vsa_plan_destroy",):
             continue
-        args = [None] * n
-        assert getattr(lib, name)(*args) == 1, name   # VSA_ERR_INVALID_ARG
+        f = getattr(lib, name)
+        # NULL for pointers, 0 for integer arguments
+        args = [0 if t in (ctypes.c_int32, ctypes.c_uint64, ctypes.c_int64, ctypes.c_double) else None
+                for t in f.argtypes]
+        assert len(args) == n, name
+        assert f(*args) == 1, name   # VSA_ERR_INVALID_ARG

@@ -36,7 +36,7 @@ def _line(args, cfg):
     e2e = {"value": 66.965, "unit": "ms", "h2d_bytes_per_step": 3 * 691273728, "d2h_bytes_per_step": 691273728}
     clocks = {"sm_mhz": 1650.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
     stats = {"computed_pairs": 3151, "dense_pairs": 10000}
-    return bench.bench_line(args, cfg, 1, ks, flops, ms_step, STAGES, roof, e2e, clocks, stats, None), peaks
+    return bench.bench_line(args, cfg, 1, ks, flops, ms_step, STAGES, roof, e2e, clocks, stats, []), peaks
 
 
 def test_line_has_every_key_and_reproduces_the_recorded_run():
@@ -52,8 +52,9 @@ def test_line_has_every_key_and_reproduces_the_recorded_run():
     r = line["roofline"]
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["algorithmic_flops_per_launch"] == O.attention_flops(cfg, _ks(cfg, 0.75))
-    if peaks["source"] == "measured" and peaks["bf16_tflops_sustained"] == 1387.5:
-        assert r["achieved"] == 826.3 and r["frac"] == 0.5956      # the committed bench line's figures
+    if peaks["source"] == "measured" and peaks["bf16_tflops"] == 1656.9:
+        assert r["achieved"] == 826.3 and r["frac"] == 0.4987      # the committed bench line's figures
+        assert r["frac_of_sustained_peak"] == 0.5956
     assert r["frac"] == pytest.approx(r["achieved"] / r["peak"], abs=1e-3)
     traffic = bench.measured_traffic("full", 0.75, 24)
     assert r["traffic"] == traffic
@@ -65,7 +66,7 @@ def test_fp8_line_uses_the_mixed_peak_and_no_traffic():
     cfg = get_config("full")
     line, peaks = _line(_args(fp8=True), cfg)
     r = line["roofline"]
-    assert r["peak"] == round(peaks["bf16_tflops_sustained"] * 4 / 3, 1)
+    assert r["peak"] == round(peaks["bf16_tflops"] * 4 / 3, 1)
     assert r["traffic"] is None and "e4m3" in r["peak_kind"]
 
 
@@ -90,3 +91,26 @@ def test_clock_summary_reads_nvidia_smi_rows():
     hot = rows[1].replace("Not Active, Not Active, Not Active, Active", "Active, Not Active, Active, Not Active")
     assert bench.summarize_clocks([hot])["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     assert bench.summarize_clocks([])["reasons"] == ["no samples"]
+
+
+def test_heads_split_line_is_one_layer_strong_scaling():
+    """With the heads of one layer split over 4 ranks, a step is that one layer: the value is the
+    slowest rank's step time (not divided by the ranks) and the scaling is strong."""
+    cfg = get_config("full")
+    args = _args(split="heads")
+    ks = _ks(cfg, 0.75)
+    flops = bench.attention_flops(cfg, ks)
+    roof = bench.attn_roofline(args, cfg, bench.measured_peaks(), flops, STAGES["attn"] / 4)
+    line = bench.bench_line(args, cfg, 4, ks, flops, 16.0, STAGES, roof, None, None,
+                            {"computed_pairs": 1, "dense_pairs": 2}, [])
+    assert line["value"] == 16.0 and line["scaling"] == "strong" and line["n_gpus"] == 4
+    assert line["config"]["layers_per_step"] == 1 and "heads" in line["config"]["parallelism"]
+    weak = bench.bench_line(_args(), cfg, 4, ks, flops, 16.0, STAGES, roof, None, None,
+                            {"computed_pairs": 1, "dense_pairs": 2}, [])
+    assert weak["value"] == 4.0 and weak["scaling"] == "weak"
+
+
+def test_other_workloads_name_their_own_metric():
+    assert bench.metric_for(get_config("full")) == bench.METRIC
+    m = bench.metric_for(get_config("long"))
+    assert "long" in m and "230400" in m

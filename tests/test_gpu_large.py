@@ -97,6 +97,23 @@ def test_long_clip_dense_and_sparse():
     sampled_parity(r2, heads=[3], n_video_samples=3)
 
 
+_long_inputs = {}
+
+
+@pytest.mark.parametrize("sparsity", [0.5, 0.75, 0.95])
+def test_long_clip_sweep(sparsity):
+    """The rest of the long clip's sparsity sweep (0 and 0.9 above), on sampled rows."""
+    cfg = get_config("long")
+    if "inp" not in _long_inputs:
+        from vsa_synth import make_layer_inputs
+        _long_inputs["inp"] = make_layer_inputs(cfg)
+    r = LayerRun(cfg, sparsity, inputs=_long_inputs["inp"]).run(fused=True)
+    all_rows_valid(r)
+    sampled_parity(r, heads=[11], n_video_samples=3)
+    want_pairs = O.attention_flops(cfg, r.k) // (4 * cfg.head_dim)
+    assert r.plan.stats()["computed_pairs"] == want_pairs
+
+
 def test_full_clip_fp8():
     """The fp8 Q K^T path at full size, against the oracle's fp8 model on sampled rows."""
     import torch

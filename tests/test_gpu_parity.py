@@ -168,7 +168,7 @@ def test_argument_errors():
     import tile_sparse_video_pack_b200 as T
     import torch
     r = gpu_run("tiny")
-    assert T.vsa.library().vsa_sparse_attn(r.plan._h, None, None, None, None, None, None, None) == 1
+    assert T.vsa.library().vsa_sparse_attn(r.plan._h, None, None, None, None, None, None, None, None) == 1
     with pytest.raises(TypeError):
         r.plan.tile_pack(r.q.float(), None, None, r.bufs["qp"], None, None)
     with pytest.raises(ValueError):

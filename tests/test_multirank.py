@@ -70,10 +70,12 @@ def test_reference_arm_prints_the_same_metric_and_config():
     cfg = get_config("tiny")
     pt, ph, pw = cfg.tile_shapes[0]
     k0 = O.k_from_sparsity(cfg.sparsity[0], -(-cfg.T // pt) * -(-cfg.H // ph) * -(-cfg.W // pw))
-    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "ms"
+    assert d["impl"] == "reference" and d["metric"] == bench.metric_for(cfg) and d["unit"] == "ms"
     assert d["higher_is_better"] is False and d["value"] > 0
     assert d["config"] == bench.workload_config(cfg, cfg.sparsity[0], k0, 1)
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    # the steps it ran were samples of the layer, and the line says the value is extrapolated
+    assert d["extrapolated"] is True and d["steps"] == 1 and 0 < d["ms_per_step"] < 600e3
     assert d["e2e"] == {"value": d["value"], "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 

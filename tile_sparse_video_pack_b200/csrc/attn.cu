@@ -155,7 +155,7 @@ enum {
   B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KEMPTY0 = B_KFULL0 + 4, B_VFULL0 = B_KEMPTY0 + 4, B_VEMPTY0 = B_VFULL0 + 4,
   // P_FULL / P_DONE: [softmax warpgroup][S buffer]
   B_SFULL0 = B_VEMPTY0 + 4, B_PFULL0 = B_SFULL0 + kSBuf, B_PDONE0 = B_PFULL0 + 2 * kSBuf,
-  B_LFULL0 = B_PDONE0 + 2 * kSBuf, B_LFULL1, B_LEMPTY0, B_LEMPTY1, B_OFULL, B_OFREE, B_LX, B_DRAIN, B_COUNT
+  B_LFULL0 = B_PDONE0 + 2 * kSBuf, B_LFULL1, B_LEMPTY0, B_LEMPTY1, B_OFULL, B_OFREE, B_LX, B_DRAIN, B_HOLD, B_COUNT
 };
 static_assert(B_COUNT <= 40, "barrier slots");
 
@@ -181,6 +181,8 @@ struct AttnParams {
   int32_t k[VSA_MAX_HEADS];
   int32_t n_ref, k_ref_max;
   int32_t k_ref[VSA_MAX_HEADS];
+  uint64_t wait_ns;        // bound of every mbarrier wait
+  int32_t hold;            // test hook: the softmax waits, at its first block, on a barrier nothing arrives on
 };
 
 __device__ __forceinline__ int warp_excl_scan(int v, int lane, int* total) {
@@ -234,12 +236,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_LFULL0 + i), 32);
-      mbar_init(bar(B_LEMPTY0 + i), kSmWarps);
+      mbar_init(bar(B_LEMPTY0 + i), kSmWarps + 5);   // + S issuer, two PV issuers, two producer lanes
     }
     mbar_init(bar(B_OFULL), 2);
     mbar_init(bar(B_OFREE), kSmWarps);
     mbar_init(bar(B_LX), kSmWarps);
     mbar_init(bar(B_DRAIN), 3);   // the three MMA issuers
+    mbar_init(bar(B_HOLD), 1);    // test hook: never arrived on
     misc[1] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (uint32_t it = 0;; ++it) {
       const int slot = it & 1;
       bool ok = true;
-      if (lane == 0) ok = wait_bar(bar(B_LEMPTY0 + slot), ((it >> 1) & 1) ^ 1, abort_flag, gerr);
+      if (lane == 0) ok = wait_bar(bar(B_LEMPTY0 + slot), ((it >> 1) & 1) ^ 1, abort_flag, gerr, prm.wait_ns);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       long long item = 0;
@@ -417,13 +420,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issuedQ = 0;    // Q loads issued
       for (uint32_t it = 0;; ++it) {
         const int slot = it & 1;
-        if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr)) break;
+        if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr, prm.wait_ns)) break;
         const ItemInfo inf = info[slot];
         if (inf.end) break;
         const uint32_t* list = lists + slot * prm.list_cap;
         const int row_base = inf.bh * prm.nt_max;
         if (is_k) {   // rows 0-63: tile qa, rows 64-127: tile qb (qa again when there is none)
-          if (!wait_bar(bar(B_QEMPTY), (it & 1) ^ 1, abort_flag, gerr)) break;
+          if (!wait_bar(bar(B_QEMPTY), (it & 1) ^ 1, abort_flag, gerr, prm.wait_ns)) break;
           mbar_expect_tx(bar(B_QFULL), 2 * (F8 ? 1 : D / 64) * kTileBytes);
           const int qb = inf.qb >= 0 ? inf.qb : inf.qa;
           for (int c = 0; c < (F8 ? 1 : D / 64); ++c) {   // 64-row boxes of 128 bytes per row
@@ -437,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < nblk; ++j) {
           const int ta = int(list[2 * j] & 0xFFFFu);
           const int tb = 2 * j + 1 < inf.n_entries ? int(list[2 * j + 1] & 0xFFFFu) : ta;
-          if (!(ok = wait_bar(bar(empty0 + st), ph ^ 1, abort_flag, gerr))) break;
+          if (!(ok = wait_bar(bar(empty0 + st), ph ^ 1, abort_flag, gerr, prm.wait_ns))) break;
           mbar_expect_tx(bar(full0 + st), 2 * (is_k && F8 ? 1 : D / 64) * kTileBytes);
           if (is_k) {   // K-major: tile a rows 0-63, tile b rows 64-127 of each 128-byte half
             const uint32_t sk = sbase + L::oK + st * L::kKBytes;
@@ -459,6 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
+        mbar_arrive(bar(B_LEMPTY0 + slot));   // this lane is done with the slot's list
       }
       if (*abort_flag) {
         // let every copy this thread issued land before shared memory is released
@@ -482,17 +486,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (uint32_t it = 0; ok; ++it) {
         const int slot = it & 1;
-        if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr)) break;
+        if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr, prm.wait_ns)) break;
         const ItemInfo inf = info[slot];
         if (inf.end) break;
-        if (!wait_bar(bar(B_QFULL), it & 1, abort_flag, gerr)) break;
+        mbar_arrive(bar(B_LEMPTY0 + slot));     // the item's info is copied
+        if (!wait_bar(bar(B_QFULL), it & 1, abort_flag, gerr, prm.wait_ns)) break;
         const int nblk = (inf.n_entries + 1) >> 1;
         if (nblk == 0) tc_commit(bar(B_QEMPTY));   // a rejected item without prefix tiles
         for (int j = 0; j < nblk; ++j) {
-          if (!(ok = wait_bar(bar(B_KFULL0 + kst), kph, abort_flag, gerr))) break;
+          if (!(ok = wait_bar(bar(B_KFULL0 + kst), kph, abort_flag, gerr, prm.wait_ns))) break;
           // the buffer's previous P has been read by both PV MMAs
-          if (su > 0 && !(ok = wait_bar(bar(B_PDONE0 + sb), (su - 1) & 1, abort_flag, gerr))) break;
-          if (su > 0 && !(ok = wait_bar(bar(B_PDONE0 + kSBuf + sb), (su - 1) & 1, abort_flag, gerr))) break;
+          if (su > 0 && !(ok = wait_bar(bar(B_PDONE0 + sb), (su - 1) & 1, abort_flag, gerr, prm.wait_ns))) break;
+          if (su > 0 && !(ok = wait_bar(bar(B_PDONE0 + kSBuf + sb), (su - 1) & 1, abort_flag, gerr, prm.wait_ns))) break;
           tc_fence_after();
           const uint64_t dk = dk0 + ((kst * L::kKBytes) >> 4);
           if constexpr (F8) {
@@ -539,17 +544,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (uint32_t it = 0; ok; ++it) {
         const int slot = it & 1;
-        if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr)) break;
+        if (!wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr, prm.wait_ns)) break;
         const ItemInfo inf = info[slot];
         if (inf.end) break;
+        mbar_arrive(bar(B_LEMPTY0 + slot));     // the item's info is copied
         const int nblk = (inf.n_entries + 1) >> 1;
         // O is free once the previous item's epilogue has read it
-        if (!wait_bar(bar(B_OFREE), (it & 1) ^ 1, abort_flag, gerr)) break;
+        if (!wait_bar(bar(B_OFREE), (it & 1) ^ 1, abort_flag, gerr, prm.wait_ns)) break;
         if (nblk == 0) tc_commit(bar(B_OFULL));    // nothing to accumulate; the epilogue skips it
         for (int j = 0; j < nblk; ++j) {
-          if (!(ok = wait_bar(bar(B_VFULL0 + vst), vph, abort_flag, gerr))) break;
+          if (!(ok = wait_bar(bar(B_VFULL0 + vst), vph, abort_flag, gerr, prm.wait_ns))) break;
           const uint64_t dv = dv0 + ((vst * L::kVBytes) >> 4);
-          if (!(ok = wait_bar(bar(B_PFULL0 + w * kSBuf + sb), su & 1, abort_flag, gerr))) break;
+          if (!(ok = wait_bar(bar(B_PFULL0 + w * kSBuf + sb), su & 1, abort_flag, gerr, prm.wait_ns))) break;
           tc_fence_after();
           const uint32_t pcol = tS + sb * 128 + w * 64;
 #pragma unroll
@@ -598,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (uint32_t it = 0; ok; ++it) {
       const int slot = it & 1;
-      ok = wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr);
+      ok = wait_bar(bar(B_LFULL0 + slot), (it >> 1) & 1, abort_flag, gerr, prm.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       const ItemInfo inf = info[slot];
       if (inf.end) break;
@@ -609,8 +615,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sbuf = int(g % kSBuf);           // S / P buffer
         const uint32_t sph = (g / kSBuf) & 1;      // its phase
         const uint32_t tSb = tS + sbuf * 128 + lane_off + 64 * sg;
-        ok = wait_bar(bar(B_SFULL0 + sbuf), sph, abort_flag, gerr);
+        ok = wait_bar(bar(B_SFULL0 + sbuf), sph, abort_flag, gerr, prm.wait_ns);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        if (prm.hold && g == 0) {   // test hook: wait for a release that nothing gives, until the limit
+          ok = wait_bar(bar(B_HOLD), 0, abort_flag, gerr, prm.wait_ns);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        }
         tc_fence_after();
         const int ei = 2 * j + sg;
         const uint32_t e = ei < inf.n_entries ? list[ei] : 0u;
@@ -693,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // once my previous PV has finished accumulating into it
         if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
           const uint32_t gp = g - 1;
-          ok = wait_bar(bar(B_PDONE0 + sg * kSBuf + int(gp % kSBuf)), (gp / kSBuf) & 1, abort_flag, gerr);
+          ok = wait_bar(bar(B_PDONE0 + sg * kSBuf + int(gp % kSBuf)), (gp / kSBuf) & 1, abort_flag, gerr, prm.wait_ns);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
@@ -716,13 +726,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // done. Row r's two partial softmaxes (m_0, l_0, O_0) and (m_1, l_1, O_1)
       // merge as O = sum_w 2^(m_w - M) O_w / sum_w 2^(m_w - M) l_w, M = max m_w;
       // warpgroup sg writes channels [sg D/2, (sg+1) D/2).
-      ok = wait_bar(bar(B_OFULL), it & 1, abort_flag, gerr);
+      ok = wait_bar(bar(B_OFULL), it & 1, abort_flag, gerr, prm.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       xm[sg * 128 + r] = m;
       xl[sg * 128 + r] = l;
       warp_arrive(bar(B_LX));
-      ok = wait_bar(bar(B_LX), it & 1, abort_flag, gerr);
+      ok = wait_bar(bar(B_LX), it & 1, abort_flag, gerr, prm.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       const float m0 = xm[r], m1 = xm[128 + r];
       const float mrow = fmaxf(m0, m1);
@@ -787,8 +797,8 @@ int attn_smem_bytes(int list_cap) {
 }
 
 cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp, const int32_t* idx,
-                        const int32_t* idx_ref, void* op, float* lse, cudaStream_t s, const float* q_scale,
-                        const float* k_scale) {
+                        const int32_t* idx_ref, const int32_t* k, void* op, float* lse, cudaStream_t s,
+                        const float* q_scale, const float* k_scale) {
   const Geometry& g = p->geo;
   const int64_t rows = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE;
   const bool f8 = q_scale != nullptr;      // qp, kp are e4m3 tiles with per-tile scales
@@ -822,9 +832,11 @@ cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void*
   prm.lists = p->d_lists;
   prm.bitmaps = p->d_lists + size_t(p->num_sms) * 2 * p->list_cap;
   prm.scale_log2 = p->desc.softmax_scale * 1.4426950408889634f;
+  prm.wait_ns = p->wait_ns;
+  prm.hold = p->test_hold;
   for (int h = 0; h < VSA_MAX_HEADS; ++h) {
     prm.ntv[h] = h < g.Hh ? g.ntv[h] : 0;
-    prm.k[h] = h < g.Hh ? g.k[h] : 0;
+    prm.k[h] = h < g.Hh ? k[h] : 0;
     prm.k_ref[h] = h < g.Hh ? g.k_ref[h] : 0;
   }
   // reset the work counter and the pair count

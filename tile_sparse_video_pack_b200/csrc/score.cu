@@ -375,7 +375,9 @@ void* g_static_scratch_addr[256] = {};   // device address per device ordinal
 
 // Device address of the scratch array on the current device. The host-side
 // symbol is only a stand-in: its device address comes from
-// cudaGetSymbolAddress, called once per device with that device current.
+// cudaGetSymbolAddress, called with that device current -- by every
+// vsa_plan_create (so a plan made after a device reset gets the new module's
+// address) and, if no plan has done so yet, by the first call here.
 cudaError_t static_scratch_address(int dev, void** out) {
   std::lock_guard<std::mutex> lock(g_static_scratch_mu);
   if (!g_static_scratch_addr[dev]) {
@@ -389,6 +391,17 @@ cudaError_t static_scratch_address(int dev, void** out) {
 }
 
 }  // namespace
+
+cudaError_t refresh_static_scratch_address(int dev) {
+  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+  void* ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_score_scratch);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  g_static_scratch_addr[dev] = ptr;
+  return cudaSuccess;
+}
+
 }  // namespace vsa
 
 extern "C" vsa_status vsa_tile_score_static(vsa_plan* p, const void* qp, const void* kp, const float* proj_q,
@@ -401,6 +414,9 @@ extern "C" vsa_status vsa_tile_score_static(vsa_plan* p, const void* qp, const v
   const auto a16 = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; };
   if (!a16(qp) || !a16(kp) || !a16(proj_q) || !a16(proj_k) || !a16(scores)) return fail(VSA_ERR_INVALID_ARG);
   if (p->info.workspace_bytes > int64_t(vsa::kStaticScoreScratchBytes)) return fail(VSA_ERR_UNSUPPORTED);
+  // R2VA plans continue with vsa_ref_score, which reads the projected pooled Q from the caller's
+  // workspace; here that stays in the library's array, so such plans must use vsa_tile_score
+  if (p->geo.n_ref > 0) return fail(VSA_ERR_UNSUPPORTED);
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     cudaGetLastError();

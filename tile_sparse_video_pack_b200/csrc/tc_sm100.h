@@ -12,7 +12,7 @@
 namespace vsa {
 namespace tc {
 
-constexpr uint64_t kTimeoutNs = 2000000000ull;   // bound of every mbarrier wait (about two seconds)
+constexpr uint64_t kTimeoutNs = kDefaultWaitNs;   // bound of the drain waits after an abort (two seconds)
 
 // ------------------------------------------------------------------ PTX ----
 
@@ -159,16 +159,17 @@ __device__ __forceinline__ void tc_mma_f8(uint32_t d, uint64_t a, uint64_t b, ui
 }
 
 
-// Bounded wait on an mbarrier phase. Returns false on timeout or when another
-// role has aborted; a timeout latches the error and raises the abort flag.
+// Wait on an mbarrier phase for at most limit_ns. Returns false on timeout or
+// when another role has aborted; a timeout latches the error and raises the
+// abort flag.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                         uint32_t* gerr) {
+                                         uint32_t* gerr, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer() - t0 > kTimeoutNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort_flag = 1u;
       atomicOr(gerr, kErrTimeout);
       return false;

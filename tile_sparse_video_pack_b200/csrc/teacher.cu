@@ -60,6 +60,7 @@ struct TeacherParams {
   uint32_t* state;         // [0] error word
   int32_t heads, nt_max, ntv_max, n_pre, pairs_max;   // pairs_max = ceil(ntv_max / 2)
   float scale_log2;
+  uint64_t wait_ns;        // bound of every mbarrier wait
   int32_t ntv[VSA_MAX_HEADS];
 };
 
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
       }
       for (int j = 0; j < nblk && ok; ++j) {
         const int st = j & 1;
-        if (!(ok = wait_bar(bar(T_KEMPTY0 + st), ((j >> 1) & 1) ^ 1, abort_flag, gerr))) break;
+        if (!(ok = wait_bar(bar(T_KEMPTY0 + st), ((j >> 1) & 1) ^ 1, abort_flag, gerr, prm.wait_ns))) break;
         const int ta = 2 * j, tb = 2 * j + 1 < ntv ? 2 * j + 1 : 2 * j;
         mbar_expect_tx(bar(T_KFULL0 + st), 2 * (D / 64) * kTTileBytes);
         const uint32_t sk = sbase + L::oK + st * L::kPairBytes;
@@ -147,11 +148,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
       const uint64_t dq = sw128_desc(sbase + L::oQ, 16, 1024);
       const uint64_t dk0 = sw128_desc(sbase + L::oK, 16, 1024);
-      bool ok = wait_bar(bar(T_QFULL), 0, abort_flag, gerr);
+      bool ok = wait_bar(bar(T_QFULL), 0, abort_flag, gerr, prm.wait_ns);
       for (int j = 0; j < nblk && ok; ++j) {
         const int st = j & 1;                     // K stage and S buffer of block j
-        if (!(ok = wait_bar(bar(T_KFULL0 + st), (j >> 1) & 1, abort_flag, gerr))) break;
-        if (!(ok = wait_bar(bar(T_SEMPTY0 + st), ((j >> 1) & 1) ^ 1, abort_flag, gerr))) break;
+        if (!(ok = wait_bar(bar(T_KFULL0 + st), (j >> 1) & 1, abort_flag, gerr, prm.wait_ns))) break;
+        if (!(ok = wait_bar(bar(T_SEMPTY0 + st), ((j >> 1) & 1) ^ 1, abort_flag, gerr, prm.wait_ns))) break;
         tc_fence_after();
         const uint64_t dk = dk0 + ((st * L::kPairBytes) >> 4);
 #pragma unroll
@@ -183,7 +184,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
     bool ok = true;
     for (int j = 0; j < nblk; ++j) {
       const int st = j & 1;
-      ok = wait_bar(bar(T_SFULL0 + st), (j >> 1) & 1, abort_flag, gerr);
+      ok = wait_bar(bar(T_SFULL0 + st), (j >> 1) & 1, abort_flag, gerr, prm.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       float mx[2];
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(T_RED0 + st));
-      ok = wait_bar(bar(T_RED0 + st), (j >> 1) & 1, abort_flag, gerr);
+      ok = wait_bar(bar(T_RED0 + st), (j >> 1) & 1, abort_flag, gerr, prm.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       if (lane == 0 && half == 0 && vq >= 0) {
 #pragma unroll
@@ -298,6 +299,7 @@ cudaError_t launch_teacher(vsa_plan* p, const void* qp, const void* kp, const fl
   prm.n_pre = g.n_pre_tiles;
   prm.pairs_max = (g.ntv_max + 1) / 2;
   prm.scale_log2 = p->desc.softmax_scale * 1.4426950408889634f;
+  prm.wait_ns = p->wait_ns;
   for (int h = 0; h < VSA_MAX_HEADS; ++h) prm.ntv[h] = h < g.Hh ? g.ntv[h] : 0;
   const int64_t grid = int64_t(g.B) * g.Hh * prm.pairs_max;
   const int smem = teacher_smem_bytes();
@@ -314,8 +316,10 @@ cudaError_t launch_teacher(vsa_plan* p, const void* qp, const void* kp, const fl
   return cudaGetLastError();
 }
 
-cudaError_t launch_overlap(vsa_plan* p, const int32_t* a, const int32_t* b, int32_t* counts, cudaStream_t s) {
-  const Geometry& g = p->geo;
+cudaError_t launch_overlap(vsa_plan* p, const int32_t* a, const int32_t* b, int32_t* counts, cudaStream_t s,
+                           const int32_t* k) {
+  Geometry g = p->geo;   // by value: this call's k per head
+  for (int h = 0; h < g.Hh; ++h) g.k[h] = k[h];
   const int64_t rows = int64_t(g.B) * g.Hh * g.ntv_max;
   overlap_kernel<<<int((rows + 7) / 8), 256, 0, s>>>(g, a, b, counts);
   return cudaGetLastError();

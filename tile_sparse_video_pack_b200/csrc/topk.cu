@@ -126,8 +126,9 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(Geometry g, const float*
 
 }  // namespace
 
-cudaError_t launch_topk(const vsa_plan* p, const float* scores, int32_t* idx, cudaStream_t s) {
-  const Geometry& g = p->geo;
+cudaError_t launch_topk(const vsa_plan* p, const float* scores, int32_t* idx, cudaStream_t s, const int32_t* k) {
+  Geometry g = p->geo;   // by value: this call's k per head
+  for (int h = 0; h < g.Hh; ++h) g.k[h] = k[h];
   const int64_t rows = int64_t(g.B) * g.Hh * g.ntv_max;
   const size_t smem = size_t(g.ntv_max) * sizeof(uint32_t);
   if (smem > 48 * 1024) {

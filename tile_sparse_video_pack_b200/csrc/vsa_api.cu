@@ -1,6 +1,7 @@
 // C ABI of libvsa: plan construction, argument validation and the entry points.
 #include <cuda_runtime.h>
 #include <math.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -18,6 +19,24 @@ namespace {
 inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// One NVTX range per entry point (named after the call), for timeline tools.
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+};
+
+// The kept tiles per head of one call: the caller's host array (each entry
+// 1 .. min(video tiles of the head, k_max), k_max being the plan's index row
+// width) or, for NULL, the plan's own k_per_head.
+bool resolve_k(const vsa_plan* p, const int32_t* k_per_head, int32_t* out) {
+  for (int h = 0; h < p->geo.Hh; ++h) {
+    const int32_t k = k_per_head ? k_per_head[h] : p->geo.k[h];
+    if (k < 1 || k > p->geo.ntv[h] || k > p->geo.k_max) return false;
+    out[h] = k;
+  }
+  return true;
+}
 
 vsa_status fail(vsa_plan* p, vsa_status s) {
   if (p && s != VSA_OK) p->stats.errors++;
@@ -249,6 +268,8 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
     }
   p->n_items = int64_t(items.size());
   info.attn_work_items = p->n_items;
+  p->wait_ns = vsa::kDefaultWaitNs;
+  p->test_hold = 0;
 
   // dense pair count (valid rows x valid keys) for the stats
   p->stats.dense_pairs = int64_t(g.B) * g.Hh * int64_t(g.n_tokens) * g.n_tokens;
@@ -276,6 +297,9 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
       e = cudaMemcpy(p->d_ref_tiles, ref_table.data(), ref_table.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
     p->d_prefix_ref = p->d_ref_tiles ? p->d_ref_tiles + g.n_ref : nullptr;
   }
+  // (re)resolve this device's address of the fixed scratch of vsa_tile_score_static, so
+  // that a plan made after a device reset never uses the address of a discarded module
+  if (e == cudaSuccess) e = vsa::refresh_static_scratch_address(p->device);
   if (e != cudaSuccess) {
     cudaGetLastError();
     vsa_status r = (e == cudaErrorMemoryAllocation) ? VSA_ERR_NO_MEMORY : VSA_ERR_CUDA;
@@ -327,6 +351,7 @@ vsa_status vsa_plan_get_stats(const vsa_plan* p, vsa_plan_stats* out) {
 
 vsa_status vsa_tile_pack(vsa_plan* p, const void* q, const void* k, const void* v, void* qp, void* kp,
                          void* vp, void* stream) {
+  Range r("vsa_tile_pack");
   if (!p) return VSA_ERR_INVALID_ARG;
   const void* src[3] = {q, k, v};
   void* dst[3] = {qp, kp, vp};
@@ -346,6 +371,7 @@ vsa_status vsa_tile_pack(vsa_plan* p, const void* q, const void* k, const void* 
 
 vsa_status vsa_tile_pack_pool(vsa_plan* p, const void* q, const void* k, const void* v, void* qp, void* kp,
                               void* vp, void* ws, void* stream) {
+  Range r("vsa_tile_pack_pool");
   if (!p || !q || !k || !v || !qp || !kp || !vp || !ws) return fail(p, VSA_ERR_INVALID_ARG);
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qp) || !aligned16(kp) || !aligned16(vp) ||
       (reinterpret_cast<uintptr_t>(ws) & 255u))
@@ -362,6 +388,7 @@ vsa_status vsa_tile_pack_pool(vsa_plan* p, const void* q, const void* k, const v
 vsa_status vsa_tile_pack_pool_fp8(vsa_plan* p, const void* q, const void* k, const void* v, void* qp, void* kp,
                                   void* vp, void* qp8, void* kp8, float* q_scale, float* k_scale, void* ws,
                                   void* stream) {
+  Range r("vsa_tile_pack_pool_fp8");
   if (!p || !q || !k || !v || !qp || !kp || !vp || !qp8 || !kp8 || !q_scale || !k_scale || !ws)
     return fail(p, VSA_ERR_INVALID_ARG);
   if (p->geo.d != 128) return fail(p, VSA_ERR_UNSUPPORTED);
@@ -380,16 +407,19 @@ vsa_status vsa_tile_pack_pool_fp8(vsa_plan* p, const void* q, const void* k, con
 }
 
 vsa_status vsa_sparse_attn_fp8(vsa_plan* p, const void* qp8, const void* kp8, const float* q_scale,
-                               const float* k_scale, const void* vp, const int32_t* idx, void* op, float* lse,
-                               void* stream) {
+                               const float* k_scale, const void* vp, const int32_t* idx, const int32_t* k_per_head,
+                               void* op, float* lse, void* stream) {
+  Range r("vsa_sparse_attn_fp8");
   if (!p || !qp8 || !kp8 || !q_scale || !k_scale || !vp || !idx || !op) return fail(p, VSA_ERR_INVALID_ARG);
   if (p->geo.d != 128) return fail(p, VSA_ERR_UNSUPPORTED);
   if (!aligned16(qp8) || !aligned16(kp8) || !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(vp) ||
       !aligned16(idx) || !aligned16(op) || (lse && !aligned16(lse)))
     return fail(p, VSA_ERR_INVALID_ARG);
+  int32_t k[VSA_MAX_HEADS];
+  if (!resolve_k(p, k_per_head, k)) return fail(p, VSA_ERR_INVALID_ARG);
   if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_attn++;
-  if (vsa::launch_attn(p, qp8, kp8, vp, idx, nullptr, op, lse, static_cast<cudaStream_t>(stream), q_scale,
+  if (vsa::launch_attn(p, qp8, kp8, vp, idx, nullptr, k, op, lse, static_cast<cudaStream_t>(stream), q_scale,
                        k_scale) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
   return VSA_OK;
@@ -397,6 +427,7 @@ vsa_status vsa_sparse_attn_fp8(vsa_plan* p, const void* qp8, const void* kp8, co
 
 vsa_status vsa_tile_score_pooled(vsa_plan* p, const float* proj_q, const float* proj_k, float* scores, void* ws,
                                  void* stream) {
+  Range r("vsa_tile_score_pooled");
   if (!p || !proj_q || !proj_k || !scores || !ws) return fail(p, VSA_ERR_INVALID_ARG);
   if (!aligned16(proj_q) || !aligned16(proj_k) || !aligned16(scores) || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return fail(p, VSA_ERR_INVALID_ARG);
@@ -408,6 +439,7 @@ vsa_status vsa_tile_score_pooled(vsa_plan* p, const float* proj_q, const float* 
 }
 
 vsa_status vsa_tile_unpack(vsa_plan* p, const void* op, void* o, void* stream) {
+  Range r("vsa_tile_unpack");
   if (!p || !op || !o || !aligned16(op) || !aligned16(o)) return fail(p, VSA_ERR_INVALID_ARG);
   if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_unpack++;
@@ -418,6 +450,7 @@ vsa_status vsa_tile_unpack(vsa_plan* p, const void* op, void* o, void* stream) {
 
 vsa_status vsa_tile_score(vsa_plan* p, const void* qp, const void* kp, const float* proj_q,
                           const float* proj_k, float* scores, void* ws, void* stream) {
+  Range r("vsa_tile_score");
   if (!p || !qp || !kp || !proj_q || !proj_k || !scores || !ws) return fail(p, VSA_ERR_INVALID_ARG);
   if (!aligned16(qp) || !aligned16(kp) || !aligned16(proj_q) || !aligned16(proj_k) ||
       !aligned16(scores) || (reinterpret_cast<uintptr_t>(ws) & 255u))
@@ -430,30 +463,39 @@ vsa_status vsa_tile_score(vsa_plan* p, const void* qp, const void* kp, const flo
   return VSA_OK;
 }
 
-vsa_status vsa_topk_select(vsa_plan* p, const float* scores, int32_t* idx, void* stream) {
+vsa_status vsa_topk_select(vsa_plan* p, const float* scores, const int32_t* k_per_head, int32_t* idx,
+                           void* stream) {
+  Range r("vsa_topk_select");
   if (!p || !scores || !idx || !aligned16(scores) || !aligned16(idx)) return fail(p, VSA_ERR_INVALID_ARG);
+  int32_t k[VSA_MAX_HEADS];
+  if (!resolve_k(p, k_per_head, k)) return fail(p, VSA_ERR_INVALID_ARG);
   if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_select++;
-  if (vsa::launch_topk(p, scores, idx, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (vsa::launch_topk(p, scores, idx, static_cast<cudaStream_t>(stream), k) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
   return VSA_OK;
 }
 
 vsa_status vsa_sparse_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp,
-                           const int32_t* idx, void* op, float* lse, void* stream) {
+                           const int32_t* idx, const int32_t* k_per_head, void* op, float* lse, void* stream) {
+  Range r("vsa_sparse_attn");
   if (!p || !qp || !kp || !vp || !idx || !op) return fail(p, VSA_ERR_INVALID_ARG);
   if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(idx) || !aligned16(op) ||
       (lse && !aligned16(lse)))
     return fail(p, VSA_ERR_INVALID_ARG);
+  int32_t k[VSA_MAX_HEADS];
+  if (!resolve_k(p, k_per_head, k)) return fail(p, VSA_ERR_INVALID_ARG);
   if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_attn++;
-  if (vsa::launch_attn(p, qp, kp, vp, idx, nullptr, op, lse, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (vsa::launch_attn(p, qp, kp, vp, idx, nullptr, k, op, lse, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
   return VSA_OK;
 }
 
 vsa_status vsa_ref_score(vsa_plan* p, const void* kp, const float* proj_k, float* scores_ref, void* ws,
                          void* stream) {
+  Range r("vsa_ref_score");
   if (!p || !kp || !proj_k || !scores_ref || !ws) return fail(p, VSA_ERR_INVALID_ARG);
   if (p->geo.n_ref == 0) return fail(p, VSA_ERR_INVALID_ARG);
   if (!aligned16(kp) || !aligned16(proj_k) || !aligned16(scores_ref) || (reinterpret_cast<uintptr_t>(ws) & 255u))
@@ -466,6 +508,7 @@ vsa_status vsa_ref_score(vsa_plan* p, const void* kp, const float* proj_k, float
 }
 
 vsa_status vsa_topk_select_ref(vsa_plan* p, const float* scores_ref, int32_t* idx_ref, void* stream) {
+  Range r("vsa_topk_select_ref");
   if (!p || !scores_ref || !idx_ref || p->geo.n_ref == 0 || !aligned16(scores_ref) || !aligned16(idx_ref))
     return fail(p, VSA_ERR_INVALID_ARG);
   if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
@@ -476,14 +519,19 @@ vsa_status vsa_topk_select_ref(vsa_plan* p, const float* scores_ref, int32_t* id
 }
 
 vsa_status vsa_sparse_attn_ref(vsa_plan* p, const void* qp, const void* kp, const void* vp, const int32_t* idx,
-                               const int32_t* idx_ref, void* op, float* lse, void* stream) {
+                               const int32_t* idx_ref, const int32_t* k_per_head, void* op, float* lse,
+                               void* stream) {
+  Range r("vsa_sparse_attn_ref");
   if (!p || !qp || !kp || !vp || !idx || !idx_ref || !op || p->geo.n_ref == 0) return fail(p, VSA_ERR_INVALID_ARG);
   if (!aligned16(qp) || !aligned16(kp) || !aligned16(vp) || !aligned16(idx) || !aligned16(idx_ref) ||
       !aligned16(op) || (lse && !aligned16(lse)))
     return fail(p, VSA_ERR_INVALID_ARG);
+  int32_t k[VSA_MAX_HEADS];
+  if (!resolve_k(p, k_per_head, k)) return fail(p, VSA_ERR_INVALID_ARG);
   if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
   p->stats.calls_attn++;
-  if (vsa::launch_attn(p, qp, kp, vp, idx, idx_ref, op, lse, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (vsa::launch_attn(p, qp, kp, vp, idx, idx_ref, k, op, lse, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
   return VSA_OK;
 }
@@ -492,17 +540,19 @@ vsa_status vsa_layer_forward(vsa_plan* p, const void* q, const void* k, const vo
                              const float* proj_q, const float* proj_k, void* qp, void* kp, void* vp,
                              float* scores, int32_t* idx, void* op, float* lse, void* ws, void* o,
                              void* stream) {
+  Range r("vsa_layer_forward");
   if (p && p->geo.n_ref) return fail(p, VSA_ERR_UNSUPPORTED);
   vsa_status s = vsa_tile_pack_pool(p, q, k, v, qp, kp, vp, ws, stream);
   if (s == VSA_OK) s = vsa_tile_score_pooled(p, proj_q, proj_k, scores, ws, stream);
-  if (s == VSA_OK) s = vsa_topk_select(p, scores, idx, stream);
-  if (s == VSA_OK) s = vsa_sparse_attn(p, qp, kp, vp, idx, op, lse, stream);
+  if (s == VSA_OK) s = vsa_topk_select(p, scores, nullptr, idx, stream);
+  if (s == VSA_OK) s = vsa_sparse_attn(p, qp, kp, vp, idx, nullptr, op, lse, stream);
   if (s == VSA_OK) s = vsa_tile_unpack(p, op, o, stream);
   return s;
 }
 
 vsa_status vsa_teacher_tiles(vsa_plan* p, const void* qp, const void* kp, const float* lse, float* teacher,
                              void* stream) {
+  Range r("vsa_teacher_tiles");
   if (!p || !qp || !kp || !lse || !teacher || !aligned16(qp) || !aligned16(kp) || !aligned16(lse) ||
       !aligned16(teacher))
     return fail(p, VSA_ERR_INVALID_ARG);
@@ -512,13 +562,30 @@ vsa_status vsa_teacher_tiles(vsa_plan* p, const void* qp, const void* kp, const 
   return VSA_OK;
 }
 
-vsa_status vsa_index_overlap(vsa_plan* p, const int32_t* idx_a, const int32_t* idx_b, int32_t* counts,
-                             void* stream) {
+vsa_status vsa_index_overlap(vsa_plan* p, const int32_t* idx_a, const int32_t* idx_b,
+                             const int32_t* k_per_head, int32_t* counts, void* stream) {
+  Range r("vsa_index_overlap");
   if (!p || !idx_a || !idx_b || !counts || !aligned16(idx_a) || !aligned16(idx_b) || !aligned16(counts))
     return fail(p, VSA_ERR_INVALID_ARG);
+  int32_t k[VSA_MAX_HEADS];
+  if (!resolve_k(p, k_per_head, k)) return fail(p, VSA_ERR_INVALID_ARG);
   if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
-  if (vsa::launch_overlap(p, idx_a, idx_b, counts, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (vsa::launch_overlap(p, idx_a, idx_b, counts, static_cast<cudaStream_t>(stream), k) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_plan_set_wait_limit(vsa_plan* p, uint64_t limit_ns) {
+  if (!p) return VSA_ERR_INVALID_ARG;
+  if (limit_ns == 0) limit_ns = vsa::kDefaultWaitNs;
+  if (limit_ns < 1000ull || limit_ns > 60000000000ull) return fail(p, VSA_ERR_INVALID_ARG);
+  p->wait_ns = limit_ns;
+  return VSA_OK;
+}
+
+vsa_status vsa_plan_set_test_hold(vsa_plan* p, int32_t on) {
+  if (!p || (on != 0 && on != 1)) return fail(p, VSA_ERR_INVALID_ARG);
+  p->test_hold = on;
   return VSA_OK;
 }
 

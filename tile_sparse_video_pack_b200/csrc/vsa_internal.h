@@ -10,6 +10,9 @@
 
 namespace vsa {
 
+// Default bound of every device-side wait of the tcgen05 kernels (two seconds).
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+
 // Bits of the device error word.
 enum : uint32_t {
   kErrTimeout = 1u << 0,
@@ -60,6 +63,8 @@ struct vsa_plan {
   int32_t* d_prefix_ref;   // [n_pre_tiles] each prefix tile's position among them, or -1
   int attn_smem_bytes;
   int list_cap;            // entries of one key-list buffer in the attention kernel
+  uint64_t wait_ns;        // bound of every device-side wait of the tcgen05 kernels
+  int32_t test_hold;       // test hook: the attention softmax waits for a release nothing gives
 };
 
 namespace vsa {
@@ -78,19 +83,25 @@ cudaError_t launch_score(const vsa_plan* p, const void* qp, const void* kp, cons
 int64_t score_workspace_bytes(const Geometry& g, int score_mode, int proj_dim);
 // Where the score stage keeps the pooled Q and K descriptors in a workspace.
 void score_pooled_ptrs(const vsa_plan* p, void* workspace, float** pooled_q, float** pooled_k);
+// Looks up (with `dev` current) and caches the device address of the fixed scratch
+// array of vsa_tile_score_static.
+cudaError_t refresh_static_scratch_address(int dev);
 cudaError_t launch_project_score(const vsa_plan* p, const float* proj_q, const float* proj_k, float* scores,
                                  void* workspace, cudaStream_t s);
-cudaError_t launch_topk(const vsa_plan* p, const float* scores, int32_t* idx, cudaStream_t s);
+// k: kept tiles per head for this call (host array of `heads` entries, validated)
+cudaError_t launch_topk(const vsa_plan* p, const float* scores, int32_t* idx, cudaStream_t s, const int32_t* k);
 cudaError_t launch_topk_ref(const vsa_plan* p, const float* scores_ref, int32_t* idx_ref, cudaStream_t s);
 cudaError_t launch_ref_score(const vsa_plan* p, const void* kp, const float* proj_k, float* scores_ref,
                              void* workspace, cudaStream_t s);
 // q_scale != null: qp, kp are e4m3 tiles (head_dim 128) with per-tile scales q_scale, k_scale
+// k: kept video tiles per head for this call (host array of `heads` entries, validated)
 cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp,
-                        const int32_t* idx, const int32_t* idx_ref, void* op, float* lse, cudaStream_t s,
-                        const float* q_scale = nullptr, const float* k_scale = nullptr);
+                        const int32_t* idx, const int32_t* idx_ref, const int32_t* k, void* op, float* lse,
+                        cudaStream_t s, const float* q_scale = nullptr, const float* k_scale = nullptr);
 int attn_smem_bytes(int list_cap);
 cudaError_t launch_teacher(vsa_plan* p, const void* qp, const void* kp, const float* lse, float* teacher,
                            cudaStream_t s);
-cudaError_t launch_overlap(vsa_plan* p, const int32_t* a, const int32_t* b, int32_t* counts, cudaStream_t s);
+cudaError_t launch_overlap(vsa_plan* p, const int32_t* a, const int32_t* b, int32_t* counts, cudaStream_t s,
+                           const int32_t* k);
 
 }  // namespace vsa

@@ -28,7 +28,7 @@ EXPORTS = ("vsa_plan_create", "vsa_plan_destroy", "vsa_plan_query", "vsa_plan_ge
            "vsa_layer_forward", "vsa_plan_check", "vsa_status_string", "vsa_tile_score_static",
            "vsa_tile_pack_pool", "vsa_tile_score_pooled", "vsa_teacher_tiles", "vsa_index_overlap",
            "vsa_ref_score", "vsa_topk_select_ref", "vsa_sparse_attn_ref", "vsa_tile_pack_pool_fp8",
-           "vsa_sparse_attn_fp8")
+           "vsa_sparse_attn_fp8", "vsa_plan_set_wait_limit", "vsa_plan_set_test_hold")
 
 
 class VsaDesc(ctypes.Structure):
@@ -89,8 +89,8 @@ def library() -> ctypes.CDLL:
         "vsa_k_from_sparsity": (I32, [D, I32]),
         "vsa_tile_pack": (I32, [P, P, P, P, P, P, P, P]),
         "vsa_tile_score": (I32, [P, P, P, P, P, P, P, P]),
-        "vsa_topk_select": (I32, [P, P, P, P]),
-        "vsa_sparse_attn": (I32, [P, P, P, P, P, P, P, P]),
+        "vsa_topk_select": (I32, [P, P, P, P, P]),
+        "vsa_sparse_attn": (I32, [P, P, P, P, P, P, P, P, P]),
         "vsa_tile_unpack": (I32, [P, P, P, P]),
         "vsa_layer_forward": (I32, [P] + [P] * 15),
         "vsa_plan_check": (I32, [P]),
@@ -99,12 +99,14 @@ def library() -> ctypes.CDLL:
         "vsa_tile_pack_pool": (I32, [P] * 9),
         "vsa_tile_score_pooled": (I32, [P] * 6),
         "vsa_teacher_tiles": (I32, [P] * 6),
-        "vsa_index_overlap": (I32, [P] * 5),
+        "vsa_index_overlap": (I32, [P] * 6),
         "vsa_ref_score": (I32, [P] * 6),
         "vsa_topk_select_ref": (I32, [P] * 4),
-        "vsa_sparse_attn_ref": (I32, [P] * 9),
+        "vsa_sparse_attn_ref": (I32, [P] * 10),
         "vsa_tile_pack_pool_fp8": (I32, [P] * 13),
-        "vsa_sparse_attn_fp8": (I32, [P] * 10),
+        "vsa_sparse_attn_fp8": (I32, [P] * 11),
+        "vsa_plan_set_wait_limit": (I32, [P, ctypes.c_uint64]),
+        "vsa_plan_set_test_hold": (I32, [P, I32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -164,6 +166,16 @@ def _ptr(t, dtype, name, min_numel=0):
     if t.numel() < min_numel:
         raise ValueError(f"{name} holds {t.numel()} elements, needs {min_numel}")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _karray(k_per_head, heads):
+    """A host int32 array of the per-call k of each head (None -> NULL: the plan's own k)."""
+    if k_per_head is None:
+        return None
+    ks = [int(x) for x in k_per_head]
+    if len(ks) != heads:
+        raise ValueError(f"k_per_head has {len(ks)} entries, the plan {heads} heads")
+    return (ctypes.c_int32 * heads)(*ks)
 
 
 def _stream(stream):
@@ -293,7 +305,7 @@ class Plan:
             _ptr(k_scale, f32, "k_scale", ns),
             _ptr(workspace, u8, "workspace", self.info.workspace_bytes), _stream(stream)), "vsa_tile_pack_pool_fp8")
 
-    def sparse_attn_fp8(self, qp8, kp8, q_scale, k_scale, vp, idx, op, lse=None, stream=None):
+    def sparse_attn_fp8(self, qp8, kp8, q_scale, k_scale, vp, idx, op, lse=None, stream=None, k_per_head=None):
         """sparse_attn with Q K^T from the e4m3 tiles and their per-tile scales."""
         import torch
         pe, u8, f32, bf = self.info.packed_elems, torch.uint8, torch.float32, torch.bfloat16
@@ -301,7 +313,8 @@ class Plan:
         _check(library().vsa_sparse_attn_fp8(
             self._h, _ptr(qp8, u8, "qp8", pe), _ptr(kp8, u8, "kp8", pe), _ptr(q_scale, f32, "q_scale", ns),
             _ptr(k_scale, f32, "k_scale", ns), _ptr(vp, bf, "vp", pe),
-            _ptr(idx, torch.int32, "idx", self.info.index_elems), _ptr(op, bf, "op", pe),
+            _ptr(idx, torch.int32, "idx", self.info.index_elems), _karray(k_per_head, self.desc.heads),
+            _ptr(op, bf, "op", pe),
             _ptr(lse, f32, "lse", self.info.lse_elems), _stream(stream)), "vsa_sparse_attn_fp8")
 
     def allocate_fp8(self, device=None):
@@ -332,13 +345,13 @@ class Plan:
             _ptr(lse, torch.float32, "lse", self.info.lse_elems),
             _ptr(teacher, torch.float32, "teacher", self.info.score_elems), _stream(stream)), "vsa_teacher_tiles")
 
-    def index_overlap(self, idx_a, idx_b, counts, stream=None):
+    def index_overlap(self, idx_a, idx_b, counts, stream=None, k_per_head=None):
         """Shared indices per row of two ascending top-k tables."""
         import torch
         n = self.desc.batch * self.desc.heads * self.info.ntv_max
         _check(library().vsa_index_overlap(
             self._h, _ptr(idx_a, torch.int32, "idx_a", self.info.index_elems),
-            _ptr(idx_b, torch.int32, "idx_b", self.info.index_elems),
+            _ptr(idx_b, torch.int32, "idx_b", self.info.index_elems), _karray(k_per_head, self.desc.heads),
             _ptr(counts, torch.int32, "counts", n), _stream(stream)), "vsa_index_overlap")
 
     def tile_score_static(self, qp, kp, proj_q, proj_k, scores, stream=None):
@@ -356,18 +369,22 @@ class Plan:
             _ptr(scores, torch.float32, "scores", self.info.score_elems), _stream(stream)),
             "vsa_tile_score_static")
 
-    def topk_select(self, scores, idx, stream=None):
+    def topk_select(self, scores, idx, stream=None, k_per_head=None):
+        """k_per_head: this call's kept tiles per head (None: the plan's)."""
         import torch
         _check(library().vsa_topk_select(
             self._h, _ptr(scores, torch.float32, "scores", self.info.score_elems),
+            _karray(k_per_head, self.desc.heads),
             _ptr(idx, torch.int32, "idx", self.info.index_elems), _stream(stream)), "vsa_topk_select")
 
-    def sparse_attn(self, qp, kp, vp, idx, op, lse=None, stream=None):
+    def sparse_attn(self, qp, kp, vp, idx, op, lse=None, stream=None, k_per_head=None):
+        """k_per_head: this call's kept tiles per head (None: the plan's); as given to topk_select."""
         import torch
         pe, bf = self.info.packed_elems, torch.bfloat16
         _check(library().vsa_sparse_attn(
             self._h, _ptr(qp, bf, "qp", pe), _ptr(kp, bf, "kp", pe), _ptr(vp, bf, "vp", pe),
-            _ptr(idx, torch.int32, "idx", self.info.index_elems), _ptr(op, bf, "op", pe),
+            _ptr(idx, torch.int32, "idx", self.info.index_elems), _karray(k_per_head, self.desc.heads),
+            _ptr(op, bf, "op", pe),
             _ptr(lse, torch.float32, "lse", self.info.lse_elems), _stream(stream)), "vsa_sparse_attn")
 
     def ref_score(self, kp, proj_k, scores_ref, workspace, stream=None):
@@ -385,13 +402,14 @@ class Plan:
             _ptr(idx_ref, torch.int32, "idx_ref", self.info.ref_index_elems), _stream(stream)),
             "vsa_topk_select_ref")
 
-    def sparse_attn_ref(self, qp, kp, vp, idx, idx_ref, op, lse=None, stream=None):
+    def sparse_attn_ref(self, qp, kp, vp, idx, idx_ref, op, lse=None, stream=None, k_per_head=None):
         import torch
         pe, bf = self.info.packed_elems, torch.bfloat16
         _check(library().vsa_sparse_attn_ref(
             self._h, _ptr(qp, bf, "qp", pe), _ptr(kp, bf, "kp", pe), _ptr(vp, bf, "vp", pe),
             _ptr(idx, torch.int32, "idx", self.info.index_elems),
-            _ptr(idx_ref, torch.int32, "idx_ref", self.info.ref_index_elems), _ptr(op, bf, "op", pe),
+            _ptr(idx_ref, torch.int32, "idx_ref", self.info.ref_index_elems), _karray(k_per_head, self.desc.heads),
+            _ptr(op, bf, "op", pe),
             _ptr(lse, torch.float32, "lse", self.info.lse_elems), _stream(stream)), "vsa_sparse_attn_ref")
 
     def tile_unpack(self, op, o, stream=None):
@@ -415,6 +433,14 @@ class Plan:
             _ptr(bufs.get("lse"), torch.float32, "lse", self.info.lse_elems),
             _ptr(bufs["workspace"], torch.uint8, "workspace", self.info.workspace_bytes),
             _ptr(o, bf, "o", n_tok), _stream(stream)), "vsa_layer_forward")
+
+    def set_wait_limit(self, limit_ns: int = 0):
+        """Bound of every device-side wait of the plan's tcgen05 kernels (0: the two-second default)."""
+        _check(library().vsa_plan_set_wait_limit(self._h, int(limit_ns)), "vsa_plan_set_wait_limit")
+
+    def set_test_hold(self, on: bool):
+        """Test hook: attention's softmax waits for a release nothing gives, until the wait limit."""
+        _check(library().vsa_plan_set_test_hold(self._h, 1 if on else 0), "vsa_plan_set_test_hold")
 
     def check(self):
         """Synchronise and raise if a kernel latched a device-side error."""

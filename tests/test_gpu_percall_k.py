@@ -74,7 +74,9 @@ def test_bad_k_is_rejected_before_launch():
     cfg = ragged_gpu_config(128)
     r = LayerRun(cfg, 0.5)
     b, p = r.bufs, r.plan
-    for bad in ([0] + r.k[1:], [r.k[0] + 1] + r.k[1:], [-3] * cfg.heads):
+    kmax = r.plan.info.k_max      # the index tables' row width: no call may keep more
+    for bad in ([0] + r.k[1:], [kmax + 1] + r.k[1:], r.k[:-1] + [r.plan.info.ntv[cfg.heads - 1] + 1],
+                [-3] * cfg.heads):
         for call in (lambda: p.topk_select(b["scores"], b["idx"], k_per_head=bad),
                      lambda: p.sparse_attn(b["qp"], b["kp"], b["vp"], b["idx"], b["op"], k_per_head=bad)):
             with pytest.raises(T.VsaError) as e:

@@ -83,23 +83,32 @@ __global__ void __launch_bounds__(256) pack_kernel(Geometry g, const uint4* __re
   }
 }
 
+// Unpack of one packed tile per CTA (the shape of the fused pack-and-pool pass):
+// thread t moves chunk t mod CPR of rows t / CPR + RG*i; each thread resolves
+// its rows' tokens once, issues all its loads, then its stores. Unused slots
+// are neither read nor written.
 template <int CPR>
-__global__ void __launch_bounds__(256) unpack_kernel(Geometry g, const uint4* __restrict__ op,
-                                                     uint4* __restrict__ o) {
-  const int64_t total = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE * CPR;
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t row = i / CPR;
-    const int c = int(i - row * CPR);
-    const int s = int(row % VSA_TILE);
-    const int64_t tile = row / VSA_TILE;
-    const int n = int(tile % g.nt_max);
-    const int bh = int(tile / g.nt_max);
-    const int h = bh % g.Hh, b = bh / g.Hh;
-    const int tok = src_token(g, h, n, s);
-    if (tok < 0) continue;
-    o[((int64_t(b) * g.n_tokens + tok) * g.Hh + h) * CPR + c] = ld_stream(op + i);
+__global__ void __launch_bounds__(256) unpack_tile_kernel(Geometry g, const uint4* __restrict__ op,
+                                                          uint4* __restrict__ o) {
+  constexpr int RG = 256 / CPR;
+  constexpr int RPT = 64 / RG;
+  const int64_t tile = blockIdx.x;    // bh * nt_max + n
+  const int n = int(tile % g.nt_max);
+  const int bh = int(tile / g.nt_max);
+  const int h = bh % g.Hh, b = bh / g.Hh;
+  const int c = threadIdx.x % CPR;
+  const int rg = threadIdx.x / CPR;
+  int tok[RPT];
+  uint4 val[RPT];
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const int s = rg + RG * i;
+    tok[i] = src_token(g, h, n, s);
+    val[i] = tok[i] >= 0 ? ld_stream(op + (tile * VSA_TILE + s) * CPR + c) : make_uint4(0, 0, 0, 0);
   }
+#pragma unroll
+  for (int i = 0; i < RPT; ++i)
+    if (tok[i] >= 0) o[((int64_t(b) * g.n_tokens + tok[i]) * g.Hh + h) * CPR + c] = val[i];
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float (&x)[8]) {
@@ -378,13 +387,12 @@ cudaError_t launch_pack_pool(const vsa_plan* p, const void* q, const void* k, co
 
 cudaError_t launch_unpack(const vsa_plan* p, const void* op, void* o, cudaStream_t s) {
   const Geometry& g = p->geo;
-  const int cpr = g.d / 8;
-  const int64_t total = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE * cpr;
-  const int grid = grid_for(p, total);
-  if (cpr == 16)
-    unpack_kernel<16><<<grid, 256, 0, s>>>(g, static_cast<const uint4*>(op), static_cast<uint4*>(o));
+  const int64_t tiles = int64_t(g.B) * g.Hh * g.nt_max;
+  if (tiles == 0) return cudaSuccess;
+  if (g.d == 128)
+    unpack_tile_kernel<16><<<unsigned(tiles), 256, 0, s>>>(g, static_cast<const uint4*>(op), static_cast<uint4*>(o));
   else
-    unpack_kernel<8><<<grid, 256, 0, s>>>(g, static_cast<const uint4*>(op), static_cast<uint4*>(o));
+    unpack_tile_kernel<8><<<unsigned(tiles), 256, 0, s>>>(g, static_cast<const uint4*>(op), static_cast<uint4*>(o));
   return cudaGetLastError();
 }
 

@@ -4,14 +4,17 @@
 // tokens): the mean for the VSA gate score (Ref2VA VSA README: the gating
 // projection to_gate_compress picks the tiles), or the TripPool descriptor
 // avg, max, min (BSAI VedaSparse README, "Core Technology: TripPool";
-// "Implementation": _tripool, eq. 5). Projection and scores are fp32 batched
-// GEMMs: q_hat = pooled(Q) W, k_hat = pooled(K) W, S = q_hat k_hat^T / sqrt(p)
+// "Implementation": _tripool, eq. 5). Projections are fp32 batched GEMMs
+// (q_hat = pooled(Q) W, k_hat = pooled(K) W); the tile-score GEMM
+// S = q_hat k_hat^T / sqrt(p) runs on the tensor cores as three-pass TF32
 // ("Scorer Modes": per-head projections, eq. 6).
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
 
 #include <mutex>
 
+#include "tc_sm100.h"
 #include "vsa_internal.h"
 
 namespace vsa {
@@ -169,10 +172,9 @@ __global__ void __launch_bounds__(256) pool_ref_kernel(Geometry g, const uint16_
   }
 }
 
-// C[z] (+)= alpha * A[z] * op(B[z]); z = b * heads + h; 128 x 128 tiles, 8 x 8 per thread.
-// A: [M][K] row-major (lda). B: [K][N] (ldb) or, with BT, [N][K] (ldb).
+// The projections: C[z] = alpha * A[z] * B[z] (fp32 SIMT); z = b * heads + h; 128 x 128 tiles, 8 x 8
+// per thread. A: [M][K] row-major (lda). B: [K][N] row-major (ldb).
 // M = m_fixed if > 0 else ntv[h]; N = n_fixed if > 0 else ntv[h]. K % 8 == 0, rows 16-byte aligned.
-template <bool BT>
 __global__ void __launch_bounds__(256) sgemm_kernel(Geometry g, const float* __restrict__ A, int64_t sA, int lda,
                                                     const float* __restrict__ Bm, int64_t sBz, int64_t sBh,
                                                     int ldb, float* __restrict__ C, int64_t sC, int ldc, int K,
@@ -206,15 +208,7 @@ __global__ void __launch_bounds__(256) sgemm_kernel(Geometry g, const float* __r
       As[kq + 2][r] = a.z;
       As[kq + 3][r] = a.w;
     }
-    if (BT) {  // B rows are n: 128 n x 8 k
-      const int r = tid >> 1, kq = (tid & 1) * 4;
-      float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (n0 + r < N) b = *reinterpret_cast<const float4*>(Bm + int64_t(n0 + r) * ldb + k0 + kq);
-      Bs[kq + 0][r] = b.x;
-      Bs[kq + 1][r] = b.y;
-      Bs[kq + 2][r] = b.z;
-      Bs[kq + 3][r] = b.w;
-    } else {  // B rows are k: 8 k x 128 n
+    {  // B rows are k: 8 k x 128 n
       const int kr = tid >> 5, c = (tid & 31) * 4;
       float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
       if (n0 + c < N) b = *reinterpret_cast<const float4*>(Bm + int64_t(k0 + kr) * ldb + n0 + c);
@@ -247,6 +241,208 @@ __global__ void __launch_bounds__(256) sgemm_kernel(Geometry g, const float* __r
   }
 }
 
+// C[z][m][n] = alpha * sum_k A[z][m][k] B[z][n][k] for m < M, n < N (rows and
+// columns past them untouched). A, B fp32, K-major rows of K = kdim values.
+// Each operand is split in shared memory into hi = tf32(x) (round to nearest)
+// and lo = x - hi (exact in fp32), and the tensor core accumulates
+// hi*hi + hi*lo + lo*hi in fp32 (the lo*lo term, ~2^-22 relative, is dropped),
+// which keeps the scores near fp32 accuracy: the selection is checked against
+// an fp64 oracle to 1e-5 of the row's score scale.
+struct ScoreTcParams {
+  float* C;
+  int64_t a_rows_per_z, b_rows_per_z;   // row offsets of batch-head z in the A and B maps
+  int64_t c_stride_z;                   // elements between the C matrices of consecutive z
+  int32_t ldc;                          // row stride of C (elements)
+  int32_t m_fixed, n_fixed;             // > 0: M / N; else the head's video tile count
+  int32_t kdim;                         // K, a multiple of 4 (rows 16-byte aligned)
+  float alpha;
+  uint64_t wait_ns;
+  uint32_t* err;
+  int32_t heads;
+  int32_t ntv[VSA_MAX_HEADS];
+};
+
+constexpr int kTcThreads = 128;
+constexpr uint32_t kTcTileBytes = 128 * 128;   // 128 rows x 32 fp32 (one 128-byte swizzle row each)
+
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// Bounded wait of every thread of the CTA on one phase of an mbarrier.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  if (tc::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = tc::globaltimer();
+  while (!tc::mbar_try_wait(bar, parity))
+    if (tc::globaltimer() - t0 > limit_ns) return false;
+  return true;
+}
+
+__global__ void __launch_bounds__(kTcThreads) score_tc_kernel(const __grid_constant__ CUtensorMap ta,
+                                                              const __grid_constant__ CUtensorMap tb,
+                                                              const __grid_constant__ ScoreTcParams prm) {
+  const int z = blockIdx.z;
+  const int h = z % prm.heads;
+  const int M = prm.m_fixed > 0 ? prm.m_fixed : prm.ntv[h];
+  const int N = prm.n_fixed > 0 ? prm.n_fixed : prm.ntv[h];
+  const int m0 = blockIdx.y * 128, n0 = blockIdx.x * 128;
+  if (m0 >= M || n0 >= N) return;   // uniform over the CTA, before any barrier or TMEM use
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // [A hi | A lo | B hi | B lo], each 128 rows x 128 bytes in the 128-byte-swizzled K-major layout
+  float* a_hi = reinterpret_cast<float*>(smem);
+  float* a_lo = reinterpret_cast<float*>(smem + kTcTileBytes);
+  float* b_hi = reinterpret_cast<float*>(smem + 2 * kTcTileBytes);
+  float* b_lo = reinterpret_cast<float*>(smem + 3 * kTcTileBytes);
+  __shared__ __align__(8) uint64_t bars[3];   // [0] chunk landed, [1] chunk's MMAs done, [2] drain
+  __shared__ uint32_t tmem_base;
+  const uint32_t sbase = tc::smem_u32(smem);
+  const uint32_t bar_full = tc::smem_u32(&bars[0]), bar_mma = tc::smem_u32(&bars[1]);
+  const uint32_t bar_drain = tc::smem_u32(&bars[2]);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(bar_full, 1);
+    tc::mbar_init(bar_mma, 1);
+    tc::mbar_init(bar_drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 128;" ::"r"(tc::smem_u32(&tmem_base)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  // instruction descriptor: kind::tf32 (A, B format 2), fp32 accumulator, both K-major, M = N = 128
+  constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(128 >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  const int chunks = (prm.kdim + 31) / 32;   // columns past kdim are read as zeros (outside the map)
+  const int64_t arow = int64_t(z) * prm.a_rows_per_z + m0;
+  const int64_t brow = int64_t(z) * prm.b_rows_per_z + n0;
+  bool ok = true;
+  int c = 0;
+  for (; c < chunks && ok; ++c) {
+    if (threadIdx.x == 0) {
+      tc::mbar_expect_tx(bar_full, 2 * kTcTileBytes);
+      tc::tma_load_2d(sbase, &ta, 32 * c, int(arow), bar_full);
+      tc::tma_load_2d(sbase + 2 * kTcTileBytes, &tb, 32 * c, int(brow), bar_full);
+    }
+    ok = tc_wait(bar_full, c & 1, prm.wait_ns);
+    if (__syncthreads_or(!ok)) {
+      ok = false;
+      tc_wait(bar_full, c & 1, tc::kTimeoutNs);   // let the copy land before shared memory is released
+      break;
+    }
+    // split in place: hi = tf32(x), lo = x - hi; elementwise, so the swizzled layout is kept
+    for (int i = threadIdx.x; i < 128 * 32; i += kTcThreads) {
+      const float xa = a_hi[i], xb = b_hi[i];
+      const float ha = __uint_as_float(tf32_rna(xa)), hb = __uint_as_float(tf32_rna(xb));
+      a_hi[i] = ha;
+      a_lo[i] = xa - ha;
+      b_hi[i] = hb;
+      b_lo[i] = xb - hb;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // generic writes -> tensor core
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc::tc_fence_after();
+      const uint64_t dah = tc::sw128_desc(sbase, 16, 1024), dal = tc::sw128_desc(sbase + kTcTileBytes, 16, 1024);
+      const uint64_t dbh = tc::sw128_desc(sbase + 2 * kTcTileBytes, 16, 1024);
+      const uint64_t dbl = tc::sw128_desc(sbase + 3 * kTcTileBytes, 16, 1024);
+#pragma unroll
+      for (int pass = 0; pass < 3; ++pass) {
+        const uint64_t da = pass == 2 ? dal : dah;
+        const uint64_t db = pass == 1 ? dbl : dbh;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {   // 8 tf32 (32 bytes) of K per instruction
+          const uint32_t off = (ks * 32) >> 4;
+          asm volatile(
+              "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+              "l"(da + off), "l"(db + off), "r"(kIdesc), "r"((c | pass | ks) ? 1u : 0u)
+              : "memory");
+        }
+      }
+      tc::tc_commit(bar_mma);
+    }
+    // the chunk's MMAs must finish reading shared memory before the next chunk lands there
+    ok = tc_wait(bar_mma, c & 1, prm.wait_ns);
+    if (__syncthreads_or(!ok)) ok = false;
+  }
+  if (!ok) {
+    // a wait ran past the limit: latch it, and let every MMA issued here finish before TMEM is freed
+    if (threadIdx.x == 0) {
+      atomicOr(prm.err, kErrTimeout);
+      tc::tc_commit(bar_drain);
+    }
+    tc_wait(bar_drain, 0, tc::kTimeoutNs);
+  } else {
+    tc::tc_fence_after();
+    // epilogue: warp w owns TMEM lanes (rows) 32w .. 32w+31; 32 columns at a time through a
+    // padded shared-memory slab per warp (row stride 144 bytes), then row-contiguous stores
+    float* slab = reinterpret_cast<float*>(smem) + warp * (32 * 36);
+    const int row0 = m0 + 32 * warp;
+    float* Cz = prm.C + int64_t(z) * prm.c_stride_z;
+    const bool vec = (prm.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(prm.C) & 15) == 0 &&
+                     (prm.c_stride_z & 3) == 0;
+#pragma unroll 1
+    for (int s = 0; s < 4; ++s) {
+      uint32_t r[32];
+      tc::tmem_ld32(tmem + (uint32_t(32 * warp) << 16) + 32 * s, r);
+      tc::tmem_wait_ld(r);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float4 v = make_float4(__uint_as_float(r[4 * q]) * prm.alpha, __uint_as_float(r[4 * q + 1]) * prm.alpha,
+                               __uint_as_float(r[4 * q + 2]) * prm.alpha, __uint_as_float(r[4 * q + 3]) * prm.alpha);
+        *reinterpret_cast<float4*>(slab + lane * 36 + 4 * q) = v;
+      }
+      __syncwarp();
+      // lanes 8j .. 8j+7 write row (4i + j) of the slab: 8 x 16 bytes = the slab's 32 columns
+      const int col = n0 + 32 * s + 4 * (lane & 7);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = 4 * i + (lane >> 3);
+        const int m = row0 + rr;
+        if (m < M) {
+          const float4 v = *reinterpret_cast<const float4*>(slab + rr * 36 + 4 * (lane & 7));
+          float* dst = Cz + int64_t(m) * prm.ldc + col;
+          if (vec && col + 3 < N) {
+            *reinterpret_cast<float4*>(dst) = v;
+          } else {
+            if (col < N) dst[0] = v.x;
+            if (col + 1 < N) dst[1] = v.y;
+            if (col + 2 < N) dst[2] = v.z;
+            if (col + 3 < N) dst[3] = v.w;
+          }
+        }
+      }
+      __syncwarp();
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 128;" ::"r"(tmem));
+}
+
+// fp32 [rows, kdim] viewed as a 2D tensor; boxes of 32 columns (128 bytes) x 128 rows, 128-byte swizzle.
+bool make_map_f32(CUtensorMap* m, const void* base, int64_t rows, int kdim) {
+  tc::EncodeTiledFn enc = tc::get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cuuint64_t(kdim), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(kdim) * 4};
+  cuuint32_t box[2] = {32, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int score_tc_smem_bytes() { return 1024 + 4 * int(kTcTileBytes); }
+
 }  // namespace
 
 int64_t score_workspace_bytes(const Geometry& g, int mode, int p) { return score_layout(g, mode, p).total; }
@@ -256,6 +452,38 @@ void score_pooled_ptrs(const vsa_plan* pl, void* workspace, float** pooled_q, fl
   char* ws = static_cast<char*>(workspace);
   *pooled_q = reinterpret_cast<float*>(ws + L.off_pq);
   *pooled_k = reinterpret_cast<float*>(ws + L.off_pk);
+}
+
+// C[z] = alpha * A[z] B[z]^T on the tensor cores (score_tc_kernel): A rows a_rows_per_z per z,
+// B rows b_rows_per_z per z, both [.., kdim] fp32; M, N as in ScoreTcParams.
+cudaError_t launch_score_tc(const vsa_plan* pl, const float* A, int64_t a_rows_per_z, const float* B,
+                            int64_t b_rows_per_z, int kdim, float* C, int64_t c_stride_z, int ldc, int m_fixed,
+                            int n_fixed, int m_max, int n_max, float alpha, cudaStream_t s) {
+  const Geometry& g = pl->geo;
+  const int Z = g.B * g.Hh;
+  CUtensorMap ta, tb;
+  if (!make_map_f32(&ta, A, int64_t(Z) * a_rows_per_z, kdim) || !make_map_f32(&tb, B, int64_t(Z) * b_rows_per_z, kdim))
+    return cudaErrorInvalidValue;
+  ScoreTcParams prm;
+  prm.C = C;
+  prm.a_rows_per_z = a_rows_per_z;
+  prm.b_rows_per_z = b_rows_per_z;
+  prm.c_stride_z = c_stride_z;
+  prm.ldc = ldc;
+  prm.m_fixed = m_fixed;
+  prm.n_fixed = n_fixed;
+  prm.kdim = kdim;
+  prm.alpha = alpha;
+  prm.wait_ns = pl->wait_ns;
+  prm.err = pl->d_state;
+  prm.heads = g.Hh;
+  for (int h = 0; h < VSA_MAX_HEADS; ++h) prm.ntv[h] = h < g.Hh ? g.ntv[h] : 0;
+  const int smem = score_tc_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((n_max + 127) / 128, (m_max + 127) / 128, Z);
+  score_tc_kernel<<<grid, kTcThreads, smem, s>>>(ta, tb, prm);
+  return cudaGetLastError();
 }
 
 // a3-a4 from the pooled descriptors already in the workspace.
@@ -276,18 +504,16 @@ cudaError_t launch_project_score(const vsa_plan* pl, const float* proj_q, const 
   const int Z = g.B * g.Hh;
   const int64_t sW = trip ? int64_t(L.kd) * p : 0;
   dim3 gp((p + 127) / 128, (g.ntv_max + 127) / 128, Z);
-  sgemm_kernel<false><<<gp, 256, 0, s>>>(g, pq, int64_t(g.ntv_max) * L.kd, L.kd, proj_q, 0, sW, p, hq,
+  sgemm_kernel<<<gp, 256, 0, s>>>(g, pq, int64_t(g.ntv_max) * L.kd, L.kd, proj_q, 0, sW, p, hq,
                                          int64_t(g.ntv_max) * p, p, L.kd, p, 1.0f);
-  sgemm_kernel<false><<<gp, 256, 0, s>>>(g, pk, int64_t(g.ntv_max) * L.kd, L.kd, proj_k, 0, sW, p, hk,
+  sgemm_kernel<<<gp, 256, 0, s>>>(g, pk, int64_t(g.ntv_max) * L.kd, L.kd, proj_k, 0, sW, p, hk,
                                          int64_t(g.ntv_max) * p, p, L.kd, p, 1.0f);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  // scores: q_hat k_hat^T / sqrt(p)
-  dim3 gs((g.ntv_max + 127) / 128, (g.ntv_max + 127) / 128, Z);
-  sgemm_kernel<true><<<gs, 256, 0, s>>>(g, hq, int64_t(g.ntv_max) * p, p, hk, int64_t(g.ntv_max) * p, 0, p, scores,
-                                        int64_t(g.ntv_max) * g.ntv_max, g.ntv_max, p, 0, 1.0f / sqrtf(float(p)));
-  return cudaGetLastError();
+  // scores: q_hat k_hat^T / sqrt(p), on the tensor cores
+  return launch_score_tc(pl, hq, g.ntv_max, hk, g.ntv_max, p, scores, int64_t(g.ntv_max) * g.ntv_max, g.ntv_max,
+                         0, 0, g.ntv_max, g.ntv_max, 1.0f / sqrtf(float(p)), s);
 }
 
 cudaError_t launch_score(const vsa_plan* pl, const void* qp, const void* kp, const float* proj_q,
@@ -340,14 +566,12 @@ cudaError_t launch_ref_score(const vsa_plan* pl, const void* kp, const float* pr
   const int Z = g.B * g.Hh;
   const int64_t sW = trip ? int64_t(L.kd) * p : 0;
   dim3 gp((p + 127) / 128, (g.n_ref + 127) / 128, Z);
-  sgemm_kernel<false><<<gp, 256, 0, s>>>(g, pr, int64_t(g.n_ref) * L.kd, L.kd, proj_k, 0, sW, p, hr,
+  sgemm_kernel<<<gp, 256, 0, s>>>(g, pr, int64_t(g.n_ref) * L.kd, L.kd, proj_k, 0, sW, p, hr,
                                          int64_t(g.n_ref) * p, p, L.kd, p, 1.0f, g.n_ref);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 gs((g.n_ref + 127) / 128, (g.ntv_max + 127) / 128, Z);
-  sgemm_kernel<true><<<gs, 256, 0, s>>>(g, hq, int64_t(g.ntv_max) * p, p, hr, int64_t(g.n_ref) * p, 0, p, scores_ref,
-                                        int64_t(g.ntv_max) * g.n_ref, g.n_ref, p, g.n_ref, 1.0f / sqrtf(float(p)));
-  return cudaGetLastError();
+  return launch_score_tc(pl, hq, g.ntv_max, hr, g.n_ref, p, scores_ref, int64_t(g.ntv_max) * g.n_ref, g.n_ref, 0,
+                         g.n_ref, g.ntv_max, g.n_ref, 1.0f / sqrtf(float(p)), s);
 }
 
 }  // namespace vsa

@@ -83,32 +83,65 @@ __global__ void __launch_bounds__(256) pack_kernel(Geometry g, const uint4* __re
   }
 }
 
-// Unpack of one packed tile per CTA (the shape of the fused pack-and-pool pass):
-// thread t moves chunk t mod CPR of rows t / CPR + RG*i; each thread resolves
-// its rows' tokens once, issues all its loads, then its stores. Unused slots
-// are neither read nor written.
-template <int CPR>
-__global__ void __launch_bounds__(256) unpack_tile_kernel(Geometry g, const uint4* __restrict__ op,
-                                                          uint4* __restrict__ o) {
-  constexpr int RG = 256 / CPR;
-  constexpr int RPT = 64 / RG;
-  const int64_t tile = blockIdx.x;    // bh * nt_max + n
-  const int n = int(tile % g.nt_max);
-  const int bh = int(tile / g.nt_max);
-  const int h = bh % g.Hh, b = bh / g.Hh;
-  const int c = threadIdx.x % CPR;
-  const int rg = threadIdx.x / CPR;
-  int tok[RPT];
-  uint4 val[RPT];
-#pragma unroll
-  for (int i = 0; i < RPT; ++i) {
-    const int s = rg + RG * i;
-    tok[i] = src_token(g, h, n, s);
-    val[i] = tok[i] >= 0 ? ld_stream(op + (tile * VSA_TILE + s) * CPR + c) : make_uint4(0, 0, 0, 0);
+// Packed row of token `tok` for head h: (tile, slot) -> tile * 64 + slot, the
+// inverse of src_token. Prefix tokens: their segment's tiles of 64 consecutive
+// tokens. Video tokens (t, y, x): the tile (t / pt, y / ph, x / pw) and the
+// token's (t, h, w) raster position inside that tile's actual extent.
+__device__ __forceinline__ int packed_row(const Geometry& g, int h, int tok) {
+  if (tok < g.n_pre_tok) {
+    int i = 0;
+#pragma unroll 1
+    while (i + 1 < g.n_seg && tok >= g.seg_tok0[i + 1]) ++i;
+    const int off = tok - g.seg_tok0[i];
+    return (g.seg_tile0[i] + off / VSA_TILE) * VSA_TILE + off % VSA_TILE;
   }
+  const int v = tok - g.n_pre_tok;
+  const int hw = g.H * g.W;
+  const int t = v / hw;
+  const int r = v - t * hw;
+  const int y = r / g.W;
+  const int x = r - y * g.W;
+  const int pt = g.pt[h], ph = g.ph[h], pw = g.pw[h];
+  const int ti = t / pt, yi = y / ph, xi = x / pw;
+  const int eh = min(ph, g.H - yi * ph), ew = min(pw, g.W - xi * pw);
+  const int slot = ((t - ti * pt) * eh + (y - yi * ph)) * ew + (x - xi * pw);
+  const int n = g.n_pre_tiles + (ti * g.nY[h] + yi) * g.nX[h] + xi;
+  return n * VSA_TILE + slot;
+}
+
+// Unpack in the output's order: one warp per token, the token's [heads, d]
+// row written front to back in 512-byte warp stores, each (head, token) row
+// gathered from its packed tile (256-byte reads, the access pattern of the
+// pack pass). Lanes first resolve one head's packed row each.
+template <int CPR>
+__global__ void __launch_bounds__(256) unpack_tok_kernel(Geometry g, const uint4* __restrict__ op,
+                                                         uint4* __restrict__ o) {
+  __shared__ int64_t src_row[8][VSA_MAX_HEADS];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int64_t n_tok = int64_t(g.B) * g.n_tokens;
+  const int per_tok = g.Hh * CPR;   // 16-byte chunks of one token's row
+  for (int64_t tk = int64_t(blockIdx.x) * 8 + wib; tk < n_tok; tk += int64_t(gridDim.x) * 8) {
+    const int b = int(tk / g.n_tokens), tok = int(tk - int64_t(b) * g.n_tokens);
+    for (int h = lane; h < g.Hh; h += 32)
+      src_row[wib][h] = (int64_t(b * g.Hh + h) * g.nt_max) * VSA_TILE + packed_row(g, h, tok);
+    __syncwarp();
+    uint4* dst = o + tk * per_tok;
+    constexpr int kBatch = 4;   // loads in flight per lane before the stores
+    for (int q0 = 0; q0 < per_tok; q0 += 32 * kBatch) {
+      uint4 val[kBatch];
 #pragma unroll
-  for (int i = 0; i < RPT; ++i)
-    if (tok[i] >= 0) o[((int64_t(b) * g.n_tokens + tok[i]) * g.Hh + h) * CPR + c] = val[i];
+      for (int u = 0; u < kBatch; ++u) {
+        const int q = q0 + 32 * u + lane;
+        val[u] = q < per_tok ? ld_stream(op + src_row[wib][q / CPR] * CPR + q % CPR) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int q = q0 + 32 * u + lane;
+        if (q < per_tok) dst[q] = val[u];
+      }
+    }
+    __syncwarp();   // src_row is rewritten for the next token
+  }
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float (&x)[8]) {
@@ -387,12 +420,15 @@ cudaError_t launch_pack_pool(const vsa_plan* p, const void* q, const void* k, co
 
 cudaError_t launch_unpack(const vsa_plan* p, const void* op, void* o, cudaStream_t s) {
   const Geometry& g = p->geo;
-  const int64_t tiles = int64_t(g.B) * g.Hh * g.nt_max;
-  if (tiles == 0) return cudaSuccess;
+  const int64_t tokens = int64_t(g.B) * g.n_tokens;
+  if (tokens == 0) return cudaSuccess;
+  const int64_t want = (tokens + 7) / 8;                // eight warps (tokens) per CTA
+  const int64_t cap = int64_t(p->num_sms) * 8;         // eight CTAs of 256 threads per SM, grid-stride
+  const unsigned grid = unsigned(want < cap ? want : cap);
   if (g.d == 128)
-    unpack_tile_kernel<16><<<unsigned(tiles), 256, 0, s>>>(g, static_cast<const uint4*>(op), static_cast<uint4*>(o));
+    unpack_tok_kernel<16><<<grid, 256, 0, s>>>(g, static_cast<const uint4*>(op), static_cast<uint4*>(o));
   else
-    unpack_tile_kernel<8><<<unsigned(tiles), 256, 0, s>>>(g, static_cast<const uint4*>(op), static_cast<uint4*>(o));
+    unpack_tok_kernel<8><<<grid, 256, 0, s>>>(g, static_cast<const uint4*>(op), static_cast<uint4*>(o));
   return cudaGetLastError();
 }
 

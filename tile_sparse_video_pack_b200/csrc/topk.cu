@@ -26,6 +26,7 @@ namespace {
 constexpr int kBins = 512;        // value bins of the first pass
 constexpr int kSmall = 64;        // candidates resolved by counting
 constexpr int kMaxWarps = 4;      // rows (warps) per CTA
+constexpr int kLoads = 16;        // score loads in flight per lane
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f + 0.0f);  // -0 -> +0
@@ -122,15 +123,28 @@ __global__ void __launch_bounds__(kMaxWarps * 32) topk_kernel(Geometry g, const 
       continue;
     }
 
-    // keys, range, NaN check
+    // keys, range, NaN check; the row streams from memory, so each lane keeps
+    // kLoads loads in flight before it uses any of them
     float lo = INFINITY, hi = -INFINITY;
     bool nan = false;
-    for (int j = lane; j < n; j += 32) {
-      const float f = srow[j] + 0.0f;
-      nan |= f != f;
-      lo = fminf(lo, f);
-      hi = fmaxf(hi, f);
-      keys[j] = order_key(f);
+    for (int j0 = 0; j0 < n; j0 += 32 * kLoads) {
+      float f[kLoads];
+#pragma unroll
+      for (int u = 0; u < kLoads; ++u) {
+        const int j = j0 + 32 * u + lane;
+        f[u] = j < n ? srow[j] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kLoads; ++u) {
+        const int j = j0 + 32 * u + lane;
+        if (j < n) {
+          const float x = f[u] + 0.0f;
+          nan |= x != x;
+          lo = fminf(lo, x);
+          hi = fmaxf(hi, x);
+          keys[j] = order_key(x);
+        }
+      }
     }
     if (__any_sync(0xffffffffu, nan)) {
       if (lane == 0) atomicOr(err, kErrBadIndex);

@@ -437,9 +437,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int nblk = (inf.n_entries + 1) >> 1;
         bool ok = true;
+        // key-list entries come from global memory: load each block's pair one block ahead
+        uint32_t na = nblk > 0 ? list[0] : 0u, nb = 1 < inf.n_entries ? list[1] : na;
         for (int j = 0; j < nblk; ++j) {
-          const int ta = int(list[2 * j] & 0xFFFFu);
-          const int tb = 2 * j + 1 < inf.n_entries ? int(list[2 * j + 1] & 0xFFFFu) : ta;
+          const int ta = int(na & 0xFFFFu);
+          const int tb = int(nb & 0xFFFFu);
+          if (j + 1 < nblk) {
+            na = list[2 * j + 2];
+            nb = 2 * j + 3 < inf.n_entries ? list[2 * j + 3] : na;
+          }
           if (!(ok = wait_bar(bar(empty0 + st), ph ^ 1, abort_flag, gerr, prm.wait_ns))) break;
           mbar_expect_tx(bar(full0 + st), 2 * (is_k && F8 ? 1 : D / 64) * kTileBytes);
           if (is_k) {   // K-major: tile a rows 0-63, tile b rows 64-127 of each 128-byte half
@@ -611,7 +617,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t* list = lists + slot * prm.list_cap;
       const int nblk = (inf.n_entries + 1) >> 1;
       float m = -INFINITY, l = 0.f;
+      // my tile's entry of each block, from global memory: loaded one block ahead so that
+      // its latency is not on the block's path
+      uint32_t e_next = sg < inf.n_entries ? list[sg] : 0u;
       for (int j = 0; j < nblk; ++j, ++g) {
+        const uint32_t e = e_next;
+        if (j + 1 < nblk) e_next = 2 * j + 2 + sg < inf.n_entries ? list[2 * j + 2 + sg] : 0u;
         const int sbuf = int(g % kSBuf);           // S / P buffer
         const uint32_t sph = (g / kSBuf) & 1;      // its phase
         const uint32_t tSb = tS + sbuf * 128 + lane_off + 64 * sg;
@@ -622,8 +633,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         }
         tc_fence_after();
-        const int ei = 2 * j + sg;
-        const uint32_t e = ei < inf.n_entries ? list[ei] : 0u;
         const int cnt = ((e >> 16) & my_bit) ? int(e >> 24) : 0;   // valid keys of my tile for my row
         float alpha = 1.f;
         uint32_t pk[32];

@@ -71,6 +71,8 @@ def parse():
                     help="Q K^T from e4m3 tiles with per-tile scales (vsa_tile_pack_pool_fp8 + vsa_sparse_attn_fp8)")
     ap.add_argument("--teacher", action="store_true",
                     help="also time the teacher tile map and report the selection's tile recall")
+    ap.add_argument("--dense-reference", action="store_true",
+                    help="also time torch's dense scaled_dot_product_attention on the same Q, K, V (context only)")
     args = ap.parse_args()
     if args.sparsity is None:
         from vsa_synth import get_config
@@ -648,8 +650,28 @@ def run_ours(args, rank, world, local_rank):
                           "algorithmic_flops": f2})
 
     teacher = teacher_measure(layer, ks) if args.teacher else None
-    return bench_line(args, layer_cfg, world, k_list(layer_cfg, args.sparsity), flops, ms_step, stages, roofline,
+    if args.dense_reference:                 # a library's dense attention on the same tensors, for context
+        qh, kh, vh = (x.transpose(1, 2) for x in (q, k, v))   # [B, heads, N, d] views
+        import torch.nn.functional as F
+        for _ in range(2):
+            F.scaled_dot_product_attention(qh, kh, vh)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            F.scaled_dot_product_attention(qh, kh, vh)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dms = e0.elapsed_time(e1) / 3
+        dflops = 4 * cfg.head_dim * cfg.batch * cfg.heads * cfg.n_tokens ** 2
+        dense_ref = {"what": "torch.nn.functional.scaled_dot_product_attention (library), dense, same q, k, v",
+                     "ms": round(dms, 3), "tflops": round(dflops / (dms * 1e-3) / 1e12, 1), "flops": dflops}
+    else:
+        dense_ref = None
+    line = bench_line(args, layer_cfg, world, k_list(layer_cfg, args.sparsity), flops, ms_step, stages, roofline,
                       e2e, clocks, stats, sweep, teacher)
+    if dense_ref is not None:
+        line["dense_reference"] = dense_ref
+    return line
 
 
 def main():

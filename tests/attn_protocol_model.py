@@ -80,9 +80,9 @@ def run(blocks_per_item, rng, slot_readers_release=True, starve=(), faults=(), h
     for i in range(V_STAGES):
         bars[f"VFULL{i}"], bars[f"VEMPTY{i}"] = Bar(1), Bar(2)      # both PV issuers release a V stage
     for i in range(S_BUFS):
-        bars[f"SFULL{i}"] = Bar(1)
+        bars[f"SFULL{i}"], bars[f"PDONE{i}"] = Bar(1), Bar(2)     # PDONE: both PV issuers' MMAs of the buffer
         for w in range(2):
-            bars[f"PFULL{w}_{i}"], bars[f"PDONE{w}_{i}"] = Bar(4), Bar(1)
+            bars[f"PFULL{w}_{i}"] = Bar(4)
     for i in range(2):
         bars[f"LFULL{i}"] = Bar(32)
         bars[f"LEMPTY{i}"] = Bar(13 if slot_readers_release else 8)
@@ -176,9 +176,7 @@ def run(blocks_per_item, rng, slot_readers_release=True, starve=(), faults=(), h
                     break
                 _check(st["K"][kst] == g, f"S({g}) reads K stage {kst} holding {st['K'][kst]}")
                 if su > 0 and "s_skips_pv_done" not in faults:   # P of block g - 2 sits in this buffer
-                    if not (ok := (yield wait(f"PDONE0_{sb}", (su - 1) & 1))):
-                        break
-                    if not (ok := (yield wait(f"PDONE1_{sb}", (su - 1) & 1))):
+                    if not (ok := (yield wait(f"PDONE{sb}", (su - 1) & 1))):
                         break
                 _check(min(st["pv_done"]) >= g - S_BUFS, f"S({g}) overwrites P({g - S_BUFS}) before PV read it")
 
@@ -229,7 +227,7 @@ def run(blocks_per_item, rng, slot_readers_release=True, starve=(), faults=(), h
 
                 def land(w=w, g=g, vst=vst, sb=sb, last=(j == nblk - 1)):
                     st["pv_done"][w] = g
-                    bars[f"PDONE{w}_{sb}"].arrive()
+                    bars[f"PDONE{sb}"].arrive()
                     bars[f"VEMPTY{vst}"].arrive()
                     if last:
                         bars["OFULL"].arrive()
@@ -262,7 +260,7 @@ def run(blocks_per_item, rng, slot_readers_release=True, starve=(), faults=(), h
                 if hold and g == 0 and not (yield wait("HOLD", 0)):
                     return
                 if j > 0 and rng.random() < 0.2:   # the O rescale waits for its previous PV
-                    if not (yield wait(f"PDONE{sg}_{(g - 1) % S_BUFS}", ((g - 1) // S_BUFS) & 1)):
+                    if not (yield wait(f"PDONE{(g - 1) % S_BUFS}", ((g - 1) // S_BUFS) & 1)):
                         return
                     _check(st["pv_done"][sg] >= g - 1, "O rescaled while the previous PV accumulates")
                 bars[f"PFULL{sg}_{sbuf}"].arrive()

@@ -29,11 +29,11 @@
 //           online softmax (running max, row sum, partial output O_w); the
 //           epilogue merges the two partial softmaxes of each row.
 //
-// One thread's tcgen05.mma stream runs one M = 128, K = 16 instruction at a
-// time, about as long for N = 128 as for N = 256, so S and the two PV halves
-// come from three issuing threads. The softmax warpgroups never wait for each
-// other inside an item, so one computes exponentials while the other loads
-// and reduces its scores.
+// Each mbarrier wait and commit costs an issuing thread tens of cycles next
+// to a 64-cycle MMA, so S and the two PV halves come from three issuing
+// threads, each waiting only on its own barriers. The softmax warpgroups never
+// wait for each other inside an item, so one computes exponentials while the
+// other loads and reduces its scores.
 //
 // TMEM holds the two S buffers and the two partial outputs; shared memory the
 // Q pair and the K and V stages, in the canonical 128-byte-swizzled UMMA
@@ -153,9 +153,9 @@ struct Smem {
 // barrier indices
 enum {
   B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KEMPTY0 = B_KFULL0 + 4, B_VFULL0 = B_KEMPTY0 + 4, B_VEMPTY0 = B_VFULL0 + 4,
-  // P_FULL / P_DONE: [softmax warpgroup][S buffer]
+  // P_FULL: [softmax warpgroup][S buffer]; P_DONE: [S buffer], both PV MMAs of the buffer's block
   B_SFULL0 = B_VEMPTY0 + 4, B_PFULL0 = B_SFULL0 + kSBuf, B_PDONE0 = B_PFULL0 + 2 * kSBuf,
-  B_LFULL0 = B_PDONE0 + 2 * kSBuf, B_LFULL1, B_LEMPTY0, B_LEMPTY1, B_OFULL, B_OFREE, B_LX, B_DRAIN, B_HOLD, B_COUNT
+  B_LFULL0 = B_PDONE0 + kSBuf, B_LFULL1, B_LEMPTY0, B_LEMPTY1, B_OFULL, B_OFREE, B_LX, B_DRAIN, B_HOLD, B_COUNT
 };
 static_assert(B_COUNT <= 40, "barrier slots");
 
@@ -230,10 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_VEMPTY0 + i), 2);   // both PV issuers
     }
     for (int i = 0; i < kSBuf; ++i) mbar_init(bar(B_SFULL0 + i), 1);
-    for (int i = 0; i < 2 * kSBuf; ++i) {
-      mbar_init(bar(B_PFULL0 + i), kSmWarps / 2);   // the four warps of one softmax warpgroup
-      mbar_init(bar(B_PDONE0 + i), 1);
-    }
+    for (int i = 0; i < 2 * kSBuf; ++i) mbar_init(bar(B_PFULL0 + i), kSmWarps / 2);   // one softmax warpgroup
+    for (int i = 0; i < kSBuf; ++i) mbar_init(bar(B_PDONE0 + i), 2);   // both PV issuers
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_LFULL0 + i), 32);
       mbar_init(bar(B_LEMPTY0 + i), kSmWarps + 5);   // + S issuer, two PV issuers, two producer lanes
@@ -501,9 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (nblk == 0) tc_commit(bar(B_QEMPTY));   // a rejected item without prefix tiles
         for (int j = 0; j < nblk; ++j) {
           if (!(ok = wait_bar(bar(B_KFULL0 + kst), kph, abort_flag, gerr, prm.wait_ns))) break;
-          // the buffer's previous P has been read by both PV MMAs
+          // the buffer's previous P has been read by both PV MMAs (one barrier counts both)
           if (su > 0 && !(ok = wait_bar(bar(B_PDONE0 + sb), (su - 1) & 1, abort_flag, gerr, prm.wait_ns))) break;
-          if (su > 0 && !(ok = wait_bar(bar(B_PDONE0 + kSBuf + sb), (su - 1) & 1, abort_flag, gerr, prm.wait_ns))) break;
           tc_fence_after();
           const uint64_t dk = dk0 + ((kst * L::kKBytes) >> 4);
           if constexpr (F8) {
@@ -569,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t boff = (w * (D / 64) * 8192 + kk * 2048) >> 4;
             tc_mma_ts(tO0 + w * 128, pcol + kk * 8, dv + boff, idPV, (j == 0 && kk == 0) ? 0u : 1u);
           }
-          tc_commit(bar(B_PDONE0 + w * kSBuf + sb));
+          tc_commit(bar(B_PDONE0 + sb));
           tc_commit(bar(B_VEMPTY0 + vst));
           if (j == nblk - 1) tc_commit(bar(B_OFULL));
           if (++vst == L::kVStages) {
@@ -709,10 +706,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P over the first half of my consumed S columns
         tmem_st32u(tSb, pk);
         // earlier blocks of this item sit in O_sg at the old max: rescale it
-        // once my previous PV has finished accumulating into it
+        // once the previous block's PV MMAs have finished accumulating
         if (__any_sync(0xffffffffu, j > 0 && alpha != 1.f)) {
           const uint32_t gp = g - 1;
-          ok = wait_bar(bar(B_PDONE0 + sg * kSBuf + int(gp % kSBuf)), (gp / kSBuf) & 1, abort_flag, gerr, prm.wait_ns);
+          ok = wait_bar(bar(B_PDONE0 + int(gp % kSBuf)), (gp / kSBuf) & 1, abort_flag, gerr, prm.wait_ns);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1

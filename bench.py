@@ -49,6 +49,7 @@ def metric_for(cfg):
     return (f"ms per attention layer, {cfg.name} workload ({cfg.n_video_tokens} video tokens), "
             f"sparsity {cfg.sparsity[0]} (other levels in sweep); effective TFLOP/s")
 KERNELS_PER_STEP = 7  # pack + pool 1, score 3 (2 projections, scores), select 1, attention 1, unpack 1
+KERNELS_PER_STEP_DIRECT = 6  # pool 1, score 3, select 1, attention straight from q, k, v into o 1
 
 
 def parse():
@@ -67,6 +68,9 @@ def parse():
                     help="multi-GPU: each rank its own layer (weak scaling) or its block of one layer's heads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
+    ap.add_argument("--direct", action="store_true",
+                    help="attention straight from the token-major q, k, v (vsa_tile_pool + vsa_sparse_attn_direct, "
+                         "no packed copies; slower) instead of pack + pool, attention on packed tiles, unpack")
     ap.add_argument("--fp8", action="store_true",
                     help="Q K^T from e4m3 tiles with per-tile scales (vsa_tile_pack_pool_fp8 + vsa_sparse_attn_fp8)")
     ap.add_argument("--teacher", action="store_true",
@@ -102,7 +106,7 @@ def attn_source_sha1() -> str:
         return hashlib.sha1(f.read()).hexdigest()
 
 
-def measured_traffic(config: str, sparsity: float, heads: int):
+def measured_traffic(config: str, sparsity: float, heads: int, path: str = "packed"):
     """DRAM bytes per attention launch from the committed ncu capture, if it is of this kernel source.
 
     The capture runs a smaller case (fewer heads) of the same workload; bytes grow
@@ -118,7 +122,7 @@ def measured_traffic(config: str, sparsity: float, heads: int):
                 a, b = ln.split("=", 1)
                 kv[a.strip()] = b.strip()
     if (kv.get("attn_source_sha1") != attn_source_sha1() or kv.get("config") != config
-            or float(kv.get("sparsity", "nan")) != sparsity):
+            or float(kv.get("sparsity", "nan")) != sparsity or kv.get("path", "packed") != path):
         return None
     per_head = (float(kv["dram_bytes_read"]) + float(kv["dram_bytes_write"])) / float(kv["heads"])
     return int(per_head * heads)
@@ -177,9 +181,11 @@ def attn_roofline(args, cfg, peaks, flops, attn_ms):
     peak = round(peaks["bf16_tflops"] * mix, 1)
     return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "traffic": None if args.fp8 else measured_traffic(args.config, args.sparsity, cfg.heads),
+            "traffic": None if args.fp8 else measured_traffic(args.config, args.sparsity, cfg.heads,
+                                                              getattr(args, "path", "packed")),
             "kernel": "attn_kernel<128, fp8> (vsa_sparse_attn_fp8; e4m3 Q K^T, bf16 P V)" if args.fp8
-                      else "attn_kernel (vsa_sparse_attn)",
+                      else ("attn_kernel, tiles straight from token-major q, k, v (vsa_sparse_attn_direct)"
+                            if getattr(args, "path", "packed") == "direct" else "attn_kernel (vsa_sparse_attn)"),
             "peak_kind": (f"half e4m3 (2x bf16, nominal ratio), half bf16: 4/3 x bf16 dense, burst, "
                           f"{peaks['source']}") if args.fp8 else f"bf16 dense, burst, {peaks['source']}",
             "frac_of_sustained_peak": round(achieved / (peaks["bf16_tflops_sustained"] * mix), 4),
@@ -207,7 +213,9 @@ def bench_line(args, cfg, world, ks, flops, ms_step, stages, roofline, e2e, cloc
         "score_select_share": round((stages["score"] + stages["select"]) / sum(stages.values()), 4),
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": (KERNELS_PER_STEP + (4 if ref else 0)) * args.steps,
+        "gpu_launches": ((KERNELS_PER_STEP_DIRECT if getattr(args, "path", "packed") == "direct" else KERNELS_PER_STEP)
+                         + (4 if ref else 0)) * args.steps,
+        "path": getattr(args, "path", "packed"),
         "clocks": clocks,
         "attention_computed_pct": round(100.0 * stats["computed_pairs"] / stats["dense_pairs"], 2),
         "sweep": sweep,
@@ -532,7 +540,8 @@ def run_ours(args, rank, world, local_rank):
         return max_over_ranks_on(x, dev, world)
 
     def timed_layer(sparsity, steps, warmup, sample_clocks):
-        layer = T.TileSparseAttention.from_config(cfg, sparsity, pq, pk)
+        layer = T.TileSparseAttention.from_config(cfg, sparsity, pq, pk, direct=args.direct and not args.fp8)
+        args.path = "direct" if layer.direct else "packed"
         out = torch.empty_like(q)
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
         for _ in range(warmup):
@@ -547,9 +556,21 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         b, p = layer.bufs, layer.plan
         f8 = p.allocate_fp8() if args.fp8 else None
+        direct = layer.direct and f8 is None
         for i in range(steps):
             e = ev[i]
             e[0].record(stream)
+            if direct:                      # no packed copies: tiles straight from q, k, v; o written directly
+                p.tile_pool(q, k, b["workspace"])
+                e[1].record(stream)
+                p.tile_score_pooled(pq, pk, b["scores"], b["workspace"])
+                e[2].record(stream)
+                p.topk_select(b["scores"], b["idx"])
+                e[3].record(stream)
+                p.sparse_attn_direct(q, k, v, b["idx"], out)
+                e[4].record(stream)
+                e[5].record(stream)
+                continue
             if f8 is not None:
                 p.tile_pack_pool_fp8(q, k, v, b["qp"], b["kp"], b["vp"], f8["qp8"], f8["kp8"], f8["q_scale"],
                                      f8["k_scale"], b["workspace"])
@@ -577,8 +598,9 @@ def run_ours(args, rank, world, local_rank):
         clocks = clk.stop() if clk else None
         layer.plan.check()
         total = sum(ev[i][0].elapsed_time(ev[i][5]) for i in range(steps))
+        names = ("pool", "score", "select", "attn") if direct else ("pack_pool", "score", "select", "attn", "unpack")
         stages = {name: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps)) / steps
-                  for j, name in enumerate(("pack_pool", "score", "select", "attn", "unpack"))}
+                  for j, name in enumerate(names)}
         ms_step = max_over_ranks(total / steps)
         stats = layer.plan.stats()
         return layer, out, ms_step, stages, clocks, stats

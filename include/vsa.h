@@ -117,6 +117,9 @@ typedef struct {
   int64_t ref_score_elems;              /* batch*heads*ntv_max*n_ref_tiles (fp32) */
   int64_t ref_index_elems;              /* batch*heads*ntv_max*k_ref_max (int32) */
   int64_t tile_scale_elems;             /* batch*heads*nt_max: one fp32 scale per packed tile (fp8 path) */
+  int32_t direct_attn;                  /* 1: vsa_tile_pool + vsa_sparse_attn_direct can run this plan (no
+                                           packed copies, slower); see vsa_sparse_attn_direct */
+  int32_t reserved0;
 } vsa_plan_info;
 
 typedef struct vsa_plan vsa_plan;
@@ -269,6 +272,37 @@ VSA_API vsa_status vsa_sparse_attn(vsa_plan* plan, const void* qp, const void* k
 
 /* a7. Inverse of the pack permutation: [B, heads, nt_max, 64, d] -> [B, N, heads, d]. */
 VSA_API vsa_status vsa_tile_unpack(vsa_plan* plan, const void* op, void* o, void* stream);
+
+/* The layer without packed copies (the other half of fusing a1 and a2: tiles
+ * straight from the token-major tensors), for callers that cannot hold the
+ * packed Q, K, V and O (four tensors the size of Q). It is the slower path:
+ * a tile of the token-major layout is 64 rows 128 or 256 bytes long spread
+ * over the tensor, which the TMA engine fetches several times more slowly
+ * than one contiguous packed tile, so the attention takes about three times
+ * as long as on packed tiles (full clip: 181 ms against 59 ms); the pack
+ * pass costs 0.7 ms. For plans whose vsa_plan_info direct_attn is 1 --
+ * batch 1, no reference segments (seg_ref), head_dim 64 or 128, every head's
+ * video tiles whole along h and w (only tiles at the far end of t may be
+ * partial), at most four distinct tile shapes -- the two calls below replace
+ * vsa_tile_pack_pool, vsa_sparse_attn and vsa_tile_unpack; any other plan
+ * gets VSA_ERR_UNSUPPORTED from them.
+ *
+ * vsa_tile_pool: a2 alone -- the score descriptors of every video tile, pooled
+ * from the token-major q and k ([1, N, heads, d] bf16, 16-byte aligned) into
+ * `workspace` exactly as vsa_tile_pack_pool pools them; follow with
+ * vsa_tile_score_pooled on the same workspace. */
+VSA_API vsa_status vsa_tile_pool(vsa_plan* plan, const void* q, const void* k, void* workspace, void* stream);
+
+/* a6 + a7 without packed tiles: the attention of vsa_sparse_attn, reading each
+ * tile of q, k, v ([1, N, heads, d] bf16, token-major, 16-byte aligned) with
+ * one multi-dimensional TMA box (a prefix tile: 64 consecutive tokens of its
+ * segment; a video tile: its (pt, ph, pw) block of the grid) and writing o
+ * ([1, N, heads, d] bf16, token-major) directly -- the same values, bit for
+ * bit, as vsa_sparse_attn followed by vsa_tile_unpack. idx, k_per_head and lse
+ * (packed rows, [B, heads, nt_max, 64], may be NULL) as for vsa_sparse_attn. */
+VSA_API vsa_status vsa_sparse_attn_direct(vsa_plan* plan, const void* q, const void* k, const void* v,
+                                          const int32_t* idx, const int32_t* k_per_head, void* o, float* lse,
+                                          void* stream);
 
 /* R2VA budgets, scores of the reference tiles: for video query tile i and
  * reference tile r (the r-th tile of the segments marked in seg_ref, in

@@ -185,6 +185,31 @@ struct AttnParams {
   int32_t hold;            // test hook: the softmax waits, at its first block, on a barrier nothing arrives on
 };
 
+// Tiles straight from the token-major Q, K, V [1, N, heads, d] (no packed
+// copies): a prefix tile is a 3-D box (64 channels, 1 head, 64 tokens) of the
+// sequence, a video tile of head h a 5-D box (64 channels, 1 head, pw, ph, pt)
+// of the video grid [T][H][W][heads][d], which TMA writes into shared memory
+// in the same (t, h, w) row order and swizzle as the packed tile's 2-D box.
+// Rows past a prefix segment hold the next tokens (masked keys, unwritten
+// query rows); rows past the grid's far edge in t are zero-filled, as the
+// packed tile's. O is written token-major.
+constexpr int kMaxShapes = 4;   // distinct (pt, ph, pw) among the heads
+struct DirectMaps {
+  CUtensorMap pre[3];                  // Q, K, V over the whole sequence
+  CUtensorMap vid[kMaxShapes][3];      // Q, K, V over the video grid, per tile shape
+  int32_t n_pre_tok, n_pre_tiles, n_seg, T, H, W;
+  int32_t seg_tok0[VSA_MAX_SEGMENTS + 1], seg_tile0[VSA_MAX_SEGMENTS + 1];
+  int32_t shp[kMaxShapes][3];          // pt, ph, pw
+  int8_t shape_of[VSA_MAX_HEADS];      // shape index of each head
+};
+
+__device__ __forceinline__ int prefix_tile_token0(const DirectMaps& dm, int tile) {
+  int s = 0;
+#pragma unroll 1
+  while (s + 1 < dm.n_seg && tile >= dm.seg_tile0[s + 1]) ++s;
+  return dm.seg_tok0[s] + (tile - dm.seg_tile0[s]) * VSA_TILE;
+}
+
 __device__ __forceinline__ int warp_excl_scan(int v, int lane, int* total) {
   int x = v;
 #pragma unroll
@@ -196,13 +221,14 @@ __device__ __forceinline__ int warp_excl_scan(int v, int lane, int* total) {
   return x - v;
 }
 
-template <int D, bool F8 = false>
+template <int D, bool F8 = false, bool DIRECT = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv,
-                const __grid_constant__ AttnParams prm) {
+                const __grid_constant__ AttnParams prm, const __grid_constant__ DirectMaps dm) {
   using L = Smem<D, F8>;
   static_assert(!F8 || D == 128, "fp8 Q K^T: one 128-byte swizzle row per token");
+  static_assert(!(F8 && DIRECT), "the fp8 instance reads the packed e4m3 copies");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -412,6 +438,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int full0 = is_k ? B_KFULL0 : B_VFULL0;
       const int empty0 = is_k ? B_KEMPTY0 : B_VEMPTY0;
       const int nst = is_k ? L::kKStages : L::kVStages;
+      // box c (channels 64c .. 64c + 63) of tile `tile` of tensor m (0 Q, 1 K, 2 V) of (batch, head) bh
+      auto load_box = [&](uint32_t dst, int m, const CUtensorMap* map2d, int c, int bh, int tile, uint32_t fb) {
+        if constexpr (DIRECT) {
+          const int h = bh % prm.heads;
+          if (tile < dm.n_pre_tiles) {
+            tma_load_3d(dst, &dm.pre[m], 64 * c, h, prefix_tile_token0(dm, tile), fb);
+          } else {
+            const int sh = dm.shape_of[h];
+            const int pt = dm.shp[sh][0], ph = dm.shp[sh][1], pw = dm.shp[sh][2];
+            const int nX = dm.W / pw, nYX = (dm.H / ph) * nX;
+            const int v = tile - dm.n_pre_tiles;
+            const int ti = v / nYX, yi = (v - ti * nYX) / nX, xi = v - ti * nYX - yi * nX;
+            tma_load_5d(dst, &dm.vid[sh][m], 64 * c, h, xi * pw, yi * ph, ti * pt, fb);
+          }
+        } else {
+          tma_load_2d(dst, map2d, 64 * c, (bh * prm.nt_max + tile) * 64, fb);
+        }
+      };
       uint32_t g = 0;          // key blocks issued
       int st = 0;              // stage of block g (g mod nst)
       uint32_t ph = 0;         // phase of that stage ((g / nst) & 1)
@@ -422,14 +466,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const ItemInfo inf = info[slot];
         if (inf.end) break;
         const uint32_t* list = lists + slot * prm.list_cap;
-        const int row_base = inf.bh * prm.nt_max;
         if (is_k) {   // rows 0-63: tile qa, rows 64-127: tile qb (qa again when there is none)
           if (!wait_bar(bar(B_QEMPTY), (it & 1) ^ 1, abort_flag, gerr, prm.wait_ns)) break;
           mbar_expect_tx(bar(B_QFULL), 2 * (F8 ? 1 : D / 64) * kTileBytes);
           const int qb = inf.qb >= 0 ? inf.qb : inf.qa;
           for (int c = 0; c < (F8 ? 1 : D / 64); ++c) {   // 64-row boxes of 128 bytes per row
-            tma_load_2d(sbase + L::oQ + c * L::kHalfBytes, &tq, 64 * c, (row_base + inf.qa) * 64, bar(B_QFULL));
-            tma_load_2d(sbase + L::oQ + c * L::kHalfBytes + 8192, &tq, 64 * c, (row_base + qb) * 64, bar(B_QFULL));
+            load_box(sbase + L::oQ + c * L::kHalfBytes, 0, &tq, c, inf.bh, inf.qa, bar(B_QFULL));
+            load_box(sbase + L::oQ + c * L::kHalfBytes + 8192, 0, &tq, c, inf.bh, qb, bar(B_QFULL));
           }
           ++issuedQ;
         }
@@ -449,14 +492,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (is_k) {   // K-major: tile a rows 0-63, tile b rows 64-127 of each 128-byte half
             const uint32_t sk = sbase + L::oK + st * L::kKBytes;
             for (int c = 0; c < (F8 ? 1 : D / 64); ++c) {
-              tma_load_2d(sk + c * L::kHalfBytes, map, 64 * c, (row_base + ta) * 64, bar(full0 + st));
-              tma_load_2d(sk + c * L::kHalfBytes + 8192, map, 64 * c, (row_base + tb) * 64, bar(full0 + st));
+              load_box(sk + c * L::kHalfBytes, 1, map, c, inf.bh, ta, bar(full0 + st));
+              load_box(sk + c * L::kHalfBytes + 8192, 1, map, c, inf.bh, tb, bar(full0 + st));
             }
           } else {      // MN-major: tile a then tile b, each as D/64 boxes of 64 keys x 64 columns
             const uint32_t sv = sbase + L::oV + st * L::kVBytes;
             for (int c = 0; c < D / 64; ++c) {
-              tma_load_2d(sv + c * 8192, map, 64 * c, (row_base + ta) * 64, bar(full0 + st));
-              tma_load_2d(sv + (D / 64) * 8192 + c * 8192, map, 64 * c, (row_base + tb) * 64, bar(full0 + st));
+              load_box(sv + c * 8192, 2, map, c, inf.bh, ta, bar(full0 + st));
+              load_box(sv + (D / 64) * 8192 + c * 8192, 2, map, c, inf.bh, tb, bar(full0 + st));
             }
           }
           ++g;
@@ -754,6 +797,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float w0 = a0 * inv, w1 = a1 * inv;
       const size_t orow = (size_t(inf.bh) * prm.nt_max + (tile >= 0 ? tile : 0)) * 64 + slot_r;
       uint4* dst = reinterpret_cast<uint4*>(prm.out + orow * D + sg * (D / 2));
+      bool store = write;
+      if constexpr (DIRECT) {   // token-major O: only the tile's real tokens
+        store = valid;
+        const int h = inf.bh % prm.heads;
+        int tok = 0;
+        if (valid) {
+          if (tile < dm.n_pre_tiles) {
+            tok = prefix_tile_token0(dm, tile) + slot_r;
+          } else {
+            const int sh = dm.shape_of[h];
+            const int pt = dm.shp[sh][0], ph = dm.shp[sh][1], pw = dm.shp[sh][2];
+            const int nX = dm.W / pw, nYX = (dm.H / ph) * nX;
+            const int v = tile - dm.n_pre_tiles;
+            const int ti = v / nYX, yi = (v - ti * nYX) / nX, xi = v - ti * nYX - yi * nX;
+            const int st = slot_r / (ph * pw), sy = (slot_r / pw) % ph, sx = slot_r % pw;
+            tok = dm.n_pre_tok + ((ti * pt + st) * dm.H + yi * ph + sy) * dm.W + xi * pw + sx;
+          }
+        }
+        dst = reinterpret_cast<uint4*>(prm.out + (size_t(tok) * prm.heads + h) * D + sg * (D / 2));
+      }
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t o0[32], o1[32];
@@ -761,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tO0 + 128 + lane_off + sg * (D / 2) + 32 * c, o1);
         tmem_wait_ld(o0);
         reg_fence(o1);
-        if (write) {
+        if (store) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             float v[8];
@@ -802,17 +865,11 @@ int attn_smem_bytes(int list_cap) {
   return 1024 + int(Smem<128>::oEnd);
 }
 
-cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp, const int32_t* idx,
-                        const int32_t* idx_ref, const int32_t* k, void* op, float* lse, cudaStream_t s,
-                        const float* q_scale, const float* k_scale) {
+namespace {
+
+AttnParams attn_params(const vsa_plan* p, const int32_t* idx, const int32_t* idx_ref, const int32_t* k, void* op,
+                       float* lse, const float* q_scale, const float* k_scale) {
   const Geometry& g = p->geo;
-  const int64_t rows = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE;
-  const bool f8 = q_scale != nullptr;      // qp, kp are e4m3 tiles with per-tile scales
-  if (f8 && g.d != 128) return cudaErrorInvalidValue;
-  CUtensorMap tq, tk, tv;
-  const bool maps = f8 ? make_map_u8(&tq, qp, rows, g.d) && make_map_u8(&tk, kp, rows, g.d)
-                       : make_map(&tq, qp, rows, g.d) && make_map(&tk, kp, rows, g.d);
-  if (!maps || !make_map(&tv, vp, rows, g.d)) return cudaErrorInvalidValue;
   AttnParams prm;
   prm.q_scale = q_scale;
   prm.k_scale = k_scale;
@@ -845,25 +902,111 @@ cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void*
     prm.k[h] = h < g.Hh ? k[h] : 0;
     prm.k_ref[h] = h < g.Hh ? g.k_ref[h] : 0;
   }
-  // reset the work counter and the pair count
+  return prm;
+}
+
+// The work counter and pair count reset, then the persistent launch.
+template <int D, bool F8, bool DIRECT>
+cudaError_t attn_launch(vsa_plan* p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const AttnParams& prm, const DirectMaps& dm, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(p->d_state + 1, 0, 12, s);
   if (e != cudaSuccess) return e;
   const int smem = p->attn_smem_bytes;
   const int grid = int(p->n_items < p->num_sms ? p->n_items : p->num_sms);
-  if (f8) {
-    e = cudaFuncSetAttribute(attn_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attn_kernel<128, true><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm);
-  } else if (g.d == 128) {
-    e = cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attn_kernel<128><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm);
-  } else {
-    e = cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attn_kernel<64><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm);
-  }
+  e = cudaFuncSetAttribute(attn_kernel<D, F8, DIRECT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  attn_kernel<D, F8, DIRECT><<<grid, kThreads, smem, s>>>(tq, tk, tv, prm, dm);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn(vsa_plan* p, const void* qp, const void* kp, const void* vp, const int32_t* idx,
+                        const int32_t* idx_ref, const int32_t* k, void* op, float* lse, cudaStream_t s,
+                        const float* q_scale, const float* k_scale) {
+  const Geometry& g = p->geo;
+  const int64_t rows = int64_t(g.B) * g.Hh * g.nt_max * VSA_TILE;
+  const bool f8 = q_scale != nullptr;      // qp, kp are e4m3 tiles with per-tile scales
+  if (f8 && g.d != 128) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv;
+  const bool maps = f8 ? make_map_u8(&tq, qp, rows, g.d) && make_map_u8(&tk, kp, rows, g.d)
+                       : make_map(&tq, qp, rows, g.d) && make_map(&tk, kp, rows, g.d);
+  if (!maps || !make_map(&tv, vp, rows, g.d)) return cudaErrorInvalidValue;
+  const AttnParams prm = attn_params(p, idx, idx_ref, k, op, lse, q_scale, k_scale);
+  static const DirectMaps kNoMaps = {};
+  if (f8) return attn_launch<128, true, false>(p, tq, tk, tv, prm, kNoMaps, s);
+  if (g.d == 128) return attn_launch<128, false, false>(p, tq, tk, tv, prm, kNoMaps, s);
+  return attn_launch<64, false, false>(p, tq, tk, tv, prm, kNoMaps, s);
+}
+
+bool direct_attn_supported(const vsa_plan* p) {
+  const Geometry& g = p->geo;
+  if (g.B != 1 || g.n_ref != 0 || (g.d != 64 && g.d != 128) || g.n_seg > VSA_MAX_SEGMENTS) return false;
+  int shapes[kMaxShapes][3], n = 0;
+  for (int h = 0; h < g.Hh; ++h) {
+    if (g.H % g.ph[h] != 0 || g.W % g.pw[h] != 0) return false;   // tiles partial only along t
+    int i = 0;
+    while (i < n && !(shapes[i][0] == g.pt[h] && shapes[i][1] == g.ph[h] && shapes[i][2] == g.pw[h])) ++i;
+    if (i == n) {
+      if (n == kMaxShapes) return false;
+      shapes[n][0] = g.pt[h];
+      shapes[n][1] = g.ph[h];
+      shapes[n][2] = g.pw[h];
+      ++n;
+    }
+  }
+  return true;
+}
+
+cudaError_t launch_attn_direct(vsa_plan* p, const void* q, const void* k, const void* v, const int32_t* idx,
+                               const int32_t* kk, void* o, float* lse, cudaStream_t s) {
+  const Geometry& g = p->geo;
+  if (!direct_attn_supported(p)) return cudaErrorInvalidValue;
+  const cuuint64_t e2 = 2;   // bf16 bytes
+  const cuuint64_t D = cuuint64_t(g.d), Hh = cuuint64_t(g.Hh);
+  DirectMaps dm = {};
+  dm.n_pre_tok = g.n_pre_tok;
+  dm.n_pre_tiles = g.n_pre_tiles;
+  dm.n_seg = g.n_seg;
+  dm.T = g.T;
+  dm.H = g.H;
+  dm.W = g.W;
+  for (int i = 0; i <= VSA_MAX_SEGMENTS; ++i) {
+    dm.seg_tok0[i] = g.seg_tok0[i];
+    dm.seg_tile0[i] = g.seg_tile0[i];
+  }
+  const void* base[3] = {q, k, v};
+  int n = 0;
+  for (int h = 0; h < g.Hh; ++h) {
+    int i = 0;
+    while (i < n && !(dm.shp[i][0] == g.pt[h] && dm.shp[i][1] == g.ph[h] && dm.shp[i][2] == g.pw[h])) ++i;
+    if (i == n) {
+      dm.shp[n][0] = g.pt[h];
+      dm.shp[n][1] = g.ph[h];
+      dm.shp[n][2] = g.pw[h];
+      // the video grid [T][H][W][heads][d] of each tensor, boxes of one tile of this shape
+      const cuuint64_t dims[5] = {D, Hh, cuuint64_t(g.W), cuuint64_t(g.H), cuuint64_t(g.T)};
+      const cuuint64_t strides[4] = {D * e2, Hh * D * e2, cuuint64_t(g.W) * Hh * D * e2,
+                                     cuuint64_t(g.H) * g.W * Hh * D * e2};
+      const cuuint32_t box[5] = {64, 1, cuuint32_t(g.pw[h]), cuuint32_t(g.ph[h]), cuuint32_t(g.pt[h])};
+      for (int m = 0; m < 3; ++m) {
+        const char* vb = static_cast<const char*>(base[m]) + size_t(g.n_pre_tok) * Hh * D * e2;
+        if (!make_map_nd(&dm.vid[n][m], vb, 5, dims, strides, box)) return cudaErrorInvalidValue;
+      }
+      ++n;
+    }
+    dm.shape_of[h] = int8_t(i);
+  }
+  {  // the whole sequence [N][heads][d], boxes of 64 tokens (prefix tiles)
+    const cuuint64_t dims[3] = {D, Hh, cuuint64_t(g.n_tokens)};
+    const cuuint64_t strides[2] = {D * e2, Hh * D * e2};
+    const cuuint32_t box[3] = {64, 1, 64};
+    for (int m = 0; m < 3; ++m)
+      if (!make_map_nd(&dm.pre[m], base[m], 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  const AttnParams prm = attn_params(p, idx, nullptr, kk, o, lse, nullptr, nullptr);
+  if (g.d == 128) return attn_launch<128, false, true>(p, dm.pre[0], dm.pre[1], dm.pre[2], prm, dm, s);
+  return attn_launch<64, false, true>(p, dm.pre[0], dm.pre[1], dm.pre[2], prm, dm, s);
 }
 
 }  // namespace vsa

@@ -169,7 +169,9 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float (&x)[8]) {
 // scale) (correctly rounded fp32 division, then rounded to nearest even and
 // saturated) -- per-tile 8-bit Q K^T, as the tile-skipping kernels on the Veda
 // page run it.
-template <int CPR, bool TRIP, bool QUANT>
+// PACK = false: the pooling alone (no V, no packed copies), for the path whose
+// attention reads the token-major tensors directly; CTAs of prefix tiles exit.
+template <int CPR, bool TRIP, bool QUANT, bool PACK = true>
 __global__ void __launch_bounds__(256) pack_pool_kernel(Geometry g, const uint4* __restrict__ q,
                                                         const uint4* __restrict__ k,
                                                         const uint4* __restrict__ v, uint4* __restrict__ qp,
@@ -193,6 +195,7 @@ __global__ void __launch_bounds__(256) pack_pool_kernel(Geometry g, const uint4*
   const int rg = threadIdx.x / CPR;
   const int vt = n - g.n_pre_tiles;
   const bool pool = vt >= 0 && vt < g.ntv[h];   // uniform over the CTA
+  if (!PACK && !pool) return;
   float st[NS][2][8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
@@ -217,11 +220,13 @@ __global__ void __launch_bounds__(256) pack_pool_kernel(Geometry g, const uint4*
       const int64_t src = ((int64_t(b) * g.n_tokens + tok) * g.Hh + h) * CPR + c;
       a = ld_stream(q + src);
       bb = ld_stream(k + src);
-      cc = ld_stream(v + src);
+      if (PACK) cc = ld_stream(v + src);
     }
-    qp[dst] = a;
-    kp[dst] = bb;
-    vp[dst] = cc;
+    if (PACK) {
+      qp[dst] = a;
+      kp[dst] = bb;
+      vp[dst] = cc;
+    }
     if constexpr (QUANT) {
       keep_q[i] = a;
       keep_k[i] = bb;
@@ -374,6 +379,32 @@ cudaError_t launch_pack(const vsa_plan* p, const void* q, const void* k, const v
     pack_kernel<16><<<grid, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4);
   else
     pack_kernel<8><<<grid, 256, 0, s>>>(g, q4, k4, v4, qp4, kp4, vp4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool(const vsa_plan* p, const void* q, const void* k, float* pooled_q, float* pooled_k,
+                        cudaStream_t s) {
+  const Geometry& g = p->geo;
+  const int64_t tiles = int64_t(g.B) * g.Hh * g.nt_max;
+  const bool trip = p->desc.score_mode == VSA_SCORE_TRIPPOOL;
+  auto* q4 = static_cast<const uint4*>(q);
+  auto* k4 = static_cast<const uint4*>(k);
+  const int32_t* cnt = p->d_tile_count;
+  if (g.d == 128) {
+    if (trip)
+      pack_pool_kernel<16, true, false, false><<<tiles, 256, 0, s>>>(g, q4, k4, nullptr, nullptr, nullptr, nullptr, cnt,
+                                                                     pooled_q, pooled_k, nullptr, nullptr, nullptr, nullptr);
+    else
+      pack_pool_kernel<16, false, false, false><<<tiles, 256, 0, s>>>(g, q4, k4, nullptr, nullptr, nullptr, nullptr, cnt,
+                                                                      pooled_q, pooled_k, nullptr, nullptr, nullptr, nullptr);
+  } else {
+    if (trip)
+      pack_pool_kernel<8, true, false, false><<<tiles, 256, 0, s>>>(g, q4, k4, nullptr, nullptr, nullptr, nullptr, cnt,
+                                                                    pooled_q, pooled_k, nullptr, nullptr, nullptr, nullptr);
+    else
+      pack_pool_kernel<8, false, false, false><<<tiles, 256, 0, s>>>(g, q4, k4, nullptr, nullptr, nullptr, nullptr, cnt,
+                                                                     pooled_q, pooled_k, nullptr, nullptr, nullptr, nullptr);
+  }
   return cudaGetLastError();
 }
 

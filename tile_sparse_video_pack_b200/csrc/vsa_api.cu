@@ -268,6 +268,7 @@ vsa_status vsa_plan_create(const vsa_desc* desc, vsa_plan** out) {
     }
   p->n_items = int64_t(items.size());
   info.attn_work_items = p->n_items;
+  info.direct_attn = vsa::direct_attn_supported(p) ? 1 : 0;
   p->wait_ns = vsa::kDefaultWaitNs;
   p->test_hold = 0;
 
@@ -489,6 +490,37 @@ vsa_status vsa_sparse_attn(vsa_plan* p, const void* qp, const void* kp, const vo
   p->stats.calls_attn++;
   if (vsa::launch_attn(p, qp, kp, vp, idx, nullptr, k, op, lse, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_tile_pool(vsa_plan* p, const void* q, const void* k, void* ws, void* stream) {
+  Range r("vsa_tile_pool");
+  if (!p || !q || !k || !ws) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!p->info.direct_attn) return fail(p, VSA_ERR_UNSUPPORTED);
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_pack++;
+  float *pq, *pk;
+  vsa::score_pooled_ptrs(p, ws, &pq, &pk);
+  if (vsa::launch_pool(p, q, k, pq, pk, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(p, VSA_ERR_CUDA);
+  return VSA_OK;
+}
+
+vsa_status vsa_sparse_attn_direct(vsa_plan* p, const void* q, const void* k, const void* v, const int32_t* idx,
+                                  const int32_t* k_per_head, void* o, float* lse, void* stream) {
+  Range r("vsa_sparse_attn_direct");
+  if (!p || !q || !k || !v || !idx || !o) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!p->info.direct_attn) return fail(p, VSA_ERR_UNSUPPORTED);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o) ||
+      (lse && !aligned16(lse)))
+    return fail(p, VSA_ERR_INVALID_ARG);
+  int32_t kk[VSA_MAX_HEADS];
+  if (!resolve_k(p, k_per_head, kk)) return fail(p, VSA_ERR_INVALID_ARG);
+  if (!on_plan_device(p)) return fail(p, VSA_ERR_INVALID_ARG);
+  p->stats.calls_attn++;
+  if (vsa::launch_attn_direct(p, q, k, v, idx, kk, o, lse, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(p, VSA_ERR_CUDA);
   return VSA_OK;
 }

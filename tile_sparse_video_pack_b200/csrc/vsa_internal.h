@@ -78,6 +78,14 @@ cudaError_t launch_pack_pool(const vsa_plan* p, const void* q, const void* k, co
                              void* qp8 = nullptr, void* kp8 = nullptr, float* q_scale = nullptr,
                              float* k_scale = nullptr);
 cudaError_t launch_unpack(const vsa_plan* p, const void* op, void* o, cudaStream_t s);
+// The score descriptors (pooled Q, K of every video tile) straight from the token-major Q, K.
+cudaError_t launch_pool(const vsa_plan* p, const void* q, const void* k, float* pooled_q, float* pooled_k,
+                        cudaStream_t s);
+// Attention with every tile loaded straight from the token-major Q, K, V and O written
+// token-major (batch 1, no reference tiles, video tiles partial only along t).
+bool direct_attn_supported(const vsa_plan* p);
+cudaError_t launch_attn_direct(vsa_plan* p, const void* q, const void* k, const void* v, const int32_t* idx,
+                               const int32_t* kk, void* o, float* lse, cudaStream_t s);
 cudaError_t launch_score(const vsa_plan* p, const void* qp, const void* kp, const float* proj_q,
                          const float* proj_k, float* scores, void* workspace, cudaStream_t s);
 int64_t score_workspace_bytes(const Geometry& g, int score_mode, int proj_dim);

@@ -9,14 +9,20 @@ class TileSparseAttention:
 
     ``proj_q`` / ``proj_k``: fp32 CUDA tensors -- the gate G ([d, d], the same
     tensor for both) for mean-pool scoring, or per-head TripPool projections
-    ([heads, 3d, p]).
+    ([heads, 3d, p]). ``direct=True`` (plans with ``info.direct_attn``) runs
+    pool -> score -> select -> sparse attention straight on the token-major
+    tensors and allocates no packed copies: less memory, about three times the
+    attention time (see vsa_sparse_attn_direct).
     """
 
-    def __init__(self, plan: Plan, proj_q, proj_k, with_lse: bool = False, device=None):
+    def __init__(self, plan: Plan, proj_q, proj_k, with_lse: bool = False, device=None, direct: bool = False):
         self.plan = plan
         self.proj_q = proj_q
         self.proj_k = proj_k
-        self.bufs = plan.allocate(device, with_lse=with_lse)
+        if direct and not plan.info.direct_attn:
+            raise ValueError("this plan's tiles are not boxes of the token-major tensors (info.direct_attn == 0)")
+        self.direct = direct
+        self.bufs = plan.allocate(device, with_lse=with_lse, packed=not direct)
 
     @classmethod
     def from_config(cls, cfg, sparsity, proj_q, proj_k, k_per_head=None, **kw):
@@ -27,8 +33,8 @@ class TileSparseAttention:
         import torch
         if out is None:
             out = torch.empty_like(q)
-        if self.plan.info.n_ref_tiles:       # R2VA budgets: the per-call path with the reference selection
-            return self.stages(q, k, v, out, stream)
+        if self.plan.info.n_ref_tiles or self.direct:
+            return self.stages(q, k, v, out, stream)   # R2VA budgets, or tiles straight from q, k, v
         self.plan.layer_forward(q, k, v, self.proj_q, self.proj_k, self.bufs, out, stream=stream)
         return out
 
@@ -38,6 +44,12 @@ class TileSparseAttention:
         """The calls one by one (same result as :meth:`forward`); with reference segments,
         the reference tiles are scored and selected and the attention uses that selection."""
         b, p = self.bufs, self.plan
+        if self.direct:
+            p.tile_pool(q, k, b["workspace"], stream)
+            p.tile_score_pooled(self.proj_q, self.proj_k, b["scores"], b["workspace"], stream)
+            p.topk_select(b["scores"], b["idx"], stream)
+            p.sparse_attn_direct(q, k, v, b["idx"], out, b["lse"], stream)
+            return out
         p.tile_pack_pool(q, k, v, b["qp"], b["kp"], b["vp"], b["workspace"], stream)
         p.tile_score_pooled(self.proj_q, self.proj_k, b["scores"], b["workspace"], stream)
         p.topk_select(b["scores"], b["idx"], stream)

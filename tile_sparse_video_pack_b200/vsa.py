@@ -28,7 +28,8 @@ EXPORTS = ("vsa_plan_create", "vsa_plan_destroy", "vsa_plan_query", "vsa_plan_ge
            "vsa_layer_forward", "vsa_plan_check", "vsa_status_string", "vsa_tile_score_static",
            "vsa_tile_pack_pool", "vsa_tile_score_pooled", "vsa_teacher_tiles", "vsa_index_overlap",
            "vsa_ref_score", "vsa_topk_select_ref", "vsa_sparse_attn_ref", "vsa_tile_pack_pool_fp8",
-           "vsa_sparse_attn_fp8", "vsa_plan_set_wait_limit", "vsa_plan_set_test_hold")
+           "vsa_sparse_attn_fp8", "vsa_plan_set_wait_limit", "vsa_plan_set_test_hold", "vsa_tile_pool",
+           "vsa_sparse_attn_direct")
 
 
 class VsaDesc(ctypes.Structure):
@@ -51,7 +52,7 @@ class VsaPlanInfo(ctypes.Structure):
         ("workspace_bytes", ctypes.c_int64), ("lse_elems", ctypes.c_int64), ("attn_work_items", ctypes.c_int64),
         ("n_ref_tiles", ctypes.c_int32), ("k_ref_max", ctypes.c_int32),
         ("ref_score_elems", ctypes.c_int64), ("ref_index_elems", ctypes.c_int64),
-        ("tile_scale_elems", ctypes.c_int64),
+        ("tile_scale_elems", ctypes.c_int64), ("direct_attn", ctypes.c_int32), ("reserved0", ctypes.c_int32),
     ]
 
 
@@ -107,6 +108,8 @@ def library() -> ctypes.CDLL:
         "vsa_sparse_attn_fp8": (I32, [P] * 11),
         "vsa_plan_set_wait_limit": (I32, [P, ctypes.c_uint64]),
         "vsa_plan_set_test_hold": (I32, [P, I32]),
+        "vsa_tile_pool": (I32, [P] * 5),
+        "vsa_sparse_attn_direct": (I32, [P] * 9),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -241,16 +244,20 @@ class Plan:
             "idx_ref": (d.batch, d.heads, i.ntv_max, i.k_ref_max),
         }
 
-    def allocate(self, device=None, with_lse=False):
-        """Device buffers for every intermediate of the layer (torch is only the allocator)."""
+    def allocate(self, device=None, with_lse=False, packed=True):
+        """Device buffers for every intermediate of the layer (torch is only the allocator).
+
+        packed=False leaves out the packed tiles (qp, kp, vp, op: None), which a plan with
+        info.direct_attn does not need."""
         import torch
         dev = torch.device("cuda") if device is None else torch.device(device)
         s = self.shapes()
+        pk = (lambda: torch.empty(s["packed"], dtype=torch.bfloat16, device=dev)) if packed else (lambda: None)
         bufs = {
-            "qp": torch.empty(s["packed"], dtype=torch.bfloat16, device=dev),
-            "kp": torch.empty(s["packed"], dtype=torch.bfloat16, device=dev),
-            "vp": torch.empty(s["packed"], dtype=torch.bfloat16, device=dev),
-            "op": torch.empty(s["packed"], dtype=torch.bfloat16, device=dev),
+            "qp": pk(),
+            "kp": pk(),
+            "vp": pk(),
+            "op": pk(),
             "scores": torch.empty(s["scores"], dtype=torch.float32, device=dev),
             "idx": torch.empty(s["idx"], dtype=torch.int32, device=dev),
             "workspace": torch.empty(s["workspace"], dtype=torch.uint8, device=dev),
@@ -280,6 +287,27 @@ class Plan:
             _ptr(scores, torch.float32, "scores", self.info.score_elems),
             _ptr(workspace, torch.uint8, "workspace", self.info.workspace_bytes), _stream(stream)),
             "vsa_tile_score")
+
+    def tile_pool(self, q, k, workspace, stream=None):
+        """Pooling of the score stage straight from token-major q, k (plans with info.direct_attn)."""
+        import torch
+        n_tok = self.desc.batch * self.info.n_tokens * self.desc.heads * self.desc.head_dim
+        bf = torch.bfloat16
+        _check(library().vsa_tile_pool(
+            self._h, _ptr(q, bf, "q", n_tok), _ptr(k, bf, "k", n_tok),
+            _ptr(workspace, torch.uint8, "workspace", self.info.workspace_bytes), _stream(stream)),
+            "vsa_tile_pool")
+
+    def sparse_attn_direct(self, q, k, v, idx, o, lse=None, stream=None, k_per_head=None):
+        """Attention from token-major q, k, v into token-major o (plans with info.direct_attn)."""
+        import torch
+        n_tok = self.desc.batch * self.info.n_tokens * self.desc.heads * self.desc.head_dim
+        bf = torch.bfloat16
+        _check(library().vsa_sparse_attn_direct(
+            self._h, _ptr(q, bf, "q", n_tok), _ptr(k, bf, "k", n_tok), _ptr(v, bf, "v", n_tok),
+            _ptr(idx, torch.int32, "idx", self.info.index_elems), _karray(k_per_head, self.desc.heads),
+            _ptr(o, bf, "o", n_tok), _ptr(lse, torch.float32, "lse", self.info.lse_elems), _stream(stream)),
+            "vsa_sparse_attn_direct")
 
     def tile_pack_pool(self, q, k, v, qp, kp, vp, workspace, stream=None):
         """tile_pack fused with the pooling of tile_score; follow with tile_score_pooled."""
@@ -420,16 +448,16 @@ class Plan:
             _ptr(o, torch.bfloat16, "o", n_tok), _stream(stream)), "vsa_tile_unpack")
 
     def layer_forward(self, q, k, v, proj_q, proj_k, bufs, o, stream=None):
-        """All five calls in one C-ABI call (vsa_layer_forward)."""
+        """The layer's calls in one C-ABI call (vsa_layer_forward; the direct path when info.direct_attn)."""
         import torch
         pe, bf = self.info.packed_elems, torch.bfloat16
         n_tok = self.desc.batch * self.info.n_tokens * self.desc.heads * self.desc.head_dim
         _check(library().vsa_layer_forward(
             self._h, _ptr(q, bf, "q", n_tok), _ptr(k, bf, "k", n_tok), _ptr(v, bf, "v", n_tok),
             _ptr(proj_q, torch.float32, "proj_q"), _ptr(proj_k, torch.float32, "proj_k"),
-            _ptr(bufs["qp"], bf, "qp", pe), _ptr(bufs["kp"], bf, "kp", pe), _ptr(bufs["vp"], bf, "vp", pe),
+            _ptr(bufs.get("qp"), bf, "qp", pe), _ptr(bufs.get("kp"), bf, "kp", pe), _ptr(bufs.get("vp"), bf, "vp", pe),
             _ptr(bufs["scores"], torch.float32, "scores", self.info.score_elems),
-            _ptr(bufs["idx"], torch.int32, "idx", self.info.index_elems), _ptr(bufs["op"], bf, "op", pe),
+            _ptr(bufs["idx"], torch.int32, "idx", self.info.index_elems), _ptr(bufs.get("op"), bf, "op", pe),
             _ptr(bufs.get("lse"), torch.float32, "lse", self.info.lse_elems),
             _ptr(bufs["workspace"], torch.uint8, "workspace", self.info.workspace_bytes),
             _ptr(o, bf, "o", n_tok), _stream(stream)), "vsa_layer_forward")

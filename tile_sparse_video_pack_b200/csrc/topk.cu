@@ -166,15 +166,25 @@ __global__ void __launch_bounds__(kMaxWarps * 32) topk_kernel(Geometry g, const 
         if (c0 + u < chunks) {
           const float x[4] = {f[u].x + 0.0f, f[u].y + 0.0f, f[u].z + 0.0f, f[u].w + 0.0f};
           uint32_t kk[4];
+          if (j + 3 < n) {                          // four real scores: no per-key checks
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const bool in = j + t < n;
-            nan |= in && x[t] != x[t];
-            if (in) {
+            for (int t = 0; t < 4; ++t) {
+              nan |= x[t] != x[t];
               lo = fminf(lo, x[t]);
               hi = fmaxf(hi, x[t]);
+              kk[t] = order_key(x[t]);
             }
-            kk[t] = in ? order_key(x[t]) : 0u;
+          } else {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const bool in = j + t < n;
+              nan |= in && x[t] != x[t];
+              if (in) {
+                lo = fminf(lo, x[t]);
+                hi = fmaxf(hi, x[t]);
+              }
+              kk[t] = in ? order_key(x[t]) : 0u;
+            }
           }
           *reinterpret_cast<uint4*>(keys + j) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
         }
@@ -206,12 +216,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32) topk_kernel(Geometry g, const 
         uint32_t code = 0;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const int b = value_bin(kk[t], lo, inv);
-          if (j + t < n) atomicAdd(&hist[b], 1);
+          // padding keys (0, past n) decode to NaN, whose bin is clamped to 0; they are taken off below
+          const int b = max(value_bin(kk[t], lo, inv), 0);
+          atomicAdd(&hist[b], 1);
           code |= uint32_t(b) << (8 * t);
         }
         reinterpret_cast<uint32_t*>(bins)[c * 32 + lane] = code;
       }
+      __syncwarp();
+      if (lane == 0) hist[0] -= chunks * 128 - n;
       __syncwarp();
       int above;
       const int bin = find_bin(hist, kBins, k, lane, &above);
@@ -284,8 +297,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32) topk_kernel(Geometry g, const 
       uint32_t gt4 = 0, eq4 = 0;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        gt4 |= (j + t < n && kk[t] > thr) ? (1u << t) : 0u;
-        eq4 |= (j + t < n && kk[t] == thr) ? (1u << t) : 0u;
+        // padding keys are 0, below every real key, so neither above nor equal to thr
+        gt4 |= kk[t] > thr ? (1u << t) : 0u;
+        eq4 |= kk[t] == thr ? (1u << t) : 0u;
       }
       uint32_t take4 = gt4;
       if (__any_sync(0xffffffffu, eq4 != 0)) {

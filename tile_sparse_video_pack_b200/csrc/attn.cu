@@ -37,7 +37,11 @@
 //
 // TMEM holds the two S buffers and the two partial outputs; shared memory the
 // Q pair and the K and V stages, in the canonical 128-byte-swizzled UMMA
-// layouts that TMA SWIZZLE_128B writes (Q and K K-major, V MN-major).
+// layouts that TMA SWIZZLE_128B writes (Q and K K-major, V MN-major). The
+// tiles come from the packed tensors as 2-D boxes, or (DIRECT) straight from
+// the token-major tensors as 3-D / 5-D boxes with O written token-major: the
+// same shared-memory images and the same results, but scattered rows that
+// TMA fetches several times more slowly, so that instance is an opt-in.
 // Every wait is bounded (about two seconds); on expiry the CTA latches a
 // timeout in the plan's error word, drains its copies and MMAs, frees TMEM and
 // returns.

@@ -28,6 +28,7 @@ namespace {
 
 constexpr int kBins = 256;        // value bins of the first pass (a byte per key)
 constexpr int kSmall = 64;        // candidates resolved by counting
+static_assert(kSmall < kBins - 1, "the candidates and their slot counter share the histogram's words");
 constexpr int kMaxWarps = 4;      // rows (warps) per CTA
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -234,21 +235,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32) topk_kernel(Geometry g, const 
       if (cnt <= kSmall) {
         // the bin's candidates (any order), then the one whose rank among them brackets need
         uint32_t* cand = reinterpret_cast<uint32_t*>(hist);
-        int base = 0;
+        int* n_cand = hist + (kBins - 1);   // a slot counter past the (at most kSmall) candidates
+        if (lane == 0) *n_cand = 0;
+        __syncwarp();
         for (int c = 0; c < chunks; ++c) {
           const int j = 4 * (c * 32 + lane);
           const uint32_t code = reinterpret_cast<const uint32_t*>(bins)[c * 32 + lane];
-          int m = 0;
 #pragma unroll
-          for (int t = 0; t < 4; ++t) m += (j + t < n && int((code >> (8 * t)) & 255u) == bin) ? 1 : 0;
-          int total;
-          int pos = base + warp_excl_scan(m, lane, &total);
-          if (m) {
-#pragma unroll
-            for (int t = 0; t < 4; ++t)
-              if (j + t < n && int((code >> (8 * t)) & 255u) == bin) cand[pos++] = keys[j + t];
-          }
-          base += total;
+          for (int t = 0; t < 4; ++t)
+            if (int((code >> (8 * t)) & 255u) == bin && j + t < n) cand[atomicAdd(n_cand, 1)] = keys[j + t];
         }
         __syncwarp();
         bool found = false;
@@ -315,8 +310,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32) topk_kernel(Geometry g, const 
           }
         base_eq += n_eq;
       }
-      int n_take;
-      int pos = base_out + warp_excl_scan(__popc(take4), lane, &n_take);
+      // output slots: this lane's count (0..4) as three bit planes of ballots, no shuffle chain
+      const uint32_t nt = __popc(take4);
+      const uint32_t b0 = __ballot_sync(0xffffffffu, nt & 1u), b1 = __ballot_sync(0xffffffffu, nt & 2u),
+                     b2 = __ballot_sync(0xffffffffu, nt & 4u);
+      const uint32_t below = (1u << lane) - 1u;
+      int pos = base_out + __popc(b0 & below) + 2 * __popc(b1 & below) + 4 * __popc(b2 & below);
+      const int n_take = __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
 #pragma unroll
       for (int t = 0; t < 4; ++t)
         if (take4 & (1u << t)) out[pos++] = j + t;

@@ -48,8 +48,8 @@ def metric_for(cfg):
         return METRIC
     return (f"ms per attention layer, {cfg.name} workload ({cfg.n_video_tokens} video tokens), "
             f"sparsity {cfg.sparsity[0]} (other levels in sweep); effective TFLOP/s")
-KERNELS_PER_STEP = 7  # pack + pool 1, score 3 (2 projections, scores), select 1, attention 1, unpack 1
-KERNELS_PER_STEP_DIRECT = 6  # pool 1, score 3, select 1, attention straight from q, k, v into o 1
+KERNELS_PER_STEP = 6  # pack + pool 1, score 2 (both projections in one launch, scores), select 1, attention 1, unpack 1
+KERNELS_PER_STEP_DIRECT = 5  # pool 1, score 2, select 1, attention straight from q, k, v into o 1
 
 
 def parse():

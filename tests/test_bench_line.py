@@ -48,7 +48,7 @@ def test_line_has_every_key_and_reproduces_the_recorded_run():
     json.dumps(line)
     assert line["metric"] == bench.METRIC and line["unit"] == "ms" and line["higher_is_better"] is False
     assert line["value"] == pytest.approx(sum(STAGES.values()), abs=1e-3)
-    assert line["gpu_launches"] == 7 * 20
+    assert line["gpu_launches"] == 6 * 20
     r = line["roofline"]
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["algorithmic_flops_per_launch"] == O.attention_flops(cfg, _ks(cfg, 0.75))
@@ -73,7 +73,7 @@ def test_fp8_line_uses_the_mixed_peak_and_no_traffic():
 def test_r2va_line_counts_the_reference_launches():
     cfg = get_config("r2va")
     line, _ = _line(_args(sparsity=cfg.sparsity[0], config="r2va"), cfg)
-    assert line["gpu_launches"] == (7 + 4) * 20
+    assert line["gpu_launches"] == (6 + 4) * 20
     assert "reference segments" in line["config"]["workload"]
 
 

@@ -172,66 +172,101 @@ __global__ void __launch_bounds__(256) pool_ref_kernel(Geometry g, const uint16_
   }
 }
 
-// The projections: C[z] = alpha * A[z] * B[z] (fp32 SIMT); z = b * heads + h; 128 x 128 tiles, 8 x 8
-// per thread. A: [M][K] row-major (lda). B: [K][N] row-major (ldb).
-// M = m_fixed if > 0 else ntv[h]; N = n_fixed if > 0 else ntv[h]. K % 8 == 0, rows 16-byte aligned.
-__global__ void __launch_bounds__(256) sgemm_kernel(Geometry g, const float* __restrict__ A, int64_t sA, int lda,
-                                                    const float* __restrict__ Bm, int64_t sBz, int64_t sBh,
-                                                    int ldb, float* __restrict__ C, int64_t sC, int ldc, int K,
-                                                    int n_fixed, float alpha, int m_fixed = 0) {
-  __shared__ __align__(16) float As[8][128];
-  __shared__ __align__(16) float Bs[8][128];
-  const int z = blockIdx.z;
+// The projections: C[z] = alpha * A[z] * B[h] (fp32 SIMT), for one or two problems per launch (the query
+// and the key side share the weights' layout): blockIdx.z = problem * Z + z, z = b * heads + h.
+// A: [M][K] row-major (lda, stride sA per z). B: [K][N] row-major (ldb, stride sBh per head; 0 when one
+// matrix serves every head). M = m_fixed if > 0 else ntv[h]; N = n_fixed. K % 8 == 0, rows 16-byte aligned.
+// Output tiles of 32 rows x 128 columns, 64 threads of 8 x 8 each: the problems are a few thousand rows of
+// K = 128 or 384, so small tiles keep every SM busy to the end (128-row tiles left one wave of 336 CTAs
+// with a nearly empty second). Shared memory is double buffered: the next k slice of B streams in by
+// cp.async and the next slice of A is held in registers while this one is used, one barrier per slice.
+// Each output is one fp32 FMA chain over k in ascending order.
+struct ProjProblem {
+  const float* A;
+  const float* B;
+  float* C;
+};
+constexpr int kProjRows = 32;
+constexpr int kProjThreads = 64;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(tc::smem_u32(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kProjThreads, 8) sgemm_kernel(Geometry g, ProjProblem p0, ProjProblem p1, int Z,
+                                                                int64_t sA, int lda, int64_t sBh, int ldb,
+                                                                int64_t sC, int ldc, int K, int N, float alpha,
+                                                                int m_fixed) {
+  constexpr int BM = kProjRows, NT = kProjThreads, BQ = 8 * 128 / 4 / NT;   // B chunks per thread per slice
+  __shared__ __align__(16) float As[2][8][BM];
+  __shared__ __align__(16) float Bs[2][8][128];
+  const int zz = blockIdx.z;
+  const ProjProblem pr = zz < Z ? p0 : p1;
+  const int z = zz < Z ? zz : zz - Z;
   const int h = z % g.Hh;
   const int M = m_fixed > 0 ? m_fixed : g.ntv[h];
-  const int N = n_fixed > 0 ? n_fixed : g.ntv[h];
-  const int m0 = blockIdx.y * 128, n0 = blockIdx.x * 128;
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * 128;
   if (m0 >= M || n0 >= N) return;
-  A += z * sA;
-  Bm += z * sBz + h * sBh;
-  C += z * sC;
+  const float* A = pr.A + z * sA;
+  const float* Bm = pr.B + h * sBh;
+  float* C = pr.C + z * sC;
   const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
+  const int tx = tid & 15, ty = tid >> 4;   // 16 column groups x 4 row groups
   float acc[8][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
-  for (int k0 = 0; k0 < K; k0 += 8) {
-    {  // A tile: 128 rows x 8 k, one float4 per thread, stored k-major
-      const int r = tid >> 1, kq = (tid & 1) * 4;
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (m0 + r < M) a = *reinterpret_cast<const float4*>(A + int64_t(m0 + r) * lda + k0 + kq);
-      As[kq + 0][r] = a.x;
-      As[kq + 1][r] = a.y;
-      As[kq + 2][r] = a.z;
-      As[kq + 3][r] = a.w;
+  // one k slice: A 32 rows x 8 k (a float4 per thread, stored k-major), B 8 k x 128 n (BQ 16-byte chunks
+  // per thread; columns past N are zero-filled)
+  const int ar = tid >> 1, akq = (tid & 1) * 4;
+  const bool a_in = m0 + ar < M;
+  float4 ra;
+  auto fetch_a = [&](int k0) {
+    ra = a_in ? *reinterpret_cast<const float4*>(A + int64_t(m0 + ar) * lda + k0 + akq)
+              : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  auto fetch_b = [&](int k0, int buf) {
+#pragma unroll
+    for (int q = 0; q < BQ; ++q) {
+      const int e = tid + q * NT, kr = e >> 5, c = (e & 31) * 4;
+      const bool in = n0 + c < N;
+      cp_async16(&Bs[buf][kr][c], in ? Bm + int64_t(k0 + kr) * ldb + n0 + c : Bm, in);
     }
-    {  // B rows are k: 8 k x 128 n
-      const int kr = tid >> 5, c = (tid & 31) * 4;
-      float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (n0 + c < N) b = *reinterpret_cast<const float4*>(Bm + int64_t(k0 + kr) * ldb + n0 + c);
-      *reinterpret_cast<float4*>(&Bs[kr][c]) = b;
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+  };
+  fetch_b(0, 0);
+  fetch_a(0);
+  for (int k0 = 0, buf = 0; k0 < K; k0 += 8, buf ^= 1) {
+    As[buf][akq + 0][ar] = ra.x;
+    As[buf][akq + 1][ar] = ra.y;
+    As[buf][akq + 2][ar] = ra.z;
+    As[buf][akq + 3][ar] = ra.w;
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+    __syncthreads();   // slice k0 complete in buf; every thread is past its reads of buf ^ 1
+    if (k0 + 8 < K) {
+      fetch_b(k0 + 8, buf ^ 1);
+      fetch_a(k0 + 8);
     }
-    __syncthreads();
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       float a[8], b[8];
-      *reinterpret_cast<float4*>(a) = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-      *reinterpret_cast<float4*>(a + 4) = *reinterpret_cast<const float4*>(&As[kk][64 + ty * 4]);
-      *reinterpret_cast<float4*>(b) = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-      *reinterpret_cast<float4*>(b + 4) = *reinterpret_cast<const float4*>(&Bs[kk][64 + tx * 4]);
+      *reinterpret_cast<float4*>(a) = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      *reinterpret_cast<float4*>(a + 4) = *reinterpret_cast<const float4*>(&As[buf][kk][BM / 2 + ty * 4]);
+      *reinterpret_cast<float4*>(b) = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+      *reinterpret_cast<float4*>(b + 4) = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
     }
-    __syncthreads();
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+    const int m = m0 + (i < 4 ? ty * 4 + i : BM / 2 + ty * 4 + (i - 4));
     if (m >= M) continue;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -503,11 +538,10 @@ cudaError_t launch_project_score(const vsa_plan* pl, const float* proj_q, const 
   // projection: [ntv, kd] x [kd, p]; the gate is shared by all heads, TripPool weights are per head
   const int Z = g.B * g.Hh;
   const int64_t sW = trip ? int64_t(L.kd) * p : 0;
-  dim3 gp((p + 127) / 128, (g.ntv_max + 127) / 128, Z);
-  sgemm_kernel<<<gp, 256, 0, s>>>(g, pq, int64_t(g.ntv_max) * L.kd, L.kd, proj_q, 0, sW, p, hq,
-                                         int64_t(g.ntv_max) * p, p, L.kd, p, 1.0f);
-  sgemm_kernel<<<gp, 256, 0, s>>>(g, pk, int64_t(g.ntv_max) * L.kd, L.kd, proj_k, 0, sW, p, hk,
-                                         int64_t(g.ntv_max) * p, p, L.kd, p, 1.0f);
+  dim3 gp((p + 127) / 128, (g.ntv_max + kProjRows - 1) / kProjRows, 2 * Z);
+  sgemm_kernel<<<gp, kProjThreads, 0, s>>>(g, ProjProblem{pq, proj_q, hq}, ProjProblem{pk, proj_k, hk}, Z,
+                                           int64_t(g.ntv_max) * L.kd, L.kd, sW, p, int64_t(g.ntv_max) * p, p,
+                                           L.kd, p, 1.0f, 0);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -565,9 +599,10 @@ cudaError_t launch_ref_score(const vsa_plan* pl, const void* kp, const float* pr
   if (e != cudaSuccess) return e;
   const int Z = g.B * g.Hh;
   const int64_t sW = trip ? int64_t(L.kd) * p : 0;
-  dim3 gp((p + 127) / 128, (g.n_ref + 127) / 128, Z);
-  sgemm_kernel<<<gp, 256, 0, s>>>(g, pr, int64_t(g.n_ref) * L.kd, L.kd, proj_k, 0, sW, p, hr,
-                                         int64_t(g.n_ref) * p, p, L.kd, p, 1.0f, g.n_ref);
+  dim3 gp((p + 127) / 128, (g.n_ref + kProjRows - 1) / kProjRows, Z);
+  const ProjProblem ref{pr, proj_k, hr};
+  sgemm_kernel<<<gp, kProjThreads, 0, s>>>(g, ref, ref, Z, int64_t(g.n_ref) * L.kd, L.kd, sW, p,
+                                           int64_t(g.n_ref) * p, p, L.kd, p, 1.0f, g.n_ref);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_score_tc(pl, hq, g.ntv_max, hr, g.n_ref, p, scores_ref, int64_t(g.ntv_max) * g.n_ref, g.n_ref, 0,

@@ -174,7 +174,7 @@ def tripool(x: np.ndarray) -> np.ndarray:
     """TripPool descriptor of a tile: avg, max and min over its tokens, concatenated (3d).
 
     BSAI VedaSparse README, "Core Technology" (Avg+Max+Min), "Implementation"
-    (``_tripool``, the paper's eq. 5).
+    (``_tripool``, which the README ties to its eq. 5).
     """
     return np.concatenate([mean_pool(x), x.max(axis=0), x.min(axis=0)])
 

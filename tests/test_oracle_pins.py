@@ -297,7 +297,7 @@ def test_tripool_projection_orientation():
     pin_tripool_projection_orientation()
 
 
-def test_permutation_closed_form():
+def pin_permutation_closed_form():
     cfg = ragged_config()
     inp, q, k, v = inputs_f64(cfg)
     packed, counts = O.pack(q, cfg)
@@ -313,7 +313,11 @@ def test_permutation_closed_form():
     assert np.array_equal(O.unpack(packed, cfg), q)
 
 
-def test_custom_tiling_golden_partitions_grid():
+def test_permutation_closed_form():
+    pin_permutation_closed_form()
+
+
+def pin_custom_tiling_golden_partitions_grid():
     with open(os.path.join(GOLDEN, "custom_tiling.txt")) as f:
         line = [x for x in f.read().splitlines() if x and not x.startswith("#")][0]
     shapes = [tuple(int(a) for a in part.split(",")) for part in line.split(";")]
@@ -327,7 +331,11 @@ def test_custom_tiling_golden_partitions_grid():
         assert np.array_equal(np.sort(allt), np.arange(T * H * W))
 
 
-def test_head_aware_tile_counts():
+def test_custom_tiling_golden_partitions_grid():
+    pin_custom_tiling_golden_partitions_grid()
+
+
+def pin_head_aware_tile_counts():
     # (16,2,2) on 28 frames: 2 x 24 x 40 tiles, the second temporal row holds 12 frames
     tiles = O.video_tiles(28, 48, 80, (16, 2, 2), 0)
     sizes = np.array([len(t) for t in tiles])
@@ -336,7 +344,11 @@ def test_head_aware_tile_counts():
     assert [len(t) for t in O.prefix_tiles((100, 30))] == [64, 36, 30]
 
 
-def test_k_from_sparsity():
+def test_head_aware_tile_counts():
+    pin_head_aware_tile_counts()
+
+
+def pin_k_from_sparsity():
     with open(os.path.join(GOLDEN, "sparsity_levels.txt")) as f:
         levels = [float(x.split()[0]) for x in f.read().splitlines() if x and not x.startswith("#")]
     for s in levels:
@@ -349,6 +361,10 @@ def test_k_from_sparsity():
     assert O.k_from_sparsity(0.0, 1680) == 1680
     assert O.k_from_sparsity(1.0, 1680) == 1
     assert [O.k_from_sparsity(s, 3600) for s in (0, .5, .75, .9, .95)] == [3600, 1800, 900, 360, 180]
+
+
+def test_k_from_sparsity():
+    pin_k_from_sparsity()
 
 
 def test_flop_count_matches_run():
@@ -540,7 +556,7 @@ def test_teacher_is_a_max_of_probabilities():
     assert np.all(T > 0) and np.all(T <= 1)   # softmax weights
 
 
-def test_recall_identities():
+def pin_recall_identities():
     rng = np.random.default_rng(5)
     T = rng.random((6, 12))
     for i in range(6):
@@ -550,6 +566,10 @@ def test_recall_identities():
         assert O.tile_recall(rest, T[i], 4) == 0.0
         assert O.tile_recall(np.arange(12), T[i], 12) == 1.0
         assert O.tile_recall(np.sort(np.r_[best[:2], rest[:2]]), T[i], 4) == 0.5
+
+
+def test_recall_identities():
+    pin_recall_identities()
 
 
 def test_mutation_teacher_mean_over_rows(monkeypatch):
@@ -702,7 +722,7 @@ def test_mutation_r2va_drops_reference_tiles(monkeypatch):
 
 # ------------------------------------------- fp8 (e4m3) Q K^T per-tile scales ---
 
-def test_e4m3_round_matches_torch_float8():
+def pin_e4m3_round_matches_torch_float8():
     """Against torch's float8_e4m3fn conversion (round to nearest even), which is a
     library routine independent of the oracle: every finite code, every midpoint between
     neighbouring codes, and random values within the finite range."""
@@ -716,6 +736,10 @@ def test_e4m3_round_matches_torch_float8():
     assert np.array_equal(O.e4m3_round(xs), want)
     assert np.array_equal(O.e4m3_round(finite), finite)          # idempotent on the codes
     assert O.e4m3_round(np.array([500.0, -1e6]))[0] == 448.0      # saturates (torch would give NaN)
+
+
+def test_e4m3_round_matches_torch_float8():
+    pin_e4m3_round_matches_torch_float8()
 
 
 def test_tile_quantisation_scale_and_range():
@@ -865,3 +889,123 @@ def test_bench_flop_count_is_the_oracle_count(name):
     cfg = get_config(name)
     ks = [O.k_from_sparsity(cfg.sparsity[-1], n_video_tiles(cfg, h)) for h in range(cfg.heads)]
     assert bench.attention_flops(cfg, ks) == O.attention_flops(cfg, ks)
+
+
+# ------------------------------- planted mistakes in tiling, k, e4m3, recall ---
+
+def _video_tiles_with(order="thw", inner="thw", edge="ceil"):
+    """The oracle's video tiling with one rule changed: the tile order (``order``), the token
+    order inside a tile (``inner``), or edge tiles dropped instead of kept partial (``edge``)."""
+    def tiles(T, H, W, shape, n_prefix):
+        pt, ph, pw = shape
+        cnt = (lambda a, b: -(-a // b)) if edge == "ceil" else (lambda a, b: a // b)
+        idx = [(ti, hi, wi) for ti in range(cnt(T, pt)) for hi in range(cnt(H, ph)) for wi in range(cnt(W, pw))]
+        if order == "wht":
+            idx.sort(key=lambda c: (c[2], c[1], c[0]))
+        out = []
+        for ti, hi, wi in idx:
+            t = np.arange(ti * pt, min(T, (ti + 1) * pt))
+            y = np.arange(hi * ph, min(H, (hi + 1) * ph))
+            x = np.arange(wi * pw, min(W, (wi + 1) * pw))
+            tok = (t[:, None, None] * H + y[None, :, None]) * W + x[None, None, :]
+            if inner == "wht":
+                tok = tok.transpose(2, 1, 0)
+            out.append(n_prefix + tok.ravel().astype(np.int64))
+        return out
+    return tiles
+
+
+def test_planted_tiling_reference_is_the_oracle():
+    # the helper with no rule changed is the oracle's tiling, so each mutation below changes one rule only
+    for shape in ((4, 4, 4), (16, 2, 2), (2, 4, 8), (8, 4, 2)):
+        want = O.video_tiles(6, 8, 8, shape, 130)
+        got = _video_tiles_with()(6, 8, 8, shape, 130)
+        assert len(got) == len(want) and all(np.array_equal(a, b) for a, b in zip(got, want))
+
+
+def test_mutation_video_tiles_w_major(monkeypatch):
+    monkeypatch.setattr(O, "video_tiles", _video_tiles_with(order="wht"))
+    _expect_pin_failure(pin_permutation_closed_form)
+
+
+def test_mutation_tokens_w_major_inside_tile(monkeypatch):
+    monkeypatch.setattr(O, "video_tiles", _video_tiles_with(inner="wht"))
+    _expect_pin_failure(pin_permutation_closed_form)
+
+
+def test_mutation_edge_tiles_dropped(monkeypatch):
+    monkeypatch.setattr(O, "video_tiles", _video_tiles_with(edge="floor"))
+    _expect_pin_failure(pin_head_aware_tile_counts)
+    _expect_pin_failure(pin_custom_tiling_golden_partitions_grid)
+
+
+def test_mutation_prefix_tiles_cross_segments(monkeypatch):
+    def bad(segments):                      # 64-token chunks of the whole prefix, segments mixed
+        n = int(sum(segments))
+        return [np.arange(s0, min(n, s0 + O.TILE), dtype=np.int64) for s0 in range(0, n, O.TILE)]
+    monkeypatch.setattr(O, "prefix_tiles", bad)
+    _expect_pin_failure(pin_head_aware_tile_counts)
+
+
+def _pack_with(padding="zero", one_tiling=False):
+    def pack(x, cfg):
+        B, N, Hh, d = x.shape
+        tilings = [O.head_tiling(cfg, 0 if one_tiling else h) for h in range(Hh)]
+        nt = max(len(t.all) for t in tilings)
+        out = np.zeros((B, Hh, nt, O.TILE, d), dtype=x.dtype)
+        counts = np.zeros((Hh, nt), dtype=np.int32)
+        for h, til in enumerate(tilings):
+            for n, tok in enumerate(til.all):
+                out[:, h, n, :len(tok)] = x[:, tok, h]
+                if padding == "repeat":
+                    out[:, h, n, len(tok):] = x[:, tok[-1], h][:, None]
+                counts[h, n] = len(tok)
+        return out, counts
+    return pack
+
+
+def test_mutation_pack_padding_repeats_last_token(monkeypatch):
+    monkeypatch.setattr(O, "pack", _pack_with(padding="repeat"))
+    _expect_pin_failure(pin_permutation_closed_form)
+
+
+def test_mutation_pack_first_heads_tiling_for_every_head(monkeypatch):
+    monkeypatch.setattr(O, "pack", _pack_with(one_tiling=True))
+    _expect_pin_failure(pin_permutation_closed_form)
+
+
+def test_mutation_k_ceil_of_kept_share(monkeypatch):
+    monkeypatch.setattr(O, "k_from_sparsity", lambda s, n: max(1, min(n, math.ceil((1.0 - s) * n))))
+    _expect_pin_failure(pin_k_from_sparsity)
+
+
+def test_mutation_k_not_clamped(monkeypatch):
+    monkeypatch.setattr(O, "k_from_sparsity", lambda s, n: n - math.floor(s * n + 0.5))
+    _expect_pin_failure(pin_k_from_sparsity)
+
+
+def test_mutation_e4m3_ties_away_from_zero(monkeypatch):
+    def bad(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.abs(x)
+        step = 2.0 ** (np.floor(np.log2(np.maximum(a, 2.0 ** -6))) - 3)
+        return np.sign(x) * np.minimum(np.floor(a / step + 0.5) * step, O.E4M3_MAX)
+    monkeypatch.setattr(O, "e4m3_round", bad)
+    _expect_pin_failure(pin_e4m3_round_matches_torch_float8)
+
+
+def test_mutation_e4m3_without_subnormals(monkeypatch):
+    def bad(x):                             # every magnitude gets 3 mantissa bits, however small
+        x = np.asarray(x, dtype=np.float64)
+        a = np.abs(x)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            step = 2.0 ** (np.floor(np.log2(a)) - 3)
+            q = np.where(a > 0, np.round(a / step) * step, 0.0)
+        return np.sign(x) * np.minimum(q, O.E4M3_MAX)
+    monkeypatch.setattr(O, "e4m3_round", bad)
+    _expect_pin_failure(pin_e4m3_round_matches_torch_float8)
+
+
+def test_mutation_recall_against_the_teachers_weakest_tiles(monkeypatch):
+    monkeypatch.setattr(O, "tile_recall", lambda kept, t, k: len(np.intersect1d(kept, np.argsort(t)[:k])) / k)
+    _expect_pin_failure(pin_recall_identities)

@@ -213,7 +213,7 @@ def test_exhaustive_selection_tiny():
             assert np.array_equal(res.kept[h][i], O.exhaustive_topk(res.scores[h][i], kk[h]))
 
 
-def test_exhaustive_with_ties():
+def pin_exhaustive_with_ties():
     rng = np.random.default_rng(5)
     for _ in range(200):
         row = rng.integers(0, 3, size=7).astype(np.float64)
@@ -221,10 +221,11 @@ def test_exhaustive_with_ties():
         assert np.array_equal(O.topk_row(row, kk), O.exhaustive_topk(row, kk))
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged", "ragged_tp"])
-def test_tile_loop_equals_explicit_mask(name):
-    cfg = {"tiny": get_config("tiny"), "ragged": ragged_config(batch=1),
-           "ragged_tp": ragged_tripool_config()}[name]
+def test_exhaustive_with_ties():
+    pin_exhaustive_with_ties()
+
+
+def pin_tile_loop_equals_explicit_mask(cfg):
     inp, q, k, v = inputs_f64(cfg)
     kk = k_list(cfg, 0.5)
     res = O.run_layer(cfg, q, k, v, kk, gate=inp.gate, w_q=inp.w_q, w_k=inp.w_k)
@@ -240,6 +241,12 @@ def test_tile_loop_equals_explicit_mask(name):
         ref = O.masked_dense_attention(q[0, :, h], k[0, :, h], v[0, :, h], allowed,
                                        1.0 / math.sqrt(cfg.head_dim))
         assert np.max(np.abs(ref - res.out[0, :, h])) <= 1e-12
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "ragged_tp"])
+def test_tile_loop_equals_explicit_mask(name):
+    pin_tile_loop_equals_explicit_mask({"tiny": get_config("tiny"), "ragged": ragged_config(batch=1),
+                                        "ragged_tp": ragged_tripool_config()}[name])
 
 
 def test_invariants_ragged():
@@ -1009,3 +1016,19 @@ def test_mutation_e4m3_without_subnormals(monkeypatch):
 def test_mutation_recall_against_the_teachers_weakest_tiles(monkeypatch):
     monkeypatch.setattr(O, "tile_recall", lambda kept, t, k: len(np.intersect1d(kept, np.argsort(t)[:k])) / k)
     _expect_pin_failure(pin_recall_identities)
+
+
+def test_mutation_prefix_rows_see_only_the_prefix(monkeypatch):
+    good = O.query_key_tokens
+
+    def bad(til, tile_id, kept_video, ref=None, kept_ref=None):
+        if tile_id < til.n_prefix:          # conditioning rows read as attending to the conditioning only
+            return np.concatenate(til.prefix)
+        return good(til, tile_id, kept_video, ref, kept_ref)
+    monkeypatch.setattr(O, "query_key_tokens", bad)
+    _expect_pin_failure(pin_tile_loop_equals_explicit_mask, ragged_config(batch=1))
+
+
+def test_mutation_kept_tiles_in_score_order(monkeypatch):
+    monkeypatch.setattr(O, "topk_row", lambda row, k: np.lexsort((np.arange(row.size), -row))[:k])
+    _expect_pin_failure(pin_exhaustive_with_ties)

@@ -1032,3 +1032,50 @@ def test_mutation_prefix_rows_see_only_the_prefix(monkeypatch):
 def test_mutation_kept_tiles_in_score_order(monkeypatch):
     monkeypatch.setattr(O, "topk_row", lambda row, k: np.lexsort((np.arange(row.size), -row))[:k])
     _expect_pin_failure(pin_exhaustive_with_ties)
+
+
+# ------------------------------------------------ the brute-force references ---
+
+def pin_dense_attention_matches_torch():
+    """The N x N references against torch's scaled_dot_product_attention in fp64 on the CPU (a
+    library routine that shares nothing with the oracle), with and without a boolean mask."""
+    import torch
+    import torch.nn.functional as F
+    rng = np.random.default_rng(8)
+    q, k, v = (rng.standard_normal((2, 50, 3, 16)) for _ in range(3))
+    scale = 0.3
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).permute(0, 2, 1, 3)   # [B, heads, N, d]
+    want = F.scaled_dot_product_attention(t(q), t(k), t(v), scale=scale).permute(0, 2, 1, 3).numpy()
+    assert np.max(np.abs(O.dense_attention(q, k, v, scale) - want)) <= 1e-12
+    allowed = rng.random((50, 50)) < 0.3
+    allowed[np.arange(50), rng.integers(0, 50, 50)] = True          # every row keeps a key
+    qh, kh, vh = (torch.from_numpy(np.ascontiguousarray(a[1, :, 2])) for a in (q, k, v))
+    want = F.scaled_dot_product_attention(qh, kh, vh, attn_mask=torch.from_numpy(allowed), scale=scale).numpy()
+    got = O.masked_dense_attention(q[1, :, 2], k[1, :, 2], v[1, :, 2], allowed, scale)
+    assert np.max(np.abs(got - want)) <= 1e-12
+
+
+def test_dense_attention_matches_torch():
+    pin_dense_attention_matches_torch()
+
+
+def test_exhaustive_topk_hand_cases():
+    # the best k-subset by score sum, worked by hand; equal sums go to the lower indices
+    assert O.exhaustive_topk(np.array([1.0, 3.0, 2.0, 3.0]), 2).tolist() == [1, 3]
+    assert O.exhaustive_topk(np.array([2.0, 2.0, 2.0]), 2).tolist() == [0, 1]
+    assert O.exhaustive_topk(np.array([2.0, 1.0, 2.0]), 1).tolist() == [0]
+    assert O.exhaustive_topk(np.array([-1.0, -5.0, 0.5, 0.5]), 3).tolist() == [0, 2, 3]
+    assert O.exhaustive_topk(np.array([0.0, 4.0, 1.0, 3.0, 2.0]), 5).tolist() == [0, 1, 2, 3, 4]
+
+
+def test_mutation_dense_softmax_over_queries(monkeypatch):
+    def bad(q, k, v, scale):                 # weights normalised down each key's column
+        out = np.empty_like(q)
+        for b in range(q.shape[0]):
+            for h in range(q.shape[2]):
+                x = scale * (q[b, :, h] @ k[b, :, h].T)
+                p = np.exp(x - x.max(axis=0, keepdims=True))
+                out[b, :, h] = (p / p.sum(axis=0, keepdims=True)) @ v[b, :, h]
+        return out
+    monkeypatch.setattr(O, "dense_attention", bad)
+    _expect_pin_failure(pin_dense_attention_matches_torch)
